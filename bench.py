@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Benchmark of the fused per-token DiT hot path on B200.
+
+One step = one pass of all three kernels over one batch of the 5 s
+1344x768 clip shape (126,552 tokens: 31x48x84 video latent patches + 1,560
+audio tokens, D = 5120 = 40 heads x 128, bf16):
+  RMS-AdaLN (x -> y), QKNorm + 3D RoPE (merged qkv -> q, k), gated residual
+  (h, branch -> out).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 is launched by torchrun (one process per GPU); each rank processes its
+own clip (weak scaling, no data exchange), the timed region is bracketed by
+barriers and the time is the max over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only other implementation
+of these operations) on the host cores, one bounded sample of clip rows per
+step; under torchrun only rank 0 runs it.
+"""
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from video_diffusion_transformer_rms_b200 import dist  # noqa: E402
+from video_diffusion_transformer_rms_b200.workloads import (WORKLOADS, activation,  # noqa: E402
+                                                            make_inputs, to_oracle_array,
+                                                            vectors)
+
+METRIC = "tokens/s and achieved HBM GB/s (% of B200 peak) per fused kernel, 1 GPU"
+WORKLOAD = "clip5s"
+KERNELS = ("rms_adaln", "qknorm_rope3d", "gate_residual")
+KERNEL_SOURCES = {
+    "rms_adaln": ["rms_adaln.cu", "sol_device.cuh"],
+    "gate_residual": ["gate_residual.cu", "sol_device.cuh"],
+    "qknorm_rope3d": ["qknorm_rope3d.cu", "sol_device.cuh"],
+}
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+ORACLE_SECONDS_PER_ROW = 0.4e-3  # all three oracle ops on one clip row (estimate)
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="oracle time budget of the CPU baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_config(w, n_gpus):
+    return {
+        "workload": (f"{w.name}: 5 s 1344x768 24 fps clip shape, B={w.B}, latent grid "
+                     f"T={w.T} H={w.H} W={w.W} ({w.n_video} video tokens) + {w.n_audio} audio "
+                     f"tokens = {w.L} tokens per sample, D={w.D} ({w.n_heads}x{w.head_dim} "
+                     f"heads), merged QKV [{w.L}, {3 * w.D}], RoPE sections "
+                     f"{'/'.join(map(str, w.sections))}, theta {w.theta:g}, eps {w.eps:g}"),
+        "tokens_per_gpu": w.rows,
+        "global_tokens_per_step": w.rows * n_gpus,
+        "D": w.D,
+        "io_dtype": w.dtype,
+        "step": "rms_adaln + qknorm_rope3d + gate_residual, one launch each",
+        "l2": "no flush: every input is larger than the 126 MB L2 (1.3-3.9 GB per tensor)",
+        "parallelism": f"{n_gpus} independent shards (one clip per GPU), no data-path collective",
+        "inputs": "seeded synthetic N(0,1) activations with 1% outlier channels x20",
+    }
+
+
+# ----------------------------------------------------------------------------
+# peaks, clocks, ncu traffic record
+# ----------------------------------------------------------------------------
+
+def load_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha(kernel):
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "video_diffusion_transformer_rms_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def traffic_record(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, or None if there
+    is none or the kernel source changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    s = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    if not m or not s or s.group(1) != kernel_source_sha(kernel):
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
+    FIELDS = ("timestamp,index,uuid,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.uuid = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            pass
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "200"]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.5)
+
+    def mark(self):
+        return time.time()
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "note": "nvidia-smi unavailable"}
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = []
+        for line in self.file.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            uuid = parts[2]
+            if self.uuid and self.uuid not in uuid and uuid not in f"GPU-{self.uuid}":
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                rows.append((ts, float(parts[3]), float(parts[4]), parts[6:10]))
+            except ValueError:
+                continue
+        os.unlink(self.file.name)
+        inside = [r for r in rows if t0 - 1 <= r[0] <= t1 + 1] or rows
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "no samples"}
+        reasons = sorted({name for r in inside for name, v in zip(self.REASONS, r[3])
+                          if v.strip().lower() == "active"})
+        return {"sm_mhz": float(np.median([r[1] for r in inside])),
+                "sm_max_mhz": float(max(r[2] for r in inside)), "reasons": reasons,
+                "samples": len(inside)}
+
+
+# ----------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of clip rows
+# ----------------------------------------------------------------------------
+
+def oracle_sample_run(w, n_rows, seed, timer):
+    """Run the three oracle ops on n_rows rows of the workload spread over the
+    sequence (video and audio); returns oracle seconds (inputs drawn outside
+    the timed part)."""
+    import oracle
+    ids = np.linspace(0, w.rows - 1, n_rows).round().astype(np.int64)
+    bf = w.torch_dtype
+    x = to_oracle_array(activation(n_rows, w.D, bf, "cpu", seed, w.outliers))
+    h = to_oracle_array(activation(n_rows, w.D, bf, "cpu", seed + 1, w.outliers))
+    br = to_oracle_array(activation(n_rows, w.D, bf, "cpu", seed + 2, w.outliers))
+    qk = to_oracle_array(activation(n_rows, 2 * w.D, bf, "cpu", seed + 3, w.outliers))
+    mod = to_oracle_array(vectors((w.B, 2, w.D), 0.0, 0.5, bf, "cpu", seed + 4))
+    gq = to_oracle_array(vectors((w.head_dim,), 1.0, 0.1, bf, "cpu", seed + 5))
+    t0 = timer()
+    oracle.rms_adaln(x, mod, mod, w.L, w.n_video, w.eps, row_ids=ids)
+    oracle.qknorm_rope3d(qk, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections,
+                         w.eps, w.theta, gamma_q=gq, gamma_k=gq, row_ids=ids)
+    oracle.gate_residual(h, br, mod, w.L, w.n_video, row_ids=ids)
+    return timer() - t0
+
+
+def cpu_baseline(w, budget_s):
+    done, spent, chunk, seed = 0, 0.0, 256, 900_000
+    while spent < budget_s:
+        spent += oracle_sample_run(w, chunk, seed, time.perf_counter)
+        done += chunk
+        seed += 10
+    return {"value": done / spent, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": (f"{done} rows of the {w.name} workload spread over video and audio, "
+                       f"all three ops, fp64 oracle, single thread, {spent:.1f} s")}
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def run_ours(args):
+    from video_diffusion_transformer_rms_b200 import _abi, api
+    from video_diffusion_transformer_rms_b200 import build as libbuild
+
+    rank, local_rank, world = dist.init("nccl", timeout_s=300.0)
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if rank == 0:
+        libbuild.build()
+    dist.barrier()
+    _abi.lib()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[WORKLOAD]
+    D = w.D
+
+    t = make_inputs(w, dev)
+    x = t["x"].view(w.B, w.L, D)
+    h = t["h"].view(w.B, w.L, D)
+    br = t["branch"].view(w.B, w.L, D)
+    qkv = t["qkv"].view(w.B, w.L, 3 * D)
+    y = torch.empty_like(x)
+    out = torch.empty_like(h)
+    qk = torch.empty((w.B, w.L, 2 * D), dtype=qkv.dtype, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    s = stream.cuda_stream
+    dt = _abi.SOL_BF16
+    st, sh_, sw = w.sections
+    p = {k: v.data_ptr() for k, v in t.items()}
+    ld_out = 2 * D
+
+    def k_rms():
+        return _abi.sol_rms_adaln(p["x"], y.data_ptr(), p["scale"], p["shift"], None, w.B, w.L,
+                                  w.n_video, D, w.eps, dt, s)
+
+    def k_qk():
+        return _abi.sol_qknorm_rope3d(p["qkv"], 3 * D, qk.data_ptr(), qk.data_ptr() + D * 2,
+                                      ld_out, p["gamma_q"], p["gamma_k"], w.B, w.T, w.H, w.W,
+                                      w.n_audio, w.n_heads, w.head_dim, st, sh_, sw, w.eps,
+                                      w.theta, dt, s)
+
+    def k_gate():
+        return _abi.sol_gate_residual(p["h"], p["branch"], p["gate"], out.data_ptr(), w.B, w.L,
+                                      w.n_video, D, dt, s)
+
+    launch = {"rms_adaln": k_rms, "qknorm_rope3d": k_qk, "gate_residual": k_gate}
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        for i, name in enumerate(KERNELS):
+            _abi.check(launch[name]())
+            if ev is not None:
+                ev[i + 1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(KERNELS) + 1)]
+           for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    dist.barrier()
+    torch.cuda.synchronize()
+    t0 = clocks.mark()
+    start.record(stream)
+    for i in range(K):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    t1 = clocks.mark()
+    dist.barrier()
+    clock_info = clocks.stop(t0, t1)
+    elapsed_s = start.elapsed_time(end) / 1e3
+    per_kernel_ms = {name: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / K
+                     for i, name in enumerate(KERNELS)}
+
+    value, total_units, slowest = dist.job_throughput(w.rows * K, elapsed_s)
+    per_kernel_ms = {k: dist.max_over_ranks(v) for k, v in per_kernel_ms.items()}
+
+    # ---- end to end through the public API, host buffers ------------------
+    e2e = run_e2e(args, w, t, stream, api)
+    e2e_value, _, _ = dist.job_throughput(w.rows * e2e["steps"], e2e["seconds"])
+
+    peak, peak_kind = load_peak()
+    bpr = w.bytes_per_row()
+    kernels = {}
+    for name in KERNELS:
+        ms = per_kernel_ms[name]
+        gbs = bpr[name] * w.rows / (ms / 1e3) / 1e9
+        kernels[name] = {"ms": round(ms, 4), "tokens_per_s": round(w.rows / (ms / 1e3)),
+                         "bytes_per_token": bpr[name], "GB_per_s": round(gbs, 1),
+                         f"frac_of_{peak_kind}_hbm": round(gbs / peak, 4),
+                         "frac_of_8TBs_nominal": round(gbs / NOMINAL_HBM_GBS, 4)}
+    dominant = max(KERNELS, key=lambda k: per_kernel_ms[k])
+    traffic = traffic_record(dominant, WORKLOAD)
+    roofline = {"kernel": dominant, "bound": "hbm",
+                "achieved": kernels[dominant]["GB_per_s"], "peak": peak, "unit": "GB/s",
+                "frac": round(kernels[dominant]["GB_per_s"] / peak, 4),
+                "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "traffic": traffic,
+                "algorithmic_bytes_per_launch": bpr[dominant] * w.rows}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
+            "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": round(slowest * 1e3 / K, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; no dataset or weights involved)",
+            "config": workload_config(w, world),
+            "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                    "steps": e2e["steps"],
+                    "path": "pinned host inputs -> H2D -> api.rms_adaln / api.qknorm_rope3d / "
+                            "api.gate_residual -> D2H of y, q, k, out; CUDA events"},
+            "gpu_launches": len(KERNELS) * K,
+            "clocks": clock_info,
+        }
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.shutdown()
+
+
+def run_e2e(args, w, t, stream, api):
+    """Same step through the public tensor API, inputs copied every step
+    from pinned host memory and every output copied back."""
+    D = w.D
+    names = ("x", "scale", "shift", "qkv", "gamma_q", "gamma_k", "h", "branch", "gate")
+    host = {n: torch.empty(t[n].shape, dtype=t[n].dtype, pin_memory=True) for n in names}
+    for n in names:
+        host[n].copy_(t[n])
+    dev = {n: torch.empty_like(t[n]) for n in names}
+    y = torch.empty((w.B, w.L, D), dtype=t["x"].dtype, device=t["x"].device)
+    qk = torch.empty((w.B, w.L, 2 * D), dtype=t["x"].dtype, device=t["x"].device)
+    out = torch.empty_like(y)
+    host_out = {"y": torch.empty(y.shape, dtype=y.dtype, pin_memory=True),
+                "qk": torch.empty(qk.shape, dtype=qk.dtype, pin_memory=True),
+                "out": torch.empty(out.shape, dtype=out.dtype, pin_memory=True)}
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+
+    def step():
+        for n in names:
+            dev[n].copy_(host[n], non_blocking=True)
+        api.rms_adaln(dev["x"].view(w.B, w.L, D), dev["scale"], dev["shift"], w.n_video,
+                      eps=w.eps, out=y)
+        api.qknorm_rope3d(dev["qkv"].view(w.B, w.L, 3 * D), w.T, w.H, w.W, w.n_audio,
+                          w.n_heads, w.head_dim, w.sections, dev["gamma_q"], dev["gamma_k"],
+                          w.eps, w.theta, q_out=qk[..., :D], k_out=qk[..., D:])
+        api.gate_residual(dev["h"].view(w.B, w.L, D), dev["branch"].view(w.B, w.L, D),
+                          dev["gate"], w.n_video, out=out)
+        host_out["y"].copy_(y, non_blocking=True)
+        host_out["qk"].copy_(qk, non_blocking=True)
+        host_out["out"].copy_(out, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    n = max(1, args.e2e_steps)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    secs = a.elapsed_time(b) / 1e3
+    del host, host_out, dev
+    return {"seconds": secs, "steps": n, "h2d": h2d, "d2h": d2h}
+
+
+# ----------------------------------------------------------------------------
+# reference arm: the oracle on the host cores
+# ----------------------------------------------------------------------------
+
+def run_reference(args):
+    rank, _, world = dist.env_world()
+    if rank != 0:
+        return  # only rank 0 times the CPU reference
+    w = WORKLOADS[WORKLOAD]
+    total_steps = args.steps + args.warmup
+    rows = int(90.0 / max(1, total_steps) / ORACLE_SECONDS_PER_ROW)
+    rows = max(8, min(2048, rows))
+    spent, done = 0.0, 0
+    for i in range(total_steps):
+        secs = oracle_sample_run(w, rows, 700_000 + 10 * i, time.perf_counter)
+        if i >= args.warmup:
+            spent += secs
+            done += rows
+    value = done / spent
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(spent * 1e3 / max(1, args.steps), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, 1),
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": 1,
+                         "kind": "oracle",
+                         "sample": f"{rows} rows of {w.name} per step, all three ops, fp64 "
+                                   f"oracle, single thread"},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,177 @@
+/*
+ * sol.h - C ABI of libsol, the fused per-token hot path of a joint
+ * video+audio diffusion-transformer block on NVIDIA B200 (sm_100a).
+ *
+ * Three operations, each one kernel launch:
+ *   sol_rms_adaln      RMSNorm then AdaLN modulation  x^ * (1 + scale) + shift
+ *   sol_gate_residual  AdaLN-gated residual add        h + gate * branch
+ *   sol_qknorm_rope3d  per-head RMS norm of q and k, then 3D multimodal RoPE
+ *
+ * The fusions are the ones the Sol Video Inference Engine MiniMax-H3
+ * on-device page lists in its fusion table ("fused RMS-AdaLN": no HBM
+ * round-trips across the modulation branch; "fused QKNorm + RoPE": no
+ * separate read/write passes over Q and K, no separate 3D MM-RoPE indexing);
+ * the KOCPC Sol-H3 article repeats them in "Technical Composition".  The
+ * gated residual is the "leftover elementwise chain" of the same page's
+ * torch.compile row, the adaLN gate of the DiT block.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Token rows.  A batch holds B samples of L rows each, row-major and
+ * contiguous: row r of sample b is global row b*L + r.  In every sample the
+ * first n_video rows are video latent patches (raster order, t-major, for
+ * sol_qknorm_rope3d n_video = T*H*W) and the remaining L - n_video rows are
+ * audio tokens (the joint single-stream sequence of the H3-Omni transformer).
+ * Row r is "video" (modality 0) if r < n_video, else "audio" (modality 1).
+ *
+ * Modulation vectors.  scale, shift and gate are [B, 2, D] arrays: index
+ * [b][0] holds sample b's video vector and [b][1] its audio vector.
+ *
+ * Element type.  All tensor arguments of one call have the same type:
+ * SOL_BF16 (bfloat16) or SOL_F32.  Arithmetic is fp32 inside the kernels;
+ * outputs are rounded once, to nearest even.
+ *
+ * Memory.  Every tensor pointer is a DEVICE pointer (cudaMalloc'd, managed,
+ * or mapped so the GPU can read it) on the current device, 16-byte aligned,
+ * with every row start 16-byte aligned (so D, and the row strides, must be
+ * multiples of 8 elements for bf16 and 4 for fp32).  The caller owns all
+ * buffers.  The library allocates nothing, keeps no per-call state and may be
+ * called from several host threads at once.
+ *
+ * Aliasing.  An output may be exactly its input (in place) as stated per
+ * call; any other overlap between an output and another argument is rejected
+ * with SOL_ERR_INVALID_ARG.
+ *
+ * Streams and errors.  Each call validates its arguments on the host, then
+ * enqueues one kernel on `stream` (NULL = the legacy default stream) and
+ * returns without synchronising.  On any non-OK status nothing has been
+ * enqueued, except SOL_ERR_CUDA, which reports a failed launch (the CUDA
+ * error was read and cleared with cudaGetLastError).  A call with zero rows
+ * is a no-op that returns SOL_OK.  sol_last_error() gives a one-line reason
+ * for the calling thread's last non-OK status.
+ */
+#ifndef SOL_H
+#define SOL_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t is `struct CUstream_st *` */
+typedef struct CUstream_st *sol_stream_t;
+
+typedef enum sol_status {
+    SOL_OK = 0,
+    SOL_ERR_INVALID_ARG = 1, /* null pointer, bad size, or forbidden overlap */
+    SOL_ERR_MISALIGNED = 2,  /* a pointer or row start not 16-byte aligned */
+    SOL_ERR_UNSUPPORTED = 3, /* valid but outside the built kernels' limits */
+    SOL_ERR_CUDA = 4         /* the CUDA runtime reported an error */
+} sol_status;
+
+typedef enum sol_dtype {
+    SOL_F32 = 0,
+    SOL_BF16 = 1
+} sol_dtype;
+
+/*
+ * Fused RMS-AdaLN (fusion table of the Sol Video Inference Engine MiniMax-H3
+ * page, row "fused RMS-AdaLN"; RMSNorm of Zhang & Sennrich, adaLN modulation
+ * of the DiT block).  For every row of sample b with modality m:
+ *
+ *   y[c] = x[c] / sqrt(mean_c(x^2) + eps) * gamma[c] * (1 + scale[b][m][c])
+ *          + shift[b][m][c]
+ *
+ *   x, y          [B, L, D] device, contiguous.  y may equal x (in place).
+ *   scale, shift  [B, 2, D] device.
+ *   gamma         [D] device, or NULL for a weight of 1 (the adaLN norm of a
+ *                 DiT block has no learnable weight; the option is kept).
+ *   n_video       0 <= n_video <= L.
+ *   D             > 0; at most 16384 (bf16) / 8192 (fp32)
+ *                 (SOL_ERR_UNSUPPORTED beyond).
+ *   eps           >= 0, added inside the square root (1e-6 in the model).
+ */
+sol_status sol_rms_adaln(const void *x, void *y, const void *scale,
+                         const void *shift, const void *gamma, int64_t B,
+                         int64_t L, int64_t n_video, int64_t D, float eps,
+                         sol_dtype dtype, sol_stream_t stream);
+
+/*
+ * AdaLN-gated residual add (the adaLN gate of the DiT block; the residual
+ * update the Sol pages fold under "leftover elementwise chains").  For every
+ * row of sample b with modality m:
+ *
+ *   out[c] = h[c] + gate[b][m][c] * branch[c]
+ *
+ *   h, branch, out [B, L, D] device, contiguous.  out may equal h or branch.
+ *   gate           [B, 2, D] device.
+ *   n_video, D     as for sol_rms_adaln (same D limit).
+ */
+sol_status sol_gate_residual(const void *h, const void *branch,
+                             const void *gate, void *out, int64_t B, int64_t L,
+                             int64_t n_video, int64_t D, sol_dtype dtype,
+                             sol_stream_t stream);
+
+/*
+ * Fused per-head QKNorm + 3D multimodal RoPE on a merged QKV projection
+ * (fusion table of the Sol Video Inference Engine MiniMax-H3 page, rows
+ * "fused QKNorm + RoPE" and "QKV merge"; RoPE of Su et al., RoFormer).
+ *
+ * Each row holds q in columns [0, D), k in [D, 2D) (v, if present after
+ * them, is neither read nor written), D = n_heads * head_dim; head j of q or
+ * k is columns [j*head_dim, (j+1)*head_dim) of that part.  For each head:
+ *
+ *   n[c]  = x[c] / sqrt(mean_c(x^2) + eps) * gamma_P[c]   (P = q or k)
+ *   pair i = (n[2i], n[2i+1]), i < head_dim/2, rotated by
+ *   phi_i = pos_a(i) * theta^(-2i/head_dim):
+ *     out[2i]   = n[2i] cos(phi_i) - n[2i+1] sin(phi_i)
+ *     out[2i+1] = n[2i] sin(phi_i) + n[2i+1] cos(phi_i)
+ *   with a(i) = t for i < sec_t, h for i < sec_t + sec_h, else w.
+ *
+ * Positions (per sample, the same for every sample): video row r < T*H*W
+ * has (t, h, w) = (r / (H*W), (r / W) mod H, r mod W); audio row
+ * i = r - T*H*W has (i, 0, 0).  So L = T*H*W + n_audio.
+ *
+ *   qkv          device; row g (= b*L + r) starts at qkv + g*ld_qkv elements;
+ *                ld_qkv >= 2*D (3*D for a packed [.., 3D] projection).
+ *   q_out, k_out device; row g of q (k) goes to q_out (k_out) + g*ld_out.
+ *                ld_out >= D.  In place: q_out == qkv, k_out == qkv + D and
+ *                ld_out == ld_qkv.  Otherwise q_out and k_out must not
+ *                overlap qkv's rows nor each other (q_out = buf,
+ *                k_out = buf + D, ld_out = 2*D is fine).
+ *   gamma_q, gamma_k [head_dim] device, or NULL for a weight of 1; one
+ *                vector for all heads.
+ *   head_dim     even, head_dim / (8 for bf16, 4 for fp32) a power of two
+ *                in [2, 32] (so 16..256 bf16, 8..128 fp32), else
+ *                SOL_ERR_UNSUPPORTED; sec_t + sec_h + sec_w == head_dim / 2.
+ *   n_heads      > 0, with D at most 16384 (bf16) / 8192 (fp32)
+ *                (SOL_ERR_UNSUPPORTED beyond).
+ *   eps >= 0; theta > 0 (10000 in the model).
+ *   T, H, W, n_audio >= 0, B >= 0.
+ */
+sol_status sol_qknorm_rope3d(const void *qkv, int64_t ld_qkv, void *q_out,
+                             void *k_out, int64_t ld_out, const void *gamma_q,
+                             const void *gamma_k, int64_t B, int64_t T,
+                             int64_t H, int64_t W, int64_t n_audio,
+                             int64_t n_heads, int64_t head_dim, int64_t sec_t,
+                             int64_t sec_h, int64_t sec_w, float eps,
+                             float theta, sol_dtype dtype,
+                             sol_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char *sol_status_string(sol_status status);
+
+/* One-line reason for the calling thread's most recent non-OK status, or ""
+ * if its last call succeeded.  The pointer stays valid until the thread's
+ * next libsol call. */
+const char *sol_last_error(void);
+
+/* ABI version, (major << 16) | minor. */
+int sol_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SOL_H */

@@ -1,0 +1,150 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/sol.h declares, and rejects bad arguments before any
+CUDA call (fake, never-dereferenced addresses are enough for that)."""
+import ctypes
+import subprocess
+
+import pytest
+
+from video_diffusion_transformer_rms_b200 import _abi
+from video_diffusion_transformer_rms_b200.build import LIB, build
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build()
+
+
+def test_header_declares_the_entry_points():
+    syms = _abi.header_symbols()
+    for name in ("sol_rms_adaln", "sol_gate_residual", "sol_qknorm_rope3d",
+                 "sol_status_string", "sol_last_error", "sol_version"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _abi.lib()
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in _abi.header_symbols():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_status_strings_and_version():
+    assert _abi.status_string(_abi.SOL_OK) == "SOL_OK"
+    assert _abi.status_string(_abi.SOL_ERR_MISALIGNED) == "SOL_ERR_MISALIGNED"
+    assert _abi.status_string(99) == "SOL_ERR_UNKNOWN"
+    assert _abi.sol_version() >> 16 == 1
+
+
+# Fake device addresses: validation must reject these calls on the host.
+A = 0x7F0000000000
+BF = _abi.SOL_BF16
+F32 = _abi.SOL_F32
+
+
+def rms(x=A, y=A + (1 << 30), sc=A + (2 << 30), sh=A + (3 << 30), g=None, B=1, L=4,
+        nv=2, D=64, eps=1e-6, dt=BF):
+    return _abi.sol_rms_adaln(x, y, sc, sh, g, B, L, nv, D, eps, dt, None)
+
+
+def gate(h=A, br=A + (1 << 30), g=A + (2 << 30), out=A + (3 << 30), B=1, L=4, nv=2, D=64,
+         dt=BF):
+    return _abi.sol_gate_residual(h, br, g, out, B, L, nv, D, dt, None)
+
+
+def qk(qkv=A, ldq=768, qo=A + (1 << 30), ko=A + (2 << 30), ldo=256, gq=None, gk=None, B=1,
+       T=2, H=4, W=6, na=8, nh=2, hd=128, secs=(16, 24, 24), eps=1e-6, theta=1e4, dt=BF):
+    return _abi.sol_qknorm_rope3d(qkv, ldq, qo, ko, ldo, gq, gk, B, T, H, W, na, nh, hd,
+                                  *secs, eps, theta, dt, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), _abi.SOL_ERR_INVALID_ARG),
+    (dict(nv=5), _abi.SOL_ERR_INVALID_ARG),
+    (dict(D=0), _abi.SOL_ERR_INVALID_ARG),
+    (dict(eps=-1.0), _abi.SOL_ERR_INVALID_ARG),
+    (dict(eps=float("nan")), _abi.SOL_ERR_INVALID_ARG),
+    (dict(dt=7), _abi.SOL_ERR_INVALID_ARG),
+    (dict(D=60), _abi.SOL_ERR_MISALIGNED),           # 120 bytes per row
+    (dict(D=62, dt=F32), _abi.SOL_ERR_MISALIGNED),
+    (dict(x=A + 8), _abi.SOL_ERR_MISALIGNED),
+    (dict(g=A + (4 << 30) + 4), _abi.SOL_ERR_MISALIGNED),
+    (dict(D=16392), _abi.SOL_ERR_UNSUPPORTED),
+    (dict(D=8196, dt=F32), _abi.SOL_ERR_UNSUPPORTED),
+    (dict(y=A + 16), _abi.SOL_ERR_INVALID_ARG),      # partial overlap with x
+    (dict(y=A + (2 << 30) + 64), _abi.SOL_ERR_INVALID_ARG),  # overlaps scale
+])
+def test_rms_adaln_rejects(kw, status):
+    assert rms(**kw) == status
+    assert _abi.last_error() != ""
+
+
+def test_zero_rows_is_a_noop_even_with_null_pointers():
+    assert rms(x=None, y=None, B=0) == _abi.SOL_OK
+    assert rms(x=None, y=None, L=0, nv=0) == _abi.SOL_OK
+    assert gate(h=None, B=0) == _abi.SOL_OK
+    assert qk(qkv=None, T=0, na=0) == _abi.SOL_OK
+    assert _abi.last_error() == ""
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(out=None), _abi.SOL_ERR_INVALID_ARG),
+    (dict(nv=-1), _abi.SOL_ERR_INVALID_ARG),
+    (dict(D=20), _abi.SOL_ERR_MISALIGNED),
+    (dict(g=A + (2 << 30) + 2), _abi.SOL_ERR_MISALIGNED),
+    (dict(D=16400), _abi.SOL_ERR_UNSUPPORTED),
+    (dict(out=A + 32), _abi.SOL_ERR_INVALID_ARG),     # partial overlap with h
+    (dict(out=A + (1 << 30) - 32), _abi.SOL_ERR_INVALID_ARG),  # straddles branch
+    (dict(out=A + (2 << 30)), _abi.SOL_ERR_INVALID_ARG),  # overlaps gate
+])
+def test_gate_residual_rejects(kw, status):
+    assert gate(**kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(qkv=None), _abi.SOL_ERR_INVALID_ARG),
+    (dict(hd=127, secs=(16, 24, 23)), _abi.SOL_ERR_INVALID_ARG),
+    (dict(secs=(16, 24, 25)), _abi.SOL_ERR_INVALID_ARG),
+    (dict(secs=(-1, 33, 32)), _abi.SOL_ERR_INVALID_ARG),
+    (dict(theta=0.0), _abi.SOL_ERR_INVALID_ARG),
+    (dict(ldq=500), _abi.SOL_ERR_INVALID_ARG),       # < 2*D
+    (dict(ldo=200), _abi.SOL_ERR_INVALID_ARG),       # < D
+    (dict(hd=96, secs=(16, 16, 16)), _abi.SOL_ERR_UNSUPPORTED),   # G = 12 lanes
+    (dict(hd=8, secs=(2, 1, 1)), _abi.SOL_ERR_UNSUPPORTED),       # G = 1 lane (bf16)
+    (dict(hd=256, secs=(32, 48, 48), dt=F32, ldq=1536, ldo=512),
+     _abi.SOL_ERR_UNSUPPORTED),  # G = 64 lanes (fp32)
+    (dict(nh=130, ldq=3 * 16640, ldo=16640), _abi.SOL_ERR_UNSUPPORTED),  # D > 16384
+    (dict(ldq=772), _abi.SOL_ERR_MISALIGNED),        # 1544-byte row stride
+    (dict(qo=A + (1 << 30) + 2), _abi.SOL_ERR_MISALIGNED),
+    (dict(qo=A + 512), _abi.SOL_ERR_INVALID_ARG),    # q_out inside qkv's k columns
+    (dict(qo=A, ko=A + 1024, ldo=768), _abi.SOL_ERR_INVALID_ARG),  # half in place
+    (dict(ko=A + (1 << 30) + 256, ldo=256), _abi.SOL_ERR_INVALID_ARG),  # q_out/k_out collide
+])
+def test_qknorm_rope3d_rejects(kw, status):
+    assert qk(**kw) == status
+
+
+def test_error_message_is_thread_local_and_cleared():
+    assert rms(x=None) == _abi.SOL_ERR_INVALID_ARG
+    msg = _abi.last_error()
+    assert "non-null" in msg
+    assert rms(B=0) == _abi.SOL_OK
+    assert _abi.last_error() == ""
+
+
+def test_python_binding_raises_with_reason():
+    with pytest.raises(_abi.SolError) as ei:
+        _abi.check(rms(D=60))
+    assert ei.value.status == _abi.SOL_ERR_MISALIGNED
+    assert "multiple of 16" in str(ei.value)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(_abi, "_lib", None)
+    monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "libsol.so"))
+    with pytest.raises(ImportError):
+        _abi.lib()
+    assert isinstance(ctypes.CDLL, type)

@@ -1,0 +1,325 @@
+"""GPU parity: the CUDA kernels (called through the C ABI) against the fp64
+oracle on the same seeded inputs, element by element, within
+|gpu - oracle| <= 2 ulp(oracle value) + 1e-3.
+
+Small workloads are compared in full; the 5 s / 15 s clip shapes and the CFG
+batch are compared on a seeded sample of rows (always including each
+sample's first/last rows and its video/audio boundary) at full size, in the
+launch configuration the benchmark uses.  Edge cases: ragged widths and row
+counts, no audio / no video, in-place outputs, strided layouts, guard bytes
+around outputs, zero rows, misaligned pointers.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.parity import assert_close, sample_rows, take_rows, take_rows_gpu
+from video_diffusion_transformer_rms_b200 import _abi, api
+from video_diffusion_transformer_rms_b200.workloads import (WORKLOADS, activation,
+                                                            make_inputs, to_oracle_array,
+                                                            vectors)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+SMALL = ("tiny", "medium")
+LARGE = ("clip5s", "clip15s", "cfg5s", "cfg5s_d3072")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    _abi.lib()
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def _ids(w, n=1024):
+    return sample_rows(w.rows, w.L, w.n_video, w.B, n, seed=7 + w.index)
+
+
+def _o(t):
+    return to_oracle_array(t)
+
+
+# ----------------------------------------------------------------------------
+# RMS-AdaLN
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", SMALL + LARGE)
+@pytest.mark.parametrize("with_gamma", [False, True])
+def test_rms_adaln_workload(name, with_gamma):
+    w = WORKLOADS[name]
+    t = make_inputs(w, DEV, which=("rms_adaln",), with_gamma=with_gamma)
+    x = t["x"].view(w.B, w.L, w.D)
+    y = api.rms_adaln(x, t["scale"], t["shift"], w.n_video, gamma=t.get("gamma"), eps=w.eps)
+    torch.cuda.synchronize()
+    x2, y2 = x.view(w.rows, w.D), y.view(w.rows, w.D)
+    g = _o(t["gamma"]) if with_gamma else None
+    if name in SMALL:
+        want = oracle.rms_adaln(_o(x2), _o(t["scale"]), _o(t["shift"]), w.L, w.n_video,
+                                w.eps, gamma=g)
+        assert_close(y2, want, f"rms_adaln[{name}]")
+    else:
+        ids = _ids(w)
+        want = oracle.rms_adaln(take_rows(x2, ids), _o(t["scale"]), _o(t["shift"]), w.L,
+                                w.n_video, w.eps, gamma=g, row_ids=ids)
+        assert_close(take_rows_gpu(y2, ids), want, f"rms_adaln[{name}] sampled")
+
+
+RMS_SHAPES = [
+    # B, L, n_video, D, dtype
+    (1, 1, 1, 8, torch.bfloat16),            # one vector per row, one row
+    (3, 37, 20, 5128, torch.bfloat16),       # ragged: 641 vectors per row
+    (2, 300, 0, 4096, torch.bfloat16),       # audio only
+    (2, 300, 300, 2056, torch.bfloat16),     # video only, ragged
+    (1, 1000, 500, 256, torch.float32),
+    (1, 33, 16, 16384, torch.bfloat16),      # widest bf16 row
+    (1, 17, 5, 8192, torch.float32),         # widest fp32 row
+    (5, 1000, 900, 3072, torch.bfloat16),
+    (1, 50001, 49000, 128, torch.bfloat16),  # many more rows than CTAs
+    (1, 7, 3, 12, torch.float32),            # 3 vectors per row
+]
+
+
+def _rand_rms(B, L, D, dt, seed):
+    x = activation(B * L, D, dt, DEV, seed, outliers=True).view(B, L, D)
+    sc = vectors((B, 2, D), 0.0, 0.5, dt, DEV, seed + 1)
+    sh = vectors((B, 2, D), 0.0, 0.5, dt, DEV, seed + 2)
+    g = vectors((D,), 1.0, 0.1, dt, DEV, seed + 3)
+    return x, sc, sh, g
+
+
+@pytest.mark.parametrize("B,L,nv,D,dt", RMS_SHAPES)
+def test_rms_adaln_shapes(B, L, nv, D, dt):
+    x, sc, sh, g = _rand_rms(B, L, D, dt, seed=D + L)
+    for gamma in (None, g):
+        y = api.rms_adaln(x, sc, sh, nv, gamma=gamma, eps=1e-6)
+        want = oracle.rms_adaln(_o(x.view(-1, D)), _o(sc), _o(sh), L, nv, 1e-6,
+                                gamma=None if gamma is None else _o(g))
+        assert_close(y.view(-1, D), want, f"rms_adaln B={B} L={L} D={D}")
+
+
+def test_rms_adaln_in_place_and_guards():
+    B, L, nv, D = 2, 777, 700, 5120
+    x, sc, sh, _ = _rand_rms(B, L, D, torch.bfloat16, seed=3)
+    want = oracle.rms_adaln(_o(x.view(-1, D)), _o(sc), _o(sh), L, nv, 1e-6)
+    # in place
+    xi = x.clone()
+    api.rms_adaln(xi, sc, sh, nv, out=xi)
+    assert_close(xi.view(-1, D), want, "rms_adaln in place")
+    # output inside a guarded buffer: the 4 KB on each side must stay intact
+    pad = 2048
+    buf = torch.full((B * L * D + 2 * pad,), 7.0, dtype=torch.bfloat16, device=DEV)
+    y = buf[pad:pad + B * L * D].view(B, L, D)
+    api.rms_adaln(x, sc, sh, nv, out=y)
+    torch.cuda.synchronize()
+    assert torch.all(buf[:pad] == 7.0) and torch.all(buf[-pad:] == 7.0)
+    assert_close(y.view(-1, D), want, "rms_adaln guarded")
+
+
+def test_rms_adaln_zero_rows_touch_nothing():
+    D = 256
+    x = torch.zeros((0, 5, D), dtype=torch.bfloat16, device=DEV)
+    y = torch.full((1, 5, D), 3.0, dtype=torch.bfloat16, device=DEV)
+    sc = torch.zeros((1, 2, D), dtype=torch.bfloat16, device=DEV)
+    st = _abi.sol_rms_adaln(x.data_ptr(), y.data_ptr(), sc.data_ptr(), sc.data_ptr(), None,
+                            0, 5, 2, D, 1e-6, _abi.SOL_BF16, None)
+    assert st == _abi.SOL_OK
+    torch.cuda.synchronize()
+    assert torch.all(y == 3.0)
+
+
+def test_rms_adaln_misaligned_is_rejected_without_writing():
+    D = 64
+    x = torch.randn((1, 4, D), device=DEV).to(torch.bfloat16)
+    y = torch.full((4 * D + 8,), 5.0, dtype=torch.bfloat16, device=DEV)
+    sc = torch.zeros((1, 2, D), dtype=torch.bfloat16, device=DEV)
+    st = _abi.sol_rms_adaln(x.data_ptr(), y.data_ptr() + 2, sc.data_ptr(), sc.data_ptr(), None,
+                            1, 4, 2, D, 1e-6, _abi.SOL_BF16, None)
+    assert st == _abi.SOL_ERR_MISALIGNED
+    torch.cuda.synchronize()
+    assert torch.all(y == 5.0)
+
+
+def test_rms_adaln_is_deterministic():
+    w = WORKLOADS["medium"]
+    t = make_inputs(w, DEV, which=("rms_adaln",))
+    x = t["x"].view(w.B, w.L, w.D)
+    y1 = api.rms_adaln(x, t["scale"], t["shift"], w.n_video)
+    y2 = api.rms_adaln(x, t["scale"], t["shift"], w.n_video)
+    assert torch.equal(y1, y2)
+
+
+# ----------------------------------------------------------------------------
+# Gated residual
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", SMALL + LARGE)
+def test_gate_residual_workload(name):
+    w = WORKLOADS[name]
+    t = make_inputs(w, DEV, which=("gate_residual",))
+    h, br = t["h"].view(w.B, w.L, w.D), t["branch"].view(w.B, w.L, w.D)
+    out = api.gate_residual(h, br, t["gate"], w.n_video)
+    torch.cuda.synchronize()
+    h2, b2, o2 = h.view(-1, w.D), br.view(-1, w.D), out.view(-1, w.D)
+    if name in SMALL:
+        want = oracle.gate_residual(_o(h2), _o(b2), _o(t["gate"]), w.L, w.n_video)
+        assert_close(o2, want, f"gate_residual[{name}]")
+    else:
+        ids = _ids(w)
+        want = oracle.gate_residual(take_rows(h2, ids), take_rows(b2, ids), _o(t["gate"]),
+                                    w.L, w.n_video, row_ids=ids)
+        assert_close(take_rows_gpu(o2, ids), want, f"gate_residual[{name}] sampled")
+
+
+@pytest.mark.parametrize("B,L,nv,D,dt", RMS_SHAPES)
+def test_gate_residual_shapes(B, L, nv, D, dt):
+    h = activation(B * L, D, dt, DEV, 11, outliers=True).view(B, L, D)
+    br = activation(B * L, D, dt, DEV, 12, outliers=True).view(B, L, D)
+    g = vectors((B, 2, D), 0.0, 0.1, dt, DEV, 13)
+    out = api.gate_residual(h, br, g, nv)
+    want = oracle.gate_residual(_o(h.view(-1, D)), _o(br.view(-1, D)), _o(g), L, nv)
+    assert_close(out.view(-1, D), want, f"gate_residual B={B} L={L} D={D}")
+
+
+def test_gate_residual_in_place_zero_gate_and_guards():
+    B, L, nv, D = 2, 513, 500, 3072
+    dt = torch.bfloat16
+    h = activation(B * L, D, dt, DEV, 21, outliers=True).view(B, L, D)
+    br = activation(B * L, D, dt, DEV, 22, outliers=True).view(B, L, D)
+    g = vectors((B, 2, D), 0.0, 0.1, dt, DEV, 23)
+    want = oracle.gate_residual(_o(h.view(-1, D)), _o(br.view(-1, D)), _o(g), L, nv)
+    for which in ("h", "branch"):
+        hi, bi = h.clone(), br.clone()
+        api.gate_residual(hi, bi, g, nv, out=hi if which == "h" else bi)
+        assert_close((hi if which == "h" else bi).view(-1, D), want, f"in place on {which}")
+    # gate = 0 returns h bit for bit
+    z = torch.zeros_like(g)
+    assert torch.equal(api.gate_residual(h, br, z, nv), h)
+    pad = 4096
+    buf = torch.full((B * L * D + 2 * pad,), -9.0, dtype=dt, device=DEV)
+    o = buf[pad:pad + B * L * D].view(B, L, D)
+    api.gate_residual(h, br, g, nv, out=o)
+    torch.cuda.synchronize()
+    assert torch.all(buf[:pad] == -9.0) and torch.all(buf[-pad:] == -9.0)
+    assert_close(o.view(-1, D), want, "gate_residual guarded")
+
+
+# ----------------------------------------------------------------------------
+# QKNorm + 3D RoPE
+# ----------------------------------------------------------------------------
+
+def _qk_oracle(qkv2, w_like, gq, gk, ids=None):
+    T, H, W, na, nh, hd, secs, eps, theta = w_like
+    return oracle.qknorm_rope3d(qkv2, T, H, W, na, nh, hd, secs, eps, theta,
+                                gamma_q=gq, gamma_k=gk, row_ids=ids)
+
+
+@pytest.mark.parametrize("name", SMALL + LARGE)
+def test_qknorm_rope3d_workload(name):
+    w = WORKLOADS[name]
+    t = make_inputs(w, DEV, which=("qknorm_rope3d",))
+    qkv = t["qkv"].view(w.B, w.L, 3 * w.D)
+    q, k = api.qknorm_rope3d(qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim,
+                             w.sections, t["gamma_q"], t["gamma_k"], w.eps, w.theta)
+    torch.cuda.synchronize()
+    spec = (w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections, w.eps, w.theta)
+    q2, k2 = q.reshape(-1, w.D), k.reshape(-1, w.D)
+    qkv2 = qkv.view(-1, 3 * w.D)
+    gq, gk = _o(t["gamma_q"]), _o(t["gamma_k"])
+    if name in SMALL:
+        wq, wk = _qk_oracle(_o(qkv2), spec, gq, gk)
+        assert_close(q2, wq, f"q[{name}]")
+        assert_close(k2, wk, f"k[{name}]")
+    else:
+        ids = _ids(w, 512)
+        wq, wk = _qk_oracle(take_rows(qkv2[:, :2 * w.D], ids), spec, gq, gk, ids)
+        assert_close(take_rows_gpu(q2, ids), wq, f"q[{name}] sampled")
+        assert_close(take_rows_gpu(k2, ids), wk, f"k[{name}] sampled")
+
+
+QK_CASES = [
+    # B, T, H, W, n_audio, n_heads, head_dim, sections, dtype, pad
+    (1, 2, 4, 6, 8, 2, 128, (16, 24, 24), torch.float32, 0),
+    (1, 2, 4, 6, 8, 3, 64, (8, 12, 12), torch.float32, 4),       # G = 16 lanes
+    (2, 3, 5, 7, 11, 5, 64, (8, 12, 12), torch.bfloat16, 8),     # G = 8, padded rows
+    (1, 2, 3, 4, 5, 3, 256, (32, 48, 48), torch.bfloat16, 0),    # G = 32
+    (1, 2, 2, 2, 3, 4, 32, (4, 6, 6), torch.bfloat16, 0),        # G = 4
+    (1, 1, 2, 2, 1, 2, 16, (2, 3, 3), torch.bfloat16, 0),        # G = 2
+    (3, 1, 1, 1, 0, 40, 128, (16, 24, 24), torch.bfloat16, 0),   # one video row, no audio
+    (2, 0, 0, 0, 300, 8, 128, (16, 24, 24), torch.bfloat16, 0),  # audio only
+    (1, 4, 9, 13, 0, 24, 128, (16, 24, 24), torch.bfloat16, 0),  # video only
+    (1, 2, 4, 6, 8, 41, 128, (16, 24, 24), torch.bfloat16, 0),   # ragged thread tail
+    (1, 2, 4, 6, 9, 128, 128, (16, 24, 24), torch.bfloat16, 0),  # widest row, D=16384
+    (1, 3, 4, 5, 7, 4, 128, (64, 0, 0), torch.bfloat16, 0),      # 1D RoPE (t only)
+    (1, 10, 40, 50, 1000, 8, 128, (16, 24, 24), torch.bfloat16, 8),  # many rows
+]
+
+
+@pytest.mark.parametrize("B,T,H,W,na,nh,hd,secs,dt,pad", QK_CASES)
+def test_qknorm_rope3d_cases(B, T, H, W, na, nh, hd, secs, dt, pad):
+    D = nh * hd
+    L = T * H * W + na
+    C = 3 * D + pad
+    qkv = activation(B * L, C, dt, DEV, 31 + hd, outliers=True).view(B, L, C)
+    gq = vectors((hd,), 1.0, 0.1, dt, DEV, 32)
+    gk = vectors((hd,), 1.0, 0.1, dt, DEV, 33)
+    spec = (T, H, W, na, nh, hd, secs, 1e-6, 1e4)
+    for gam in ((gq, gk), (None, None)):
+        q, k = api.qknorm_rope3d(qkv, T, H, W, na, nh, hd, secs, gam[0], gam[1])
+        wq, wk = _qk_oracle(_o(qkv.view(B * L, C)), spec,
+                            None if gam[0] is None else _o(gq),
+                            None if gam[1] is None else _o(gk))
+        assert_close(q.reshape(-1, D), wq, "q")
+        assert_close(k.reshape(-1, D), wk, "k")
+
+
+def test_qknorm_rope3d_layouts_and_v_untouched():
+    w = WORKLOADS["medium"]
+    D = w.D
+    t = make_inputs(w, DEV, which=("qknorm_rope3d",))
+    qkv = t["qkv"].view(w.B, w.L, 3 * D)
+    args = (w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections, t["gamma_q"],
+            t["gamma_k"])
+    spec = (w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections, w.eps, w.theta)
+    ids = sample_rows(w.rows, w.L, w.n_video, w.B, 1500, seed=5)
+    wq, wk = _qk_oracle(take_rows(qkv.view(-1, 3 * D)[:, :2 * D], ids), spec,
+                        _o(t["gamma_q"]), _o(t["gamma_k"]), ids)
+    # separate q and k tensors (ld_out = D)
+    qo = torch.empty((w.B, w.L, D), dtype=qkv.dtype, device=DEV)
+    ko = torch.empty_like(qo)
+    api.qknorm_rope3d(qkv, *args, q_out=qo, k_out=ko)
+    assert_close(take_rows_gpu(qo.view(-1, D), ids), wq, "q separate")
+    assert_close(take_rows_gpu(ko.view(-1, D), ids), wk, "k separate")
+    # in place, v columns untouched
+    qi = qkv.clone()
+    v_before = qi[..., 2 * D:].clone()
+    api.qknorm_rope3d(qi, *args, q_out=qi[..., :D], k_out=qi[..., D:2 * D])
+    torch.cuda.synchronize()
+    assert torch.equal(qi[..., 2 * D:], v_before)
+    assert_close(take_rows_gpu(qi.view(-1, 3 * D)[:, :D], ids), wq, "q in place")
+    assert_close(take_rows_gpu(qi.view(-1, 3 * D)[:, D:2 * D], ids), wk, "k in place")
+    # guarded [L, 2D] output
+    pad = 4096
+    n = w.rows * 2 * D
+    buf = torch.full((n + 2 * pad,), 1.5, dtype=qkv.dtype, device=DEV)
+    o = buf[pad:pad + n].view(w.B, w.L, 2 * D)
+    api.qknorm_rope3d(qkv, *args, q_out=o[..., :D], k_out=o[..., D:])
+    torch.cuda.synchronize()
+    assert torch.all(buf[:pad] == 1.5) and torch.all(buf[-pad:] == 1.5)
+    assert_close(take_rows_gpu(o.view(-1, 2 * D)[:, :D], ids), wq, "q guarded")
+
+
+def test_qknorm_rope3d_large_positions_are_accurate():
+    # audio positions up to 4679 (15 s clip): angles reach thousands of radians
+    B, T, H, W, na, nh, hd = 1, 0, 0, 0, 4680, 4, 128
+    L = na
+    qkv = activation(L, 3 * nh * hd, torch.bfloat16, DEV, 77, outliers=False).view(1, L, -1)
+    q, k = api.qknorm_rope3d(qkv, T, H, W, na, nh, hd)
+    ids = np.arange(L - 300, L)
+    wq, wk = oracle.qknorm_rope3d(take_rows(qkv.view(L, -1), ids), T, H, W, na, nh, hd,
+                                  (16, 24, 24), 1e-6, 1e4, row_ids=ids)
+    assert_close(take_rows_gpu(q.reshape(L, -1), ids), wq, "q far positions")
+    assert_close(take_rows_gpu(k.reshape(L, -1), ids), wk, "k far positions")

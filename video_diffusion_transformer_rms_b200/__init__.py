@@ -1,0 +1,15 @@
+"""Fused per-token hot path of a joint video+audio diffusion-transformer
+block on NVIDIA B200 (sm_100a): RMS-AdaLN, the AdaLN-gated residual and
+per-head QKNorm + 3D multimodal RoPE, as CUDA kernels behind a C ABI
+(include/sol.h, libsol.so).
+
+    from video_diffusion_transformer_rms_b200 import api
+    y = api.rms_adaln(x, scale, shift, n_video)
+
+The CUDA library is loaded on first use and must be built; there is no CPU
+path.
+"""
+from ._abi import (SOL_BF16, SOL_F32, SolError, sol_gate_residual, sol_last_error,  # noqa: F401
+                   sol_qknorm_rope3d, sol_rms_adaln, sol_status_string, sol_version)
+
+__version__ = "1.0"

@@ -1,0 +1,96 @@
+"""Tensor-level calls on top of the C ABI: take torch CUDA tensors, pass
+their pointers, shapes and the current stream to libsol.  Marshalling only
+(PyTorch allocates outputs when the caller does not pass them); the
+arithmetic runs in libsol's kernels.
+"""
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+from . import _abi
+
+_DT = {torch.float32: _abi.SOL_F32, torch.bfloat16: _abi.SOL_BF16}
+
+
+def _dtype(*ts) -> int:
+    dts = {t.dtype for t in ts if t is not None}
+    if len(dts) != 1:
+        raise TypeError(f"all tensors must share one dtype, got {dts}")
+    dt = dts.pop()
+    if dt not in _DT:
+        raise TypeError(f"dtype {dt} is not supported (float32 or bfloat16)")
+    return _DT[dt]
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libsol takes CUDA tensors")
+    return t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def rms_adaln(x: torch.Tensor, scale: torch.Tensor, shift: torch.Tensor, n_video: int,
+              gamma: Optional[torch.Tensor] = None, eps: float = 1e-6,
+              out: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """y = RMSNorm(x) * gamma * (1 + scale[b, m]) + shift[b, m]; x: [B, L, D],
+    scale/shift: [B, 2, D]."""
+    if x.dim() != 3 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous [B, L, D] tensor")
+    B, L, D = x.shape
+    y = torch.empty_like(x) if out is None else out
+    _abi.check(_abi.sol_rms_adaln(_ptr(x), _ptr(y), _ptr(scale), _ptr(shift), _ptr(gamma),
+                                  B, L, n_video, D, eps, _dtype(x, y, scale, shift, gamma),
+                                  _stream(stream)))
+    return y
+
+
+def gate_residual(h: torch.Tensor, branch: torch.Tensor, gate: torch.Tensor, n_video: int,
+                  out: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """out = h + gate[b, m] * branch; h/branch: [B, L, D], gate: [B, 2, D]."""
+    if h.dim() != 3 or not h.is_contiguous() or branch.shape != h.shape:
+        raise ValueError("h and branch must be contiguous [B, L, D] tensors of one shape")
+    B, L, D = h.shape
+    o = torch.empty_like(h) if out is None else out
+    _abi.check(_abi.sol_gate_residual(_ptr(h), _ptr(branch), _ptr(gate), _ptr(o), B, L,
+                                      n_video, D, _dtype(h, branch, gate, o), _stream(stream)))
+    return o
+
+
+def qknorm_rope3d(qkv: torch.Tensor, T: int, H: int, W: int, n_audio: int, n_heads: int,
+                  head_dim: int, sections: Sequence[int] = (16, 24, 24),
+                  gamma_q: Optional[torch.Tensor] = None,
+                  gamma_k: Optional[torch.Tensor] = None, eps: float = 1e-6,
+                  theta: float = 10000.0, q_out: Optional[torch.Tensor] = None,
+                  k_out: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None
+                  ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-head QKNorm + 3D RoPE of q and k in a merged qkv [B, L, >=2D]
+    (row stride qkv.stride(1)); returns (q, k) as [B, L, D] views."""
+    if qkv.dim() != 3 or qkv.stride(2) != 1 or qkv.stride(0) != qkv.shape[1] * qkv.stride(1):
+        raise ValueError("qkv must be [B, L, C] with unit column stride and packed rows")
+    B, L, _ = qkv.shape
+    D = n_heads * head_dim
+    if L != T * H * W + n_audio:
+        raise ValueError("L must equal T*H*W + n_audio")
+    if q_out is None and k_out is None:
+        buf = torch.empty((B, L, 2 * D), dtype=qkv.dtype, device=qkv.device)
+        q_out, k_out = buf[..., :D], buf[..., D:]
+    elif q_out is None or k_out is None:
+        raise ValueError("pass both q_out and k_out, or neither")
+    if q_out.stride() != k_out.stride() or q_out.stride(2) != 1:
+        raise ValueError("q_out and k_out must share a row stride with unit column stride")
+    ld_out = q_out.stride(1)
+    st, sh, sw = sections
+    _abi.check(_abi.sol_qknorm_rope3d(
+        _ptr(qkv), qkv.stride(1), _ptr(q_out), _ptr(k_out), ld_out, _ptr(gamma_q),
+        _ptr(gamma_k), B, T, H, W, n_audio, n_heads, head_dim, st, sh, sw, eps, theta,
+        _dtype(qkv, q_out, k_out, gamma_q, gamma_k), _stream(stream)))
+    return q_out, k_out

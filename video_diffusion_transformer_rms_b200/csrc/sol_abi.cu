@@ -1,0 +1,347 @@
+// C ABI of libsol (declared in include/sol.h): host-side argument checks,
+// then one kernel launch on the caller's stream.  Nothing is allocated and
+// nothing is synchronised.
+#include <cstdarg>
+#include <cstdio>
+#include <map>
+#include <mutex>
+#include <string>
+#include <tuple>
+
+#include "sol.h"
+#include "sol_launch.h"
+
+namespace sol {
+namespace {
+
+thread_local std::string g_last_error;
+
+sol_status fail(sol_status s, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+sol_status ok() {
+  g_last_error.clear();
+  return SOL_OK;
+}
+
+sol_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(SOL_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int esize_of(sol_dtype dt) { return dt == SOL_F32 ? 4 : 2; }
+
+// Byte range [begin, end) touched by `rows` rows of `width` bytes, `ld`
+// bytes apart, starting at p.
+struct Span {
+  uintptr_t begin, end;
+};
+Span span_of(const void *p, int64_t rows, int64_t ld, int64_t width) {
+  uintptr_t b = reinterpret_cast<uintptr_t>(p);
+  return Span{b, b + static_cast<uintptr_t>((rows - 1) * ld + width)};
+}
+bool spans_overlap(Span a, Span b) { return a.begin < b.end && b.begin < a.end; }
+
+// True if the strided blocks A (base a, width wa) and B (base b, width wb),
+// both `rows` rows with the same row pitch `ld`, share no byte.  With equal
+// pitches, B's columns sit at offset c = (b - a) mod ld inside A's rows and
+// the blocks are disjoint when wa <= c <= ld - wb.
+bool strided_disjoint(const void *a, int64_t wa, const void *b, int64_t wb, int64_t rows,
+                      int64_t lda, int64_t ldb) {
+  if (!spans_overlap(span_of(a, rows, lda, wa), span_of(b, rows, ldb, wb))) return true;
+  if (lda != ldb) return false;
+  const int64_t off = static_cast<int64_t>(reinterpret_cast<intptr_t>(b) -
+                                           reinterpret_cast<intptr_t>(a));
+  int64_t c = off % lda;
+  if (c < 0) c += lda;
+  return wa <= c && c <= lda - wb;
+}
+
+// Identical or disjoint, for two contiguous [rows, width] tensors.
+bool same_or_disjoint(const void *a, const void *b, int64_t bytes) {
+  if (a == b) return true;
+  return !spans_overlap(span_of(a, 1, 0, bytes), span_of(b, 1, 0, bytes));
+}
+
+struct DevCache {
+  std::mutex mu;
+  std::map<int, int> sms;
+  std::map<std::tuple<const void *, int, int, size_t>, int> occ;
+  std::map<std::pair<const void *, int>, bool> attr_set;
+};
+DevCache &cache() {
+  static DevCache c;
+  return c;
+}
+
+}  // namespace
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  DevCache &c = cache();
+  std::lock_guard<std::mutex> lk(c.mu);
+  auto it = c.sms.find(dev);
+  if (it != c.sms.end()) return it->second;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  c.sms[dev] = n;
+  return n;
+}
+
+int resident_blocks(const void *kernel, int threads, size_t smem) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  DevCache &c = cache();
+  std::lock_guard<std::mutex> lk(c.mu);
+  auto key = std::make_tuple(kernel, dev, threads, smem);
+  auto it = c.occ.find(key);
+  if (it != c.occ.end()) return it->second;
+  auto akey = std::make_pair(kernel, dev);
+  if (!c.attr_set[akey]) {
+    int optin = 0;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+        cudaSuccess)
+      return 0;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) !=
+        cudaSuccess)
+      return 0;
+    c.attr_set[akey] = true;
+  }
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess)
+    return 0;
+  c.occ[key] = n;
+  return n;
+}
+
+bool row_split(int64_t nvec, int pref_vpt, int max_vpt, int max_threads, int group, int *threads,
+               int *vpt) {
+  if (nvec <= 0) return false;
+  int64_t t = (nvec + pref_vpt - 1) / pref_vpt;
+  t = (t + group - 1) / group * group;
+  if (t > max_threads) t = max_threads;
+  const int64_t v = (nvec + t - 1) / t;
+  if (v > max_vpt) return false;
+  *threads = static_cast<int>(t);
+  *vpt = static_cast<int>(v);
+  return true;
+}
+
+}  // namespace sol
+
+using namespace sol;
+
+extern "C" {
+
+int sol_version(void) { return (1 << 16) | 0; }
+
+const char *sol_status_string(sol_status s) {
+  switch (s) {
+    case SOL_OK: return "SOL_OK";
+    case SOL_ERR_INVALID_ARG: return "SOL_ERR_INVALID_ARG";
+    case SOL_ERR_MISALIGNED: return "SOL_ERR_MISALIGNED";
+    case SOL_ERR_UNSUPPORTED: return "SOL_ERR_UNSUPPORTED";
+    case SOL_ERR_CUDA: return "SOL_ERR_CUDA";
+  }
+  return "SOL_ERR_UNKNOWN";
+}
+
+const char *sol_last_error(void) { return g_last_error.c_str(); }
+
+sol_status sol_rms_adaln(const void *x, void *y, const void *scale, const void *shift,
+                         const void *gamma, int64_t B, int64_t L, int64_t n_video, int64_t D,
+                         float eps, sol_dtype dtype, sol_stream_t stream) {
+  if (dtype != SOL_F32 && dtype != SOL_BF16)
+    return fail(SOL_ERR_INVALID_ARG, "sol_rms_adaln: unknown dtype %d", (int)dtype);
+  if (B < 0 || L < 0 || D <= 0 || n_video < 0 || n_video > L)
+    return fail(SOL_ERR_INVALID_ARG,
+                "sol_rms_adaln: need B >= 0, L >= 0, D > 0, 0 <= n_video <= L "
+                "(B=%lld L=%lld n_video=%lld D=%lld)",
+                (long long)B, (long long)L, (long long)n_video, (long long)D);
+  if (!(eps >= 0.f)) return fail(SOL_ERR_INVALID_ARG, "sol_rms_adaln: eps must be >= 0");
+  const int64_t rows = B * L;
+  if (rows == 0) return ok();
+  if (!x || !y || !scale || !shift)
+    return fail(SOL_ERR_INVALID_ARG, "sol_rms_adaln: x, y, scale and shift must be non-null");
+  const int es = esize_of(dtype);
+  const int64_t row_bytes = D * es;
+  if (row_bytes % 16 != 0)
+    return fail(SOL_ERR_MISALIGNED, "sol_rms_adaln: D*%d bytes must be a multiple of 16 (D=%lld)",
+                es, (long long)D);
+  if (!aligned16(x) || !aligned16(y) || !aligned16(scale) || !aligned16(shift) ||
+      (gamma && !aligned16(gamma)))
+    return fail(SOL_ERR_MISALIGNED, "sol_rms_adaln: every pointer must be 16-byte aligned");
+  if (row_bytes > kMaxRowBytesRms)
+    return fail(SOL_ERR_UNSUPPORTED, "sol_rms_adaln: D=%lld exceeds %lld elements", (long long)D,
+                (long long)(kMaxRowBytesRms / es));
+  const int64_t act = rows * row_bytes, mod = B * 2 * row_bytes;
+  if (!same_or_disjoint(x, y, act))
+    return fail(SOL_ERR_INVALID_ARG, "sol_rms_adaln: y must equal x or not overlap it");
+  Span ys = span_of(y, 1, 0, act);
+  if (spans_overlap(ys, span_of(scale, 1, 0, mod)) || spans_overlap(ys, span_of(shift, 1, 0, mod)) ||
+      (gamma && spans_overlap(ys, span_of(gamma, 1, 0, row_bytes))))
+    return fail(SOL_ERR_INVALID_ARG, "sol_rms_adaln: y overlaps scale, shift or gamma");
+
+  RmsArgs a{};
+  a.x = x;
+  a.y = y;
+  a.scale = scale;
+  a.shift = shift;
+  a.gamma = gamma;
+  a.rows = rows;
+  a.L = L;
+  a.n_video = n_video;
+  a.nvec = static_cast<int>(row_bytes / 16);
+  a.eps = eps;
+  a.inv_D = static_cast<float>(1.0 / static_cast<double>(D));
+  cudaError_t e = launch_rms_adaln(a, dtype == SOL_F32 ? 0 : 1, stream, nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_rms_adaln launch");
+  return ok();
+}
+
+sol_status sol_gate_residual(const void *h, const void *branch, const void *gate, void *out,
+                             int64_t B, int64_t L, int64_t n_video, int64_t D, sol_dtype dtype,
+                             sol_stream_t stream) {
+  if (dtype != SOL_F32 && dtype != SOL_BF16)
+    return fail(SOL_ERR_INVALID_ARG, "sol_gate_residual: unknown dtype %d", (int)dtype);
+  if (B < 0 || L < 0 || D <= 0 || n_video < 0 || n_video > L)
+    return fail(SOL_ERR_INVALID_ARG,
+                "sol_gate_residual: need B >= 0, L >= 0, D > 0, 0 <= n_video <= L "
+                "(B=%lld L=%lld n_video=%lld D=%lld)",
+                (long long)B, (long long)L, (long long)n_video, (long long)D);
+  const int64_t rows = B * L;
+  if (rows == 0) return ok();
+  if (!h || !branch || !gate || !out)
+    return fail(SOL_ERR_INVALID_ARG, "sol_gate_residual: h, branch, gate and out must be non-null");
+  const int es = esize_of(dtype);
+  const int64_t row_bytes = D * es;
+  if (row_bytes % 16 != 0)
+    return fail(SOL_ERR_MISALIGNED,
+                "sol_gate_residual: D*%d bytes must be a multiple of 16 (D=%lld)", es,
+                (long long)D);
+  if (!aligned16(h) || !aligned16(branch) || !aligned16(gate) || !aligned16(out))
+    return fail(SOL_ERR_MISALIGNED, "sol_gate_residual: every pointer must be 16-byte aligned");
+  if (row_bytes > kMaxRowBytesGate)
+    return fail(SOL_ERR_UNSUPPORTED, "sol_gate_residual: D=%lld exceeds %lld elements",
+                (long long)D, (long long)(kMaxRowBytesGate / es));
+  const int64_t act = rows * row_bytes, mod = B * 2 * row_bytes;
+  if (!same_or_disjoint(out, h, act) || !same_or_disjoint(out, branch, act))
+    return fail(SOL_ERR_INVALID_ARG,
+                "sol_gate_residual: out must equal h or branch, or overlap neither");
+  if (spans_overlap(span_of(out, 1, 0, act), span_of(gate, 1, 0, mod)))
+    return fail(SOL_ERR_INVALID_ARG, "sol_gate_residual: out overlaps gate");
+
+  GateArgs a{};
+  a.h = h;
+  a.branch = branch;
+  a.gate = gate;
+  a.out = out;
+  a.rows = rows;
+  a.L = L;
+  a.n_video = n_video;
+  a.nvec = static_cast<int>(row_bytes / 16);
+  cudaError_t e = launch_gate_residual(a, dtype == SOL_F32 ? 0 : 1, stream, nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_gate_residual launch");
+  return ok();
+}
+
+sol_status sol_qknorm_rope3d(const void *qkv, int64_t ld_qkv, void *q_out, void *k_out,
+                             int64_t ld_out, const void *gamma_q, const void *gamma_k, int64_t B,
+                             int64_t T, int64_t H, int64_t W, int64_t n_audio, int64_t n_heads,
+                             int64_t head_dim, int64_t sec_t, int64_t sec_h, int64_t sec_w,
+                             float eps, float theta, sol_dtype dtype, sol_stream_t stream) {
+  if (dtype != SOL_F32 && dtype != SOL_BF16)
+    return fail(SOL_ERR_INVALID_ARG, "sol_qknorm_rope3d: unknown dtype %d", (int)dtype);
+  if (B < 0 || T < 0 || H < 0 || W < 0 || n_audio < 0)
+    return fail(SOL_ERR_INVALID_ARG, "sol_qknorm_rope3d: B, T, H, W, n_audio must be >= 0");
+  if (n_heads <= 0 || head_dim <= 0 || head_dim % 2 != 0)
+    return fail(SOL_ERR_INVALID_ARG,
+                "sol_qknorm_rope3d: need n_heads > 0 and an even head_dim > 0 (%lld, %lld)",
+                (long long)n_heads, (long long)head_dim);
+  if (sec_t < 0 || sec_h < 0 || sec_w < 0 || sec_t + sec_h + sec_w != head_dim / 2)
+    return fail(SOL_ERR_INVALID_ARG,
+                "sol_qknorm_rope3d: sections %lld+%lld+%lld must sum to head_dim/2 = %lld",
+                (long long)sec_t, (long long)sec_h, (long long)sec_w, (long long)(head_dim / 2));
+  if (!(eps >= 0.f) || !(theta > 0.f))
+    return fail(SOL_ERR_INVALID_ARG, "sol_qknorm_rope3d: need eps >= 0 and theta > 0");
+  const int64_t n_video = T * H * W;
+  const int64_t L = n_video + n_audio;
+  const int64_t rows = B * L;
+  const int64_t D = n_heads * head_dim;
+  if (ld_qkv < 2 * D || ld_out < D)
+    return fail(SOL_ERR_INVALID_ARG, "sol_qknorm_rope3d: need ld_qkv >= 2*D and ld_out >= D");
+  if (rows == 0) return ok();
+  if (!qkv || !q_out || !k_out)
+    return fail(SOL_ERR_INVALID_ARG, "sol_qknorm_rope3d: qkv, q_out and k_out must be non-null");
+  const int es = esize_of(dtype);
+  const int64_t hd_bytes = head_dim * es;
+  const int64_t G = hd_bytes / 16;
+  if (hd_bytes % 16 != 0 || G < 2 || G > 32 || (G & (G - 1)) != 0)
+    return fail(SOL_ERR_UNSUPPORTED,
+                "sol_qknorm_rope3d: head_dim*%d bytes must be 16*G with G a power of two in "
+                "[2, 32] (head_dim=%lld)",
+                es, (long long)head_dim);
+  const int64_t ldq_b = ld_qkv * es, ldo_b = ld_out * es, D_b = D * es;
+  if (!aligned16(qkv) || !aligned16(q_out) || !aligned16(k_out) || ldq_b % 16 || ldo_b % 16 ||
+      (gamma_q && !aligned16(gamma_q)) || (gamma_k && !aligned16(gamma_k)))
+    return fail(SOL_ERR_MISALIGNED,
+                "sol_qknorm_rope3d: pointers and row strides must be 16-byte aligned");
+  if (2 * D_b > kMaxRowBytesQk)
+    return fail(SOL_ERR_UNSUPPORTED, "sol_qknorm_rope3d: 2*D=%lld exceeds %lld elements",
+                (long long)(2 * D), (long long)(kMaxRowBytesQk / es));
+  const bool in_place = q_out == qkv && ld_out == ld_qkv &&
+                        static_cast<const unsigned char *>(k_out) ==
+                            static_cast<const unsigned char *>(qkv) + D_b;
+  if (!in_place) {
+    if (!strided_disjoint(qkv, 2 * D_b, q_out, D_b, rows, ldq_b, ldo_b) ||
+        !strided_disjoint(qkv, 2 * D_b, k_out, D_b, rows, ldq_b, ldo_b) ||
+        !strided_disjoint(q_out, D_b, k_out, D_b, rows, ldo_b, ldo_b))
+      return fail(SOL_ERR_INVALID_ARG,
+                  "sol_qknorm_rope3d: outputs must be exactly in place (q_out=qkv, "
+                  "k_out=qkv+D, ld_out=ld_qkv) or overlap neither qkv nor each other");
+  }
+  for (const void *g : {gamma_q, gamma_k}) {
+    if (!g) continue;
+    Span gs = span_of(g, 1, 0, hd_bytes);
+    if (spans_overlap(gs, span_of(q_out, rows, ldo_b, D_b)) ||
+        spans_overlap(gs, span_of(k_out, rows, ldo_b, D_b)))
+      return fail(SOL_ERR_INVALID_ARG, "sol_qknorm_rope3d: an output overlaps gamma");
+  }
+
+  QkArgs a{};
+  a.qkv = qkv;
+  a.q_out = q_out;
+  a.k_out = k_out;
+  a.gamma_q = gamma_q;
+  a.gamma_k = gamma_k;
+  a.ld_qkv_bytes = ldq_b;
+  a.ld_out_bytes = ldo_b;
+  a.rows = rows;
+  a.L = L;
+  a.n_video = n_video;
+  a.HW = H * W;
+  a.W = W;
+  a.nvec = static_cast<int>(2 * D_b / 16);
+  a.nvec_q = static_cast<int>(D_b / 16);
+  a.npairs = static_cast<int>(head_dim / 2);
+  a.sec_t = static_cast<int>(sec_t);
+  a.sec_th = static_cast<int>(sec_t + sec_h);
+  a.head_dim = static_cast<int>(head_dim);
+  a.eps = eps;
+  a.inv_hd = static_cast<float>(1.0 / static_cast<double>(head_dim));
+  a.theta = theta;
+  cudaError_t e = launch_qknorm_rope3d(a, dtype == SOL_F32 ? 0 : 1, stream, nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_qknorm_rope3d launch");
+  return ok();
+}
+
+}  // extern "C"

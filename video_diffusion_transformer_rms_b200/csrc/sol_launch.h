@@ -1,0 +1,99 @@
+// Host-side interface between the C ABI (sol_abi.cu) and the kernel
+// launchers.  Internal to libsol: arguments arrive here already validated.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sol {
+
+// Launch geometry of one persistent row-streaming kernel.
+struct Geometry {
+  int threads;   // CTA size, a multiple of 32
+  int vpt;       // 16-byte vectors per thread per row (1 .. max)
+  int stages;    // depth of the cp.async ring
+  size_t smem;   // dynamic shared memory per CTA
+  int grid;      // CTAs (at most one wave of resident CTAs)
+};
+
+// CTAs of `kernel` resident per SM at (threads, smem) on the current device;
+// raises the kernel's dynamic shared-memory limit once per device.  Returns
+// 0 if the configuration cannot be resident (or on a CUDA error, which is
+// left for cudaGetLastError).
+int resident_blocks(const void *kernel, int threads, size_t smem);
+
+// Streaming multiprocessors of the current device (cached per device).
+int device_sms();
+
+// Pick threads / vectors-per-thread for a row of `nvec` 16-byte vectors:
+// up to `pref_vpt` vectors per thread, CTAs of at most `max_threads`
+// threads (a multiple of `group`), at most `max_vpt` vectors per thread.
+// Returns false if the row does not fit.
+bool row_split(int64_t nvec, int pref_vpt, int max_vpt, int max_threads, int group,
+               int *threads, int *vpt);
+
+struct RmsArgs {
+  const void *x;
+  void *y;
+  const void *scale;
+  const void *shift;
+  const void *gamma;  // may be null
+  int64_t rows;       // B * L
+  int64_t L;
+  int64_t n_video;
+  int nvec;           // 16-byte vectors per row
+  float eps;
+  float inv_D;
+};
+
+struct GateArgs {
+  const void *h;
+  const void *branch;
+  const void *gate;
+  void *out;
+  int64_t rows;
+  int64_t L;
+  int64_t n_video;
+  int nvec;
+};
+
+struct QkArgs {
+  const void *qkv;
+  void *q_out;
+  void *k_out;
+  const void *gamma_q;  // may be null
+  const void *gamma_k;  // may be null
+  int64_t ld_qkv_bytes;
+  int64_t ld_out_bytes;
+  int64_t rows;       // B * L
+  int64_t L;
+  int64_t n_video;    // T * H * W
+  int64_t HW;         // H * W
+  int64_t W;
+  int nvec;           // 16-byte vectors in q and k of one row (2 * nvec_q)
+  int nvec_q;         // 16-byte vectors in q of one row
+  int npairs;         // head_dim / 2
+  int sec_t;          // pairs on the t axis
+  int sec_th;         // sec_t + sec_h
+  int head_dim;
+  float eps;
+  float inv_hd;
+  float theta;
+};
+
+// dtype: 0 = fp32, 1 = bf16 (sol_dtype).  Each returns the launch error
+// (cudaSuccess if the kernel was enqueued) and fills `geo` if non-null.
+cudaError_t launch_rms_adaln(const RmsArgs &a, int dtype, cudaStream_t stream, Geometry *geo);
+cudaError_t launch_gate_residual(const GateArgs &a, int dtype, cudaStream_t stream,
+                                 Geometry *geo);
+cudaError_t launch_qknorm_rope3d(const QkArgs &a, int dtype, cudaStream_t stream,
+                                 Geometry *geo);
+
+// Limits the launchers accept (checked by the ABI before calling them).
+constexpr int kMaxThreads = 512;
+constexpr int64_t kMaxRowBytesRms = 32768;   // D * esize for RMS-AdaLN
+constexpr int64_t kMaxRowBytesGate = 32768;  // D * esize for the gated residual
+constexpr int64_t kMaxRowBytesQk = 65536;    // 2 * D * esize for QKNorm + RoPE
+
+}  // namespace sol
