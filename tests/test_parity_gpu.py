@@ -255,6 +255,8 @@ QK_CASES = [
     (1, 2, 4, 6, 9, 128, 128, (16, 24, 24), torch.bfloat16, 0),  # widest row, D=16384
     (1, 3, 4, 5, 7, 4, 128, (64, 0, 0), torch.bfloat16, 0),      # 1D RoPE (t only)
     (1, 10, 40, 50, 1000, 8, 128, (16, 24, 24), torch.bfloat16, 8),  # many rows
+    (3, 3, 7, 11, 500, 40, 128, (16, 24, 24), torch.bfloat16, 16),   # CTAs cross W, H,
+    # video/audio and sample boundaries inside their row share
 ]
 
 

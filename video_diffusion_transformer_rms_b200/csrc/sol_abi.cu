@@ -123,17 +123,17 @@ int resident_blocks(const void *kernel, int threads, size_t smem) {
   return n;
 }
 
-bool row_split(int64_t nvec, int pref_vpt, int max_vpt, int max_threads, int group, int *threads,
-               int *vpt) {
+bool pick_split(int64_t nvec, int *threads, int *vpt) {
   if (nvec <= 0) return false;
-  int64_t t = (nvec + pref_vpt - 1) / pref_vpt;
-  t = (t + group - 1) / group * group;
-  if (t > max_threads) t = max_threads;
-  const int64_t v = (nvec + t - 1) / t;
-  if (v > max_vpt) return false;
-  *threads = static_cast<int>(t);
-  *vpt = static_cast<int>(v);
-  return true;
+  for (int t = 32; t <= kMaxThreads; t *= 2) {
+    const int64_t v = (nvec + t - 1) / t;
+    if (v <= 6 || (t == kMaxThreads && v <= kMaxVpt)) {
+      *threads = t;
+      *vpt = static_cast<int>(v);
+      return true;
+    }
+  }
+  return false;
 }
 
 }  // namespace sol
@@ -329,8 +329,8 @@ sol_status sol_qknorm_rope3d(const void *qkv, int64_t ld_qkv, void *q_out, void 
   a.L = L;
   a.n_video = n_video;
   a.HW = H * W;
+  a.H = H;
   a.W = W;
-  a.nvec = static_cast<int>(2 * D_b / 16);
   a.nvec_q = static_cast<int>(D_b / 16);
   a.npairs = static_cast<int>(head_dim / 2);
   a.sec_t = static_cast<int>(sec_t);

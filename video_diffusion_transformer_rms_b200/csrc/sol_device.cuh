@@ -2,7 +2,8 @@
 //
 // Every kernel streams token rows HBM -> shared memory with cp.async
 // (16-byte LDGSTS, L2-only, no register staging) in an S-stage ring per CTA,
-// computes in fp32 registers and writes results back with 16-byte
+// computes in fp32 registers with Blackwell's packed fp32x2 FMA/MUL (two
+// lanes of arithmetic per instruction) and writes results back with 16-byte
 // streaming stores.  Each thread copies and later consumes exactly the same
 // 16-byte slots of every stage, so the ring needs no CTA barrier: a thread's
 // own cp.async.wait_group is enough.
@@ -13,6 +14,10 @@
 #include <stdint.h>
 
 namespace sol {
+
+// ---------------------------------------------------------------------------
+// memory movement
+// ---------------------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -48,49 +53,86 @@ __device__ __forceinline__ uint4 ld_shared_vec(const void *gmem_src) {
   return __ldg(reinterpret_cast<const uint4 *>(gmem_src));
 }
 
-// Element type traits: E elements per 16-byte vector, exact widening to fp32
-// and round-to-nearest-even narrowing.
+// ---------------------------------------------------------------------------
+// packed fp32x2 arithmetic (one instruction for two lanes on sm_100)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
+
+// ---------------------------------------------------------------------------
+// element types: a 16-byte vector holds E elements = E/2 natural pairs
+// (elements 2i, 2i+1).  Widening is exact, narrowing rounds to nearest even.
+// ---------------------------------------------------------------------------
+
 template <typename T>
 struct Io;
 
 template <>
 struct Io<float> {
   static constexpr int E = 4;
-  __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[E]) {
-    f[0] = __uint_as_float(v.x);
-    f[1] = __uint_as_float(v.y);
-    f[2] = __uint_as_float(v.z);
-    f[3] = __uint_as_float(v.w);
+  __device__ __forceinline__ static void unpack(const uint4 &v, float2 (&p)[2]) {
+    p[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+    p[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
   }
-  __device__ __forceinline__ static uint4 pack(const float (&f)[E]) {
-    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
-                      __float_as_uint(f[3]));
+  __device__ __forceinline__ static uint4 pack(const float2 (&p)[2]) {
+    return make_uint4(__float_as_uint(p[0].x), __float_as_uint(p[0].y), __float_as_uint(p[1].x),
+                      __float_as_uint(p[1].y));
+  }
+  // Rotary split: ev[m] = (x[4m], x[4m+2]), od[m] = (x[4m+1], x[4m+3]), so
+  // that lane 0 / lane 1 of each float2 belong to rotary pairs 2m / 2m+1.
+  __device__ __forceinline__ static void unpack_eo(const uint4 &v, float2 (&ev)[1],
+                                                   float2 (&od)[1]) {
+    ev[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.z));
+    od[0] = make_float2(__uint_as_float(v.y), __uint_as_float(v.w));
+  }
+  // Inverse of unpack_eo for the rotated pair components u0 (first) / u1.
+  __device__ __forceinline__ static uint4 pack_eo(const float2 (&u0)[1], const float2 (&u1)[1]) {
+    return make_uint4(__float_as_uint(u0[0].x), __float_as_uint(u1[0].x),
+                      __float_as_uint(u0[0].y), __float_as_uint(u1[0].y));
   }
 };
 
 template <>
 struct Io<__nv_bfloat16> {
   static constexpr int E = 8;
-  // bf16 is the upper half of a binary32 pattern: widening is a shift.
-  __device__ __forceinline__ static void unpack2(uint32_t w, float &lo, float &hi) {
-    lo = __uint_as_float(w << 16);
-    hi = __uint_as_float(w & 0xffff0000u);
+  // bf16 is the upper half of a binary32 pattern: widening is a shift / mask.
+  __device__ __forceinline__ static float lo(uint32_t w) { return __uint_as_float(w << 16); }
+  __device__ __forceinline__ static float hi(uint32_t w) {
+    return __uint_as_float(w & 0xffff0000u);
   }
-  __device__ __forceinline__ static uint32_t pack2(float lo, float hi) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
-    return *reinterpret_cast<uint32_t *>(&h);
+  __device__ __forceinline__ static uint32_t pack2(float l, float h) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(l, h);  // .x (low half) = l
+    return *reinterpret_cast<uint32_t *>(&b);
   }
-  __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[E]) {
-    unpack2(v.x, f[0], f[1]);
-    unpack2(v.y, f[2], f[3]);
-    unpack2(v.z, f[4], f[5]);
-    unpack2(v.w, f[6], f[7]);
+  __device__ __forceinline__ static void unpack(const uint4 &v, float2 (&p)[4]) {
+    p[0] = make_float2(lo(v.x), hi(v.x));
+    p[1] = make_float2(lo(v.y), hi(v.y));
+    p[2] = make_float2(lo(v.z), hi(v.z));
+    p[3] = make_float2(lo(v.w), hi(v.w));
   }
-  __device__ __forceinline__ static uint4 pack(const float (&f)[E]) {
-    return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]),
-                      pack2(f[6], f[7]));
+  __device__ __forceinline__ static uint4 pack(const float2 (&p)[4]) {
+    return make_uint4(pack2(p[0].x, p[0].y), pack2(p[1].x, p[1].y), pack2(p[2].x, p[2].y),
+                      pack2(p[3].x, p[3].y));
+  }
+  __device__ __forceinline__ static void unpack_eo(const uint4 &v, float2 (&ev)[2],
+                                                   float2 (&od)[2]) {
+    ev[0] = make_float2(lo(v.x), lo(v.y));
+    od[0] = make_float2(hi(v.x), hi(v.y));
+    ev[1] = make_float2(lo(v.z), lo(v.w));
+    od[1] = make_float2(hi(v.z), hi(v.w));
+  }
+  __device__ __forceinline__ static uint4 pack_eo(const float2 (&u0)[2], const float2 (&u1)[2]) {
+    return make_uint4(pack2(u0[0].x, u1[0].x), pack2(u0[0].y, u1[0].y), pack2(u0[1].x, u1[1].x),
+                      pack2(u0[1].y, u1[1].y));
   }
 };
+
+// ---------------------------------------------------------------------------
+// reductions
+// ---------------------------------------------------------------------------
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -105,5 +147,70 @@ __device__ __forceinline__ float group_sum(float v) {
   for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
+
+// ---------------------------------------------------------------------------
+// row bookkeeping
+// ---------------------------------------------------------------------------
+
+// Contiguous share [begin, end) of `rows` for CTA `cta` out of `ctas`; the
+// shares differ by at most one row.
+__device__ __forceinline__ void cta_rows(int64_t rows, int64_t cta, int64_t ctas,
+                                         int64_t &begin, int64_t &end) {
+  begin = rows * cta / ctas;
+  end = rows * (cta + 1) / ctas;
+}
+
+// (sample b, row r in the sample) of a global row, advanced one row at a
+// time: one division per CTA instead of one per row.
+struct TokenCursor {
+  int64_t b, r;
+  __device__ __forceinline__ void init(int64_t row, int64_t L) {
+    b = row / L;
+    r = row - b * L;
+  }
+  __device__ __forceinline__ void next(int64_t L) {
+    if (++r == L) {
+      r = 0;
+      ++b;
+    }
+  }
+};
+
+// 3D rotary position (t, h, w) of the row a TokenCursor points at: video
+// rows r < n_video walk the T x H x W grid in raster order (t-major), audio
+// row i = r - n_video sits at (i, 0, 0).
+struct GridCursor {
+  int64_t t, h, w;
+  __device__ __forceinline__ void init(int64_t r, int64_t n_video, int64_t HW, int64_t W) {
+    if (r < n_video) {
+      t = r / HW;
+      const int64_t rem = r - t * HW;
+      h = rem / W;
+      w = rem - h * W;
+    } else {
+      t = r - n_video;
+      h = 0;
+      w = 0;
+    }
+  }
+  // Move to row r_next (= r + 1, or 0 when a new sample starts).
+  __device__ __forceinline__ void next(int64_t r_next, int64_t n_video, int64_t H, int64_t W) {
+    if (r_next == 0 || r_next == n_video) {
+      t = 0;
+      h = 0;
+      w = 0;
+    } else if (r_next < n_video) {
+      if (++w == W) {
+        w = 0;
+        if (++h == H) {
+          h = 0;
+          ++t;
+        }
+      }
+    } else {
+      ++t;
+    }
+  }
+};
 
 }  // namespace sol

@@ -26,12 +26,18 @@ int resident_blocks(const void *kernel, int threads, size_t smem);
 // Streaming multiprocessors of the current device (cached per device).
 int device_sms();
 
-// Pick threads / vectors-per-thread for a row of `nvec` 16-byte vectors:
-// up to `pref_vpt` vectors per thread, CTAs of at most `max_threads`
-// threads (a multiple of `group`), at most `max_vpt` vectors per thread.
-// Returns false if the row does not fit.
-bool row_split(int64_t nvec, int pref_vpt, int max_vpt, int max_threads, int group,
-               int *threads, int *vpt);
+// CTA size and 16-byte vectors per thread for a row of `nvec` vectors: the
+// smallest CTA of {32, 64, 128, 256} threads that needs at most 6 vectors
+// per thread, else 256 threads with up to 8.  Wide per-thread slices keep
+// the per-row bookkeeping (one barrier, one reduction, address math) small
+// against the streamed bytes.  Returns false if the row does not fit.
+bool pick_split(int64_t nvec, int *threads, int *vpt);
+
+// Every (threads, vectors per thread) pick_split can return, for the
+// launchers' compile-time dispatch.
+#define SOL_SPLITS(X)                                                              \
+  X(32, 1) X(32, 2) X(32, 3) X(32, 4) X(32, 5) X(32, 6) X(64, 4) X(64, 5) X(64, 6) \
+  X(128, 4) X(128, 5) X(128, 6) X(256, 4) X(256, 5) X(256, 6) X(256, 7) X(256, 8)
 
 struct RmsArgs {
   const void *x;
@@ -70,9 +76,9 @@ struct QkArgs {
   int64_t L;
   int64_t n_video;    // T * H * W
   int64_t HW;         // H * W
+  int64_t H;
   int64_t W;
-  int nvec;           // 16-byte vectors in q and k of one row (2 * nvec_q)
-  int nvec_q;         // 16-byte vectors in q of one row
+  int nvec_q;         // 16-byte vectors in q (and in k) of one row
   int npairs;         // head_dim / 2
   int sec_t;          // pairs on the t axis
   int sec_th;         // sec_t + sec_h
@@ -87,11 +93,17 @@ struct QkArgs {
 cudaError_t launch_rms_adaln(const RmsArgs &a, int dtype, cudaStream_t stream, Geometry *geo);
 cudaError_t launch_gate_residual(const GateArgs &a, int dtype, cudaStream_t stream,
                                  Geometry *geo);
-cudaError_t launch_qknorm_rope3d(const QkArgs &a, int dtype, cudaStream_t stream,
-                                 Geometry *geo);
+cudaError_t launch_qknorm_rope3d_f32(const QkArgs &a, cudaStream_t stream, Geometry *geo);
+cudaError_t launch_qknorm_rope3d_bf16(const QkArgs &a, cudaStream_t stream, Geometry *geo);
+inline cudaError_t launch_qknorm_rope3d(const QkArgs &a, int dtype, cudaStream_t stream,
+                                        Geometry *geo) {
+  return dtype == 0 ? launch_qknorm_rope3d_f32(a, stream, geo)
+                    : launch_qknorm_rope3d_bf16(a, stream, geo);
+}
 
 // Limits the launchers accept (checked by the ABI before calling them).
-constexpr int kMaxThreads = 512;
+constexpr int kMaxThreads = 256;
+constexpr int kMaxVpt = 8;
 constexpr int64_t kMaxRowBytesRms = 32768;   // D * esize for RMS-AdaLN
 constexpr int64_t kMaxRowBytesGate = 32768;  // D * esize for the gated residual
 constexpr int64_t kMaxRowBytesQk = 65536;    // 2 * D * esize for QKNorm + RoPE
