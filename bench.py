@@ -42,10 +42,11 @@ from video_diffusion_transformer_rms_b200.workloads import (WORKLOADS, activatio
 METRIC = "tokens/s and achieved HBM GB/s (% of B200 peak) per fused kernel, 1 GPU"
 WORKLOAD = "clip5s"
 KERNELS = ("rms_adaln", "qknorm_rope3d", "gate_residual")
+_COMMON_SOURCES = ["sol_device.cuh", "sol_launch.h", "sol_abi.cu"]
 KERNEL_SOURCES = {
-    "rms_adaln": ["rms_adaln.cu", "sol_device.cuh"],
-    "gate_residual": ["gate_residual.cu", "sol_device.cuh"],
-    "qknorm_rope3d": ["qknorm_rope3d.cu", "sol_device.cuh"],
+    "rms_adaln": ["rms_adaln.cu"] + _COMMON_SOURCES,
+    "gate_residual": ["gate_residual.cu"] + _COMMON_SOURCES,
+    "qknorm_rope3d": ["qknorm_rope3d.cuh", "qknorm_rope3d_bf16.cu"] + _COMMON_SOURCES,
 }
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0

@@ -74,6 +74,8 @@ def qk(qkv=A, ldq=768, qo=A + (1 << 30), ko=A + (2 << 30), ldo=256, gq=None, gk=
     (dict(g=A + (4 << 30) + 4), _abi.SOL_ERR_MISALIGNED),
     (dict(D=16392), _abi.SOL_ERR_UNSUPPORTED),
     (dict(D=8196, dt=F32), _abi.SOL_ERR_UNSUPPORTED),
+    (dict(B=1 << 20, L=1 << 12), _abi.SOL_ERR_UNSUPPORTED),  # 2^32 rows
+    (dict(B=1, L=1 << 31, nv=0), _abi.SOL_ERR_UNSUPPORTED),
     (dict(y=A + 16), _abi.SOL_ERR_INVALID_ARG),      # partial overlap with x
     (dict(y=A + (2 << 30) + 64), _abi.SOL_ERR_INVALID_ARG),  # overlaps scale
 ])
@@ -96,6 +98,7 @@ def test_zero_rows_is_a_noop_even_with_null_pointers():
     (dict(D=20), _abi.SOL_ERR_MISALIGNED),
     (dict(g=A + (2 << 30) + 2), _abi.SOL_ERR_MISALIGNED),
     (dict(D=16400), _abi.SOL_ERR_UNSUPPORTED),
+    (dict(B=3, L=1 << 30, nv=0), _abi.SOL_ERR_UNSUPPORTED),
     (dict(out=A + 32), _abi.SOL_ERR_INVALID_ARG),     # partial overlap with h
     (dict(out=A + (1 << 30) - 32), _abi.SOL_ERR_INVALID_ARG),  # straddles branch
     (dict(out=A + (2 << 30)), _abi.SOL_ERR_INVALID_ARG),  # overlaps gate
@@ -117,6 +120,9 @@ def test_gate_residual_rejects(kw, status):
     (dict(hd=256, secs=(32, 48, 48), dt=F32, ldq=1536, ldo=512),
      _abi.SOL_ERR_UNSUPPORTED),  # G = 64 lanes (fp32)
     (dict(nh=130, ldq=3 * 16640, ldo=16640), _abi.SOL_ERR_UNSUPPORTED),  # D > 16384
+    (dict(T=1, H=1 << 16, W=1 << 16, na=0), _abi.SOL_ERR_UNSUPPORTED),  # H*W = 2^32
+    (dict(T=0, H=1 << 16, W=1 << 16), _abi.SOL_ERR_UNSUPPORTED),
+    (dict(B=1 << 22, T=1, H=32, W=32, na=0), _abi.SOL_ERR_UNSUPPORTED),  # 2^32 rows
     (dict(ldq=772), _abi.SOL_ERR_MISALIGNED),        # 1544-byte row stride
     (dict(qo=A + (1 << 30) + 2), _abi.SOL_ERR_MISALIGNED),
     (dict(qo=A + 512), _abi.SOL_ERR_INVALID_ARG),    # q_out inside qkv's k columns

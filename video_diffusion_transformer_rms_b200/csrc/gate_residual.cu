@@ -32,19 +32,23 @@ __global__ void __launch_bounds__(NT) gate_residual_kernel(const GateArgs a) {
 #pragma unroll
   for (int k = 0; k < VPT; ++k) ok[k] = k * NT + tid < a.nvec;
 
-  int64_t begin, end;
-  cta_rows(a.rows, blockIdx.x, gridDim.x, begin, end);
-  const int64_t iters = (end - begin + R - 1) / R;
+  int64_t begin;
+  int count;
+  cta_rows(a.rows, blockIdx.x, gridDim.x, begin, count);
+  const int iters = (count + R - 1) / R;
+  const unsigned char *hc = hb + begin * row_bytes;
+  const unsigned char *bc = bb + begin * row_bytes;
+  unsigned char *oc = ob + begin * row_bytes;
   auto slot = [&](int s, int q, int which, int k) -> uint4 * {
     return &ring[(((s * R + q) * 2 + which) * VPT + k) * NT + tid];
   };
-  auto issue = [&](int64_t it, int s) {
+  auto issue = [&](int it, int s) {
 #pragma unroll
     for (int q = 0; q < R; ++q) {
-      const int64_t row = begin + it * R + q;
-      if (it < iters && row < end) {
-        const uint4 *hs = reinterpret_cast<const uint4 *>(hb + row * row_bytes) + tid;
-        const uint4 *bs = reinterpret_cast<const uint4 *>(bb + row * row_bytes) + tid;
+      const int j = it * R + q;
+      if (j < count) {
+        const uint4 *hs = reinterpret_cast<const uint4 *>(hc + j * row_bytes) + tid;
+        const uint4 *bs = reinterpret_cast<const uint4 *>(bc + j * row_bytes) + tid;
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
           if (ok[k]) {
@@ -61,26 +65,27 @@ __global__ void __launch_bounds__(NT) gate_residual_kernel(const GateArgs a) {
   for (int s = 0; s < S - 1; ++s) issue(s, s);
 
   float2 gv[VPT][P];
-  int64_t key = -1;
+  int key = -1;
   int cons = 0;
   TokenCursor cur;
   cur.init(begin, a.L);
-  for (int64_t it = 0; it < iters; ++it) {
+  for (int it = 0; it < iters; ++it) {
     issue(it + S - 1, cons == 0 ? S - 1 : cons - 1);
     cp_async_wait<S - 1>();
 #pragma unroll
     for (int q = 0; q < R; ++q) {
-      const int64_t row = begin + it * R + q;
-      if (row < end) {
-        const int64_t nkey = 2 * cur.b + (cur.r >= a.n_video ? 1 : 0);
+      const int j = it * R + q;
+      if (j < count) {
+        const int nkey = 2 * cur.b + (cur.r >= a.n_video ? 1 : 0);
         if (nkey != key) {
           key = nkey;
-          const uint4 *g0 = static_cast<const uint4 *>(a.gate) + key * a.nvec + tid;
+          const uint4 *g0 =
+              static_cast<const uint4 *>(a.gate) + static_cast<int64_t>(key) * a.nvec + tid;
 #pragma unroll
           for (int k = 0; k < VPT; ++k)
             if (ok[k]) IO::unpack(ld_shared_vec(g0 + k * NT), gv[k]);
         }
-        uint4 *orow = reinterpret_cast<uint4 *>(ob + row * row_bytes) + tid;
+        uint4 *orow = reinterpret_cast<uint4 *>(oc + j * row_bytes) + tid;
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
           if (ok[k]) {

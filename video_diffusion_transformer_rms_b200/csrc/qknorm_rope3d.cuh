@@ -79,18 +79,22 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
   for (int p = tid; p < a.npairs; p += NT)
     freq[p] = pow(static_cast<double>(a.theta), -2.0 * p / a.head_dim);
 
-  int64_t begin, end;
-  cta_rows(a.rows, blockIdx.x, gridDim.x, begin, end);
-  const int64_t iters = (end - begin + R - 1) / R;
+  int64_t begin;
+  int count;
+  cta_rows(a.rows, blockIdx.x, gridDim.x, begin, count);
+  const int iters = (count + R - 1) / R;
+  const unsigned char *src_c = qkv + begin * a.ld_qkv_bytes;
+  unsigned char *qo_c = qo + begin * a.ld_out_bytes;
+  unsigned char *ko_c = ko + begin * a.ld_out_bytes;
   auto slot = [&](int s, int q, int part, int k) -> uint4 * {
     return &ring[(((s * R + q) * 2 + part) * VPT + k) * NT + tid];
   };
-  auto issue = [&](int64_t it, int s) {
+  auto issue = [&](int it, int s) {
 #pragma unroll
     for (int q = 0; q < R; ++q) {
-      const int64_t row = begin + it * R + q;
-      if (it < iters && row < end) {
-        const unsigned char *src = qkv + row * a.ld_qkv_bytes;
+      const int j = it * R + q;
+      if (j < count) {
+        const unsigned char *src = src_c + j * a.ld_qkv_bytes;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
           const uint4 *ps = reinterpret_cast<const uint4 *>(src + part * part_bytes) + tid;
@@ -113,11 +117,11 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
   pos.init(tok.r, a.n_video, a.HW, a.W);
   int cons = 0;
   int buf = 0;
-  for (int64_t it = 0; it < iters; ++it) {
+  for (int it = 0; it < iters; ++it) {
     issue(it + S - 1, cons == 0 ? S - 1 : cons - 1);
 
     // positions of this iteration's rows (rows past `end` are never read)
-    int64_t pt[R], ph[R], pw[R];
+    int pt[R], ph[R], pw[R];
     {
       TokenCursor t2 = tok;
       GridCursor g2 = pos;
@@ -139,7 +143,7 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
           p -= a.npairs;
           q = qq;
         }
-      int64_t at = pw[0];
+      int at = pw[0];
 #pragma unroll
       for (int qq = 0; qq < R; ++qq)
         if (q == qq) at = p < a.sec_t ? pt[qq] : (p < a.sec_th ? ph[qq] : pw[qq]);
@@ -157,8 +161,8 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
 
 #pragma unroll
     for (int q = 0; q < R; ++q) {
-      const int64_t row = begin + it * R + q;
-      if (row < end) {
+      const int j = it * R + q;
+      if (j < count) {
         // cs[m] = (cos of pair p0+2m, cos of pair p0+2m+1); likewise sn
         float2 cs[Q], sn[Q];
 #pragma unroll
@@ -179,7 +183,7 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
             c1[m] = mul2(god[part][m], cs[m]);
           }
           uint4 *dst =
-              reinterpret_cast<uint4 *>((part == 0 ? qo : ko) + row * a.ld_out_bytes) + tid;
+              reinterpret_cast<uint4 *>((part == 0 ? qo_c : ko_c) + j * a.ld_out_bytes) + tid;
 #pragma unroll
           for (int k = 0; k < VPT; ++k) {
             // every lane joins the shuffles; ok[] only guards memory accesses

@@ -23,6 +23,36 @@
 namespace sol {
 namespace {
 
+// Widen the modulation of (sample, modality) `key` to fp32:
+// fac = gamma * (1 + scale), sh = shift, for this thread's slots.
+template <typename T, int NT, int VPT>
+__device__ __forceinline__ void load_modulation(const RmsArgs &a, int key, int tid,
+                                                const bool (&ok)[VPT],
+                                                float2 (&fac)[VPT][Io<T>::E / 2],
+                                                float2 (&sh)[VPT][Io<T>::E / 2]) {
+  using IO = Io<T>;
+  constexpr int P = IO::E / 2;
+  const int64_t koff = static_cast<int64_t>(key) * a.nvec + tid;
+  const uint4 *s0 = static_cast<const uint4 *>(a.scale) + koff;
+  const uint4 *h0 = static_cast<const uint4 *>(a.shift) + koff;
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    if (ok[k]) {
+      float2 sc[P];
+      IO::unpack(ld_shared_vec(s0 + k * NT), sc);
+      IO::unpack(ld_shared_vec(h0 + k * NT), sh[k]);
+#pragma unroll
+      for (int m = 0; m < P; ++m) fac[k][m] = add2(sc[m], splat2(1.f));
+      if (a.gamma) {
+        float2 g[P];
+        IO::unpack(ld_shared_vec(static_cast<const uint4 *>(a.gamma) + k * NT + tid), g);
+#pragma unroll
+        for (int m = 0; m < P; ++m) fac[k][m] = mul2(fac[k][m], g[m]);
+      }
+    }
+  }
+}
+
 template <typename T, int NT, int VPT, int R, int S>
 __global__ void __launch_bounds__(NT) rms_adaln_kernel(const RmsArgs a) {
   using IO = Io<T>;
@@ -46,18 +76,21 @@ __global__ void __launch_bounds__(NT) rms_adaln_kernel(const RmsArgs a) {
   for (int i = tid; i < 2 * R * 32; i += NT) red[i] = 0.f;  // unused warp slots read 0
   __syncthreads();
 
-  int64_t begin, end;
-  cta_rows(a.rows, blockIdx.x, gridDim.x, begin, end);
-  const int64_t iters = (end - begin + R - 1) / R;
+  int64_t begin;
+  int count;  // rows of this CTA's share, walked with local index j
+  cta_rows(a.rows, blockIdx.x, gridDim.x, begin, count);
+  const int iters = (count + R - 1) / R;
+  const unsigned char *xc = xb + begin * row_bytes;
+  unsigned char *yc = yb + begin * row_bytes;
 
   // Copy this thread's slots of iteration `it`'s rows into ring stage s;
   // always commits a group (possibly empty) so the group count is uniform.
-  auto issue = [&](int64_t it, int s) {
+  auto issue = [&](int it, int s) {
 #pragma unroll
     for (int q = 0; q < R; ++q) {
-      const int64_t row = begin + it * R + q;
-      if (it < iters && row < end) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(xb + row * row_bytes) + tid;
+      const int j = it * R + q;
+      if (j < count) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(xc + j * row_bytes) + tid;
 #pragma unroll
         for (int k = 0; k < VPT; ++k)
           if (ok[k]) cp_async16(&ring[((s * R + q) * VPT + k) * NT + tid], src + k * NT);
@@ -70,13 +103,13 @@ __global__ void __launch_bounds__(NT) rms_adaln_kernel(const RmsArgs a) {
   for (int s = 0; s < S - 1; ++s) issue(s, s);
 
   float2 fac[VPT][P], sh[VPT][P];  // gamma*(1+scale) and shift of `key`
-  int64_t key = -1;                // 2*b + m those belong to
+  int key = -1;                    // 2*b + m those belong to
   int cons = 0;                    // ring stage of iteration `it`
   int buf = 0;                     // which half of `red`
   TokenCursor cur;
   cur.init(begin, a.L);
 
-  for (int64_t it = 0; it < iters; ++it) {
+  for (int it = 0; it < iters; ++it) {
     issue(it + S - 1, cons == 0 ? S - 1 : cons - 1);
     cp_async_wait<S - 1>();
 
@@ -115,40 +148,67 @@ __global__ void __launch_bounds__(NT) rms_adaln_kernel(const RmsArgs a) {
       buf ^= 1;
     }
 
+    float2 inv2[R];
 #pragma unroll
-    for (int q = 0; q < R; ++q) {
-      const int64_t row = begin + it * R + q;
-      if (row < end) {
-        const int64_t nkey = 2 * cur.b + (cur.r >= a.n_video ? 1 : 0);
-        if (nkey != key) {
-          key = nkey;
-          const uint4 *s0 = static_cast<const uint4 *>(a.scale) + key * a.nvec + tid;
-          const uint4 *h0 = static_cast<const uint4 *>(a.shift) + key * a.nvec + tid;
+    for (int q = 0; q < R; ++q) inv2[q] = splat2(rsqrtf(fmaf(tot[q], a.inv_D, a.eps)));
+
+    // Fast path: every row of this iteration uses the cached modulation.
+    const int nrows = count - it * R < R ? count - it * R : R;
+    bool same = true;
+    {
+      TokenCursor c = cur;
+#pragma unroll
+      for (int q = 0; q < R; ++q) {
+        if (q < nrows) same &= (2 * c.b + (c.r >= a.n_video ? 1 : 0)) == key;
+        c.next(a.L);
+      }
+    }
+    if (same) {
+#pragma unroll
+      for (int q = 0; q < R; ++q) {
+        if (q < nrows) {
+          uint4 *yrow = reinterpret_cast<uint4 *>(yc + (it * R + q) * row_bytes) + tid;
 #pragma unroll
           for (int k = 0; k < VPT; ++k) {
             if (ok[k]) {
-              float2 sc[P];
-              IO::unpack(ld_shared_vec(s0 + k * NT), sc);
-              IO::unpack(ld_shared_vec(h0 + k * NT), sh[k]);
+              float2 o[P];
 #pragma unroll
-              for (int m = 0; m < P; ++m) fac[k][m] = add2(sc[m], splat2(1.f));
-              if (a.gamma) {
-                float2 g[P];
-                IO::unpack(ld_shared_vec(static_cast<const uint4 *>(a.gamma) + k * NT + tid), g);
-#pragma unroll
-                for (int m = 0; m < P; ++m) fac[k][m] = mul2(fac[k][m], g[m]);
-              }
+              for (int m = 0; m < P; ++m)
+                o[m] = fma2(xp[q][k][m], mul2(fac[k][m], inv2[q]), sh[k][m]);
+              st_stream16(yrow + k * NT, IO::pack(o));
             }
           }
+          cur.next(a.L);
         }
-        const float2 inv2 = splat2(rsqrtf(fmaf(tot[q], a.inv_D, a.eps)));
-        uint4 *yrow = reinterpret_cast<uint4 *>(yb + row * row_bytes) + tid;
+      }
+    } else {
+      // A modality or sample boundary falls in this iteration: reload the
+      // modulation row by row (at most a few times per CTA).
+#pragma unroll 1
+      for (int q = 0; q < nrows; ++q) {
+        const int nkey = 2 * cur.b + (cur.r >= a.n_video ? 1 : 0);
+        if (nkey != key) {
+          key = nkey;
+          load_modulation<T, NT, VPT>(a, key, tid, ok, fac, sh);
+        }
+        uint4 *yrow = reinterpret_cast<uint4 *>(yc + (it * R + q) * row_bytes) + tid;
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
           if (ok[k]) {
             float2 o[P];
 #pragma unroll
-            for (int m = 0; m < P; ++m) o[m] = fma2(xp[q][k][m], mul2(fac[k][m], inv2), sh[k][m]);
+            for (int m = 0; m < P; ++m) {
+              // q is not a compile-time index here: select the row's values
+              float2 x = xp[0][k][m];
+#pragma unroll
+              for (int qq = 1; qq < R; ++qq)
+                if (q == qq) x = xp[qq][k][m];
+              float2 iv = inv2[0];
+#pragma unroll
+              for (int qq = 1; qq < R; ++qq)
+                if (q == qq) iv = inv2[qq];
+              o[m] = fma2(x, mul2(fac[k][m], iv), sh[k][m]);
+            }
             st_stream16(yrow + k * NT, IO::pack(o));
           }
         }

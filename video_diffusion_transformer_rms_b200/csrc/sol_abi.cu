@@ -168,6 +168,8 @@ sol_status sol_rms_adaln(const void *x, void *y, const void *scale, const void *
                 "(B=%lld L=%lld n_video=%lld D=%lld)",
                 (long long)B, (long long)L, (long long)n_video, (long long)D);
   if (!(eps >= 0.f)) return fail(SOL_ERR_INVALID_ARG, "sol_rms_adaln: eps must be >= 0");
+  if (B > kMaxRows || L > kMaxRows || B * L > kMaxRows)
+    return fail(SOL_ERR_UNSUPPORTED, "sol_rms_adaln: B*L must be below 2^31 rows");
   const int64_t rows = B * L;
   if (rows == 0) return ok();
   if (!x || !y || !scale || !shift)
@@ -198,8 +200,8 @@ sol_status sol_rms_adaln(const void *x, void *y, const void *scale, const void *
   a.shift = shift;
   a.gamma = gamma;
   a.rows = rows;
-  a.L = L;
-  a.n_video = n_video;
+  a.L = static_cast<int>(L);
+  a.n_video = static_cast<int>(n_video);
   a.nvec = static_cast<int>(row_bytes / 16);
   a.eps = eps;
   a.inv_D = static_cast<float>(1.0 / static_cast<double>(D));
@@ -218,6 +220,8 @@ sol_status sol_gate_residual(const void *h, const void *branch, const void *gate
                 "sol_gate_residual: need B >= 0, L >= 0, D > 0, 0 <= n_video <= L "
                 "(B=%lld L=%lld n_video=%lld D=%lld)",
                 (long long)B, (long long)L, (long long)n_video, (long long)D);
+  if (B > kMaxRows || L > kMaxRows || B * L > kMaxRows)
+    return fail(SOL_ERR_UNSUPPORTED, "sol_gate_residual: B*L must be below 2^31 rows");
   const int64_t rows = B * L;
   if (rows == 0) return ok();
   if (!h || !branch || !gate || !out)
@@ -246,8 +250,8 @@ sol_status sol_gate_residual(const void *h, const void *branch, const void *gate
   a.gate = gate;
   a.out = out;
   a.rows = rows;
-  a.L = L;
-  a.n_video = n_video;
+  a.L = static_cast<int>(L);
+  a.n_video = static_cast<int>(n_video);
   a.nvec = static_cast<int>(row_bytes / 16);
   cudaError_t e = launch_gate_residual(a, dtype == SOL_F32 ? 0 : 1, stream, nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "sol_gate_residual launch");
@@ -273,6 +277,10 @@ sol_status sol_qknorm_rope3d(const void *qkv, int64_t ld_qkv, void *q_out, void 
                 (long long)sec_t, (long long)sec_h, (long long)sec_w, (long long)(head_dim / 2));
   if (!(eps >= 0.f) || !(theta > 0.f))
     return fail(SOL_ERR_INVALID_ARG, "sol_qknorm_rope3d: need eps >= 0 and theta > 0");
+  if (T > kMaxRows || H > kMaxRows || W > kMaxRows || n_audio > kMaxRows || B > kMaxRows ||
+      H * W > kMaxRows || T * H * W > kMaxRows || T * H * W + n_audio > kMaxRows ||
+      B * (T * H * W + n_audio) > kMaxRows)
+    return fail(SOL_ERR_UNSUPPORTED, "sol_qknorm_rope3d: B*L and H*W must be below 2^31");
   const int64_t n_video = T * H * W;
   const int64_t L = n_video + n_audio;
   const int64_t rows = B * L;
@@ -326,11 +334,11 @@ sol_status sol_qknorm_rope3d(const void *qkv, int64_t ld_qkv, void *q_out, void 
   a.ld_qkv_bytes = ldq_b;
   a.ld_out_bytes = ldo_b;
   a.rows = rows;
-  a.L = L;
-  a.n_video = n_video;
-  a.HW = H * W;
-  a.H = H;
-  a.W = W;
+  a.L = static_cast<int>(L);
+  a.n_video = static_cast<int>(n_video);
+  a.HW = static_cast<int>(H * W);
+  a.H = static_cast<int>(H);
+  a.W = static_cast<int>(W);
   a.nvec_q = static_cast<int>(D_b / 16);
   a.npairs = static_cast<int>(head_dim / 2);
   a.sec_t = static_cast<int>(sec_t);

@@ -152,23 +152,24 @@ __device__ __forceinline__ float group_sum(float v) {
 // row bookkeeping
 // ---------------------------------------------------------------------------
 
-// Contiguous share [begin, end) of `rows` for CTA `cta` out of `ctas`; the
-// shares differ by at most one row.
+// Contiguous share [begin, begin + count) of `rows` for CTA `cta` out of
+// `ctas`; the shares differ by at most one row.  A share is walked with a
+// 32-bit local row index (the host rejects sizes that would overflow it).
 __device__ __forceinline__ void cta_rows(int64_t rows, int64_t cta, int64_t ctas,
-                                         int64_t &begin, int64_t &end) {
+                                         int64_t &begin, int &count) {
   begin = rows * cta / ctas;
-  end = rows * (cta + 1) / ctas;
+  count = static_cast<int>(rows * (cta + 1) / ctas - begin);
 }
 
 // (sample b, row r in the sample) of a global row, advanced one row at a
-// time: one division per CTA instead of one per row.
+// time: one division per CTA instead of one per row.  L < 2^31.
 struct TokenCursor {
-  int64_t b, r;
-  __device__ __forceinline__ void init(int64_t row, int64_t L) {
-    b = row / L;
-    r = row - b * L;
+  int b, r;
+  __device__ __forceinline__ void init(int64_t row, int L) {
+    b = static_cast<int>(row / L);
+    r = static_cast<int>(row - static_cast<int64_t>(b) * L);
   }
-  __device__ __forceinline__ void next(int64_t L) {
+  __device__ __forceinline__ void next(int L) {
     if (++r == L) {
       r = 0;
       ++b;
@@ -180,11 +181,11 @@ struct TokenCursor {
 // rows r < n_video walk the T x H x W grid in raster order (t-major), audio
 // row i = r - n_video sits at (i, 0, 0).
 struct GridCursor {
-  int64_t t, h, w;
-  __device__ __forceinline__ void init(int64_t r, int64_t n_video, int64_t HW, int64_t W) {
+  int t, h, w;
+  __device__ __forceinline__ void init(int r, int n_video, int HW, int W) {
     if (r < n_video) {
       t = r / HW;
-      const int64_t rem = r - t * HW;
+      const int rem = r - t * HW;
       h = rem / W;
       w = rem - h * W;
     } else {
@@ -194,7 +195,7 @@ struct GridCursor {
     }
   }
   // Move to row r_next (= r + 1, or 0 when a new sample starts).
-  __device__ __forceinline__ void next(int64_t r_next, int64_t n_video, int64_t H, int64_t W) {
+  __device__ __forceinline__ void next(int r_next, int n_video, int H, int W) {
     if (r_next == 0 || r_next == n_video) {
       t = 0;
       h = 0;

@@ -46,8 +46,8 @@ struct RmsArgs {
   const void *shift;
   const void *gamma;  // may be null
   int64_t rows;       // B * L
-  int64_t L;
-  int64_t n_video;
+  int L;              // < 2^31
+  int n_video;
   int nvec;           // 16-byte vectors per row
   float eps;
   float inv_D;
@@ -59,8 +59,8 @@ struct GateArgs {
   const void *gate;
   void *out;
   int64_t rows;
-  int64_t L;
-  int64_t n_video;
+  int L;
+  int n_video;
   int nvec;
 };
 
@@ -73,11 +73,11 @@ struct QkArgs {
   int64_t ld_qkv_bytes;
   int64_t ld_out_bytes;
   int64_t rows;       // B * L
-  int64_t L;
-  int64_t n_video;    // T * H * W
-  int64_t HW;         // H * W
-  int64_t H;
-  int64_t W;
+  int L;              // < 2^31
+  int n_video;        // T * H * W
+  int HW;             // H * W
+  int H;
+  int W;
   int nvec_q;         // 16-byte vectors in q (and in k) of one row
   int npairs;         // head_dim / 2
   int sec_t;          // pairs on the t axis
@@ -103,6 +103,7 @@ inline cudaError_t launch_qknorm_rope3d(const QkArgs &a, int dtype, cudaStream_t
 
 // Limits the launchers accept (checked by the ABI before calling them).
 constexpr int kMaxThreads = 256;
+constexpr int64_t kMaxRows = 0x7fffffff;  // B*L, L, H*W: 32-bit row bookkeeping
 constexpr int kMaxVpt = 8;
 constexpr int64_t kMaxRowBytesRms = 32768;   // D * esize for RMS-AdaLN
 constexpr int64_t kMaxRowBytesGate = 32768;  // D * esize for the gated residual
