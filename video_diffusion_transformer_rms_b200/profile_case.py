@@ -1,0 +1,52 @@
+"""Run each hot-path kernel a few times on a seeded slice of a clip workload,
+for profilers (ncu) that should capture a small, self-contained case.
+
+    python -m video_diffusion_transformer_rms_b200.profile_case \
+        [--workload clip5s] [--frames 4] [--launches 1]
+
+The slice keeps the clip's H x W latent grid, D and head layout, takes the
+first `--frames` latent frames (T) and scales the audio rows by the same
+fraction.  Inputs are larger than L2 at the default 4 frames (16,384 rows:
+168 MB per activation, 503 MB of merged QKV), so DRAM counters stay
+meaningful while the device footprint stays near 1.5 GB.
+"""
+import argparse
+import dataclasses
+
+import torch
+
+from . import api
+from .workloads import WORKLOADS, make_inputs
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="clip5s", choices=sorted(WORKLOADS))
+    ap.add_argument("--frames", type=int, default=4)
+    ap.add_argument("--launches", type=int, default=1)
+    args = ap.parse_args()
+    full = WORKLOADS[args.workload]
+    T = max(1, min(full.T, args.frames))
+    n_audio = full.n_audio * T // full.T
+    w = dataclasses.replace(full, name=f"{full.name}_slice{T}", T=T, n_audio=n_audio)
+    t = make_inputs(w, "cuda")
+    D = w.D
+    x = t["x"].view(w.B, w.L, D)
+    h = t["h"].view(w.B, w.L, D)
+    br = t["branch"].view(w.B, w.L, D)
+    qkv = t["qkv"].view(w.B, w.L, 3 * D)
+    y = torch.empty_like(x)
+    out = torch.empty_like(h)
+    qk = torch.empty((w.B, w.L, 2 * D), dtype=qkv.dtype, device=qkv.device)
+    for _ in range(args.launches):
+        api.rms_adaln(x, t["scale"], t["shift"], w.n_video, eps=w.eps, out=y)
+        api.qknorm_rope3d(qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections,
+                          t["gamma_q"], t["gamma_k"], w.eps, w.theta, q_out=qk[..., :D],
+                          k_out=qk[..., D:])
+        api.gate_residual(h, br, t["gate"], w.n_video, out=out)
+    torch.cuda.synchronize()
+    print(f"{w.name}: {w.rows} rows, D={D}, {args.launches} launch(es) of each kernel")
+
+
+if __name__ == "__main__":
+    main()
