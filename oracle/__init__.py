@@ -35,6 +35,9 @@ def _load():
         lib.oracle_rms_adaln.restype = i
         lib.oracle_gate_residual.argtypes = [p, p, p, p, i64, i64, i64, i64, i, p]
         lib.oracle_gate_residual.restype = i
+        lib.oracle_gate_residual_rms_adaln.argtypes = [p, p, p, p, p, p, p, i64, i64, i64, i64,
+                                                       d, i, p, p]
+        lib.oracle_gate_residual_rms_adaln.restype = i
         lib.oracle_qknorm_rope3d.argtypes = [p, i64, p, p, p, i64, i64, i64, i64,
                                              i64, i64, i64, i64, i64, i64, d, d,
                                              i, p, p]
@@ -105,6 +108,25 @@ def gate_residual(h, branch, gate, L, n_video, row_ids=None):
     if rc != 0:
         raise ValueError("oracle_gate_residual rejected its arguments")
     return out.reshape(h.shape)
+
+
+def gate_residual_rms_adaln(h, branch, gate, scale, shift, L, n_video, eps, gamma=None,
+                            row_ids=None):
+    """h, branch: [n_rows, D]; gate, scale, shift: [B, 2, D]; returns (h_out, y)."""
+    h, branch, gate, scale, shift, gamma = (_c(a) for a in (h, branch, gate, scale, shift, gamma))
+    D = h.shape[-1]
+    h2, b2 = h.reshape(-1, D), branch.reshape(-1, D)
+    rid, n = _rows(row_ids, h2.shape[0])
+    if n != h2.shape[0] or b2.shape != h2.shape:
+        raise ValueError("h, branch and row_ids must agree")
+    h_out = np.empty((n, D), dtype=np.float64)
+    y = np.empty((n, D), dtype=np.float64)
+    rc = _load().oracle_gate_residual_rms_adaln(
+        _ptr(h2), _ptr(b2), _ptr(gate), _ptr(scale), _ptr(shift), _ptr(gamma), _ptr(rid), n, L,
+        n_video, D, eps, _dtype_code(h, branch, gate, scale, shift, gamma), _ptr(h_out), _ptr(y))
+    if rc != 0:
+        raise ValueError("oracle_gate_residual_rms_adaln rejected its arguments")
+    return h_out.reshape(h.shape), y.reshape(h.shape)
 
 
 def qknorm_rope3d(qkv, T, H, W, n_audio, n_heads, head_dim, sections, eps, theta,

@@ -144,6 +144,52 @@ int oracle_gate_residual(const void *h, const void *branch, const void *gate,
 }
 
 /*
+ * Gated residual followed by RMS-AdaLN of its result, the chain
+ * "h = h + gate1 * attn; x2 = RMS-AdaLN(h)" of the DiT block.  For each
+ * given row (sample b, row r, modality m):
+ *   hn[c]  = h[c] + gate[b, m, c] * branch[c]          (kept in fp64)
+ *   ms     = (1/D) * sum_c hn[c]^2
+ *   y[c]   = hn[c] / sqrt(ms + eps) * gamma[c] * (1 + scale[b, m, c])
+ *            + shift[b, m, c]
+ * Outputs hn (h_out) and y, both [n_rows, D] doubles; the normalisation
+ * reads hn unrounded.
+ */
+int oracle_gate_residual_rms_adaln(const void *h, const void *branch, const void *gate,
+                                   const void *scale, const void *shift, const void *gamma,
+                                   const int64_t *row_ids, int64_t n_rows, int64_t L,
+                                   int64_t n_video, int64_t D, double eps, int dtype,
+                                   double *h_out, double *y)
+{
+    if (n_rows < 0 || L <= 0 || D <= 0 || n_video < 0 || n_video > L)
+        return -1;
+    for (int64_t k = 0; k < n_rows; ++k) {
+        int64_t g = row_id(row_ids, k);
+        int64_t b = g / L;
+        int64_t r = g % L;
+        int64_t m = (r < n_video) ? 0 : 1;
+        int64_t mod = (b * 2 + m) * D;
+
+        double ss = 0.0;
+        for (int64_t c = 0; c < D; ++c) {
+            double hv = in_val(h, k * D + c, dtype);
+            double bv = in_val(branch, k * D + c, dtype);
+            double hn = hv + in_val(gate, mod + c, dtype) * bv;
+            h_out[k * D + c] = hn;
+            ss += hn * hn;
+        }
+        double denom = sqrt(ss / (double)D + eps);
+        for (int64_t c = 0; c < D; ++c) {
+            double n = h_out[k * D + c] / denom;
+            if (gamma)
+                n = n * in_val(gamma, c, dtype);
+            y[k * D + c] = n * (1.0 + in_val(scale, mod + c, dtype)) +
+                           in_val(shift, mod + c, dtype);
+        }
+    }
+    return 0;
+}
+
+/*
  * Position of row r of a sample on the three rotary axes.
  * Video rows r < T*H*W are the latent grid in raster order, t-major:
  *   t = r / (H*W), h = (r / W) mod H, w = r mod W.

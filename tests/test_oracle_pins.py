@@ -408,3 +408,50 @@ def test_ulp_values():
     np.testing.assert_array_equal(oracle.ulp([1.0, 0.1], oracle.F32),
                                   [2.0 ** -23, 2.0 ** -27])
     assert oracle.tolerance(0.0, oracle.BF16) == pytest.approx(1e-3)
+
+
+# ----------------------------------------------------------------------------
+# Fused gated residual + RMS-AdaLN
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("conv", [f32, bf16_bits], ids=["f32", "bf16"])
+def test_fused_residual_norm_hand_worked(conv):
+    h = _hand()
+    hh = conv(np.stack([h["fused_h0"], h["fused_h1"]]))
+    br = conv(np.stack([h["fused_b0"], h["fused_b1"]]))
+    gate = conv(np.stack([h["fused_gate_video"], h["fused_gate_audio"]])[None])
+    scale = conv(np.stack([h["scale_video"], h["scale_audio"]])[None])
+    shift = conv(np.stack([h["shift_video"], h["shift_audio"]])[None])
+    h_out, y = oracle.gate_residual_rms_adaln(hh, br, gate, scale, shift, L=2, n_video=1,
+                                              eps=0.0)
+    np.testing.assert_array_equal(h_out[0], h["fused_hout0"])
+    np.testing.assert_array_equal(h_out[1], h["fused_hout1"])
+    np.testing.assert_allclose(y[0], h["y0"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(y[1], h["y1"], rtol=0, atol=1e-14)
+    _, yg = oracle.gate_residual_rms_adaln(hh, br, gate, scale, shift, L=2, n_video=1, eps=0.0,
+                                           gamma=conv(h["gamma"]))
+    np.testing.assert_allclose(yg[0], h["y0_gamma"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(yg[1], h["y1_gamma"], rtol=0, atol=1e-14)
+
+
+def test_fused_residual_norm_closed_forms():
+    # gate = 0: h_out is h exactly; with scale = shift = 0 and eps = 0 the
+    # output has unit RMS; with scale = -1 the output is the shift.
+    B, L, nv, D = 2, 5, 3, 32
+    hh = f32(RNG.standard_normal((B * L, D)))
+    br = f32(RNG.standard_normal((B * L, D)))
+    z = f32(np.zeros((B, 2, D)))
+    h_out, y = oracle.gate_residual_rms_adaln(hh, br, z, z, z, L=L, n_video=nv, eps=0.0)
+    np.testing.assert_array_equal(h_out, hh.astype(np.float64))
+    np.testing.assert_allclose(np.sqrt(np.mean(y ** 2, axis=1)), 1.0, rtol=1e-13)
+    g = f32(RNG.standard_normal((B, 2, D)))
+    shift = f32(np.array([[[10 * b + m + 1] * D for m in range(2)] for b in range(B)]))
+    _, y = oracle.gate_residual_rms_adaln(hh, br, g, f32(np.full((B, 2, D), -1.0)), shift,
+                                          L=L, n_video=nv, eps=1e-6)
+    for row in range(B * L):
+        b, r = divmod(row, L)
+        assert np.all(y[row] == 10 * b + (0 if r < nv else 1) + 1)
+    # h_out is linear in the gate: h_out(2g) - h_out(g) == h_out(g) - h_out(0)
+    h1, _ = oracle.gate_residual_rms_adaln(hh, br, g, z, z, L=L, n_video=nv, eps=1e-6)
+    h2, _ = oracle.gate_residual_rms_adaln(hh, br, f32(2 * g), z, z, L=L, n_video=nv, eps=1e-6)
+    np.testing.assert_allclose(h2 - h1, h1 - hh.astype(np.float64), rtol=1e-12, atol=1e-12)
