@@ -114,6 +114,33 @@ sol_status sol_gate_residual(const void *h, const void *branch,
                              sol_stream_t stream);
 
 /*
+ * Fused AdaLN-gated residual + RMS-AdaLN: the block's "h = h + gate * attn;
+ * x = RMS-AdaLN(h)" chain in one pass (the pages' "leftover elementwise
+ * chains" of the torch.compile row fused into the "fused RMS-AdaLN" row of
+ * the Sol Video Inference Engine MiniMax-H3 fusion table).  For every row of
+ * sample b with modality m:
+ *
+ *   h_out[c] = h[c] + gate[b][m][c] * branch[c]
+ *   y[c]     = h_out[c] / sqrt(mean_c(h_out^2) + eps) * gamma[c]
+ *              * (1 + scale[b][m][c]) + shift[b][m][c]
+ *
+ * The normalisation reads h_out before it is rounded to the I/O type.  HBM
+ * traffic per row is 4*D elements instead of 5*D for sol_gate_residual
+ * followed by sol_rms_adaln.
+ *
+ *   h, branch, h_out, y  [B, L, D] device, contiguous.  h_out may equal h
+ *                        (in place); y must not overlap any other argument.
+ *   gate, scale, shift   [B, 2, D] device.
+ *   gamma, n_video, D, eps  as for sol_rms_adaln (same D limit).
+ */
+sol_status sol_gate_residual_rms_adaln(const void *h, const void *branch,
+                                       const void *gate, void *h_out, void *y,
+                                       const void *scale, const void *shift,
+                                       const void *gamma, int64_t B, int64_t L,
+                                       int64_t n_video, int64_t D, float eps,
+                                       sol_dtype dtype, sol_stream_t stream);
+
+/*
  * Fused per-head QKNorm + 3D multimodal RoPE on a merged QKV projection
  * (fusion table of the Sol Video Inference Engine MiniMax-H3 page, rows
  * "fused QKNorm + RoPE" and "QKV merge"; RoPE of Su et al., RoFormer).

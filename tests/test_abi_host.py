@@ -18,6 +18,7 @@ def built():
 def test_header_declares_the_entry_points():
     syms = _abi.header_symbols()
     for name in ("sol_rms_adaln", "sol_gate_residual", "sol_qknorm_rope3d",
+                 "sol_gate_residual_rms_adaln",
                  "sol_status_string", "sol_last_error", "sol_version"):
         assert name in syms
 
@@ -105,6 +106,35 @@ def test_zero_rows_is_a_noop_even_with_null_pointers():
 ])
 def test_gate_residual_rejects(kw, status):
     assert gate(**kw) == status
+
+
+def fused(h=A, br=A + (1 << 30), g=A + (2 << 30), ho=A + (3 << 30), y=A + (4 << 30),
+          sc=A + (5 << 30), sh=A + (6 << 30), gm=None, B=1, L=4, nv=2, D=64, eps=1e-6, dt=BF):
+    return _abi.sol_gate_residual_rms_adaln(h, br, g, ho, y, sc, sh, gm, B, L, nv, D, eps, dt,
+                                            None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(y=None), _abi.SOL_ERR_INVALID_ARG),
+    (dict(sh=None), _abi.SOL_ERR_INVALID_ARG),
+    (dict(nv=5), _abi.SOL_ERR_INVALID_ARG),
+    (dict(eps=-1.0), _abi.SOL_ERR_INVALID_ARG),
+    (dict(D=36), _abi.SOL_ERR_MISALIGNED),
+    (dict(gm=A + (7 << 30) + 8), _abi.SOL_ERR_MISALIGNED),
+    (dict(D=16392), _abi.SOL_ERR_UNSUPPORTED),
+    (dict(B=1 << 20, L=1 << 12), _abi.SOL_ERR_UNSUPPORTED),
+    (dict(ho=A + 64), _abi.SOL_ERR_INVALID_ARG),            # partial overlap with h
+    (dict(ho=A + (1 << 30)), _abi.SOL_ERR_INVALID_ARG),     # h_out on branch
+    (dict(y=A), _abi.SOL_ERR_INVALID_ARG),                  # y on h
+    (dict(y=A + (3 << 30)), _abi.SOL_ERR_INVALID_ARG),      # y on h_out
+    (dict(y=A + (5 << 30)), _abi.SOL_ERR_INVALID_ARG),      # y on scale
+])
+def test_gate_residual_rms_adaln_rejects(kw, status):
+    assert fused(**kw) == status
+
+
+def test_gate_residual_rms_adaln_zero_rows_noop():
+    assert fused(h=None, y=None, B=0) == _abi.SOL_OK
 
 
 @pytest.mark.parametrize("kw,status", [

@@ -208,6 +208,89 @@ def test_gate_residual_in_place_zero_gate_and_guards():
 
 
 # ----------------------------------------------------------------------------
+# Fused gated residual + RMS-AdaLN
+# ----------------------------------------------------------------------------
+
+def _check_fused(h2, b2, gate, sc, sh, L, nv, eps, gamma, ho2, y2, what, ids=None):
+    if ids is None:
+        wh, wy = oracle.gate_residual_rms_adaln(_o(h2), _o(b2), _o(gate), _o(sc), _o(sh), L, nv,
+                                                eps, gamma=None if gamma is None else _o(gamma))
+        assert_close(ho2, wh, f"{what} h_out")
+        assert_close(y2, wy, f"{what} y")
+    else:
+        wh, wy = oracle.gate_residual_rms_adaln(take_rows(h2, ids), take_rows(b2, ids), _o(gate),
+                                                _o(sc), _o(sh), L, nv, eps,
+                                                gamma=None if gamma is None else _o(gamma),
+                                                row_ids=ids)
+        assert_close(take_rows_gpu(ho2, ids), wh, f"{what} h_out sampled")
+        assert_close(take_rows_gpu(y2, ids), wy, f"{what} y sampled")
+
+
+@pytest.mark.parametrize("name", SMALL + ("clip5s", "cfg5s", "cfg5s_d3072"))
+@pytest.mark.parametrize("with_gamma", [False, True])
+def test_gate_residual_rms_adaln_workload(name, with_gamma):
+    w = WORKLOADS[name]
+    t = make_inputs(w, DEV, which=("rms_adaln", "gate_residual"), with_gamma=with_gamma)
+    h, br = t["h"].view(w.B, w.L, w.D), t["branch"].view(w.B, w.L, w.D)
+    gamma = t.get("gamma")
+    ho, y = api.gate_residual_rms_adaln(h, br, t["gate"], t["scale"], t["shift"], w.n_video,
+                                        gamma=gamma, eps=w.eps)
+    torch.cuda.synchronize()
+    ids = None if name in SMALL else _ids(w)
+    _check_fused(h.view(-1, w.D), br.view(-1, w.D), t["gate"], t["scale"], t["shift"], w.L,
+                 w.n_video, w.eps, gamma, ho.view(-1, w.D), y.view(-1, w.D), f"fused[{name}]",
+                 ids)
+
+
+@pytest.mark.parametrize("B,L,nv,D,dt", RMS_SHAPES)
+def test_gate_residual_rms_adaln_shapes(B, L, nv, D, dt):
+    h = activation(B * L, D, dt, DEV, 41, outliers=True).view(B, L, D)
+    br = activation(B * L, D, dt, DEV, 42, outliers=True).view(B, L, D)
+    g = vectors((B, 2, D), 0.0, 0.1, dt, DEV, 43)
+    _, sc, sh, gm = _rand_rms(1, 1, D, dt, seed=44)
+    sc = vectors((B, 2, D), 0.0, 0.5, dt, DEV, 45)
+    sh = vectors((B, 2, D), 0.0, 0.5, dt, DEV, 46)
+    for gamma in (None, gm):
+        ho, y = api.gate_residual_rms_adaln(h, br, g, sc, sh, nv, gamma=gamma)
+        _check_fused(h.view(-1, D), br.view(-1, D), g, sc, sh, L, nv, 1e-6, gamma,
+                     ho.view(-1, D), y.view(-1, D), f"fused B={B} L={L} D={D}")
+
+
+def test_gate_residual_rms_adaln_in_place_and_guards():
+    B, L, nv, D = 2, 601, 555, 5120
+    dt = torch.bfloat16
+    h = activation(B * L, D, dt, DEV, 51, outliers=True).view(B, L, D)
+    br = activation(B * L, D, dt, DEV, 52, outliers=True).view(B, L, D)
+    g = vectors((B, 2, D), 0.0, 0.1, dt, DEV, 53)
+    sc = vectors((B, 2, D), 0.0, 0.5, dt, DEV, 54)
+    sh = vectors((B, 2, D), 0.0, 0.5, dt, DEV, 55)
+    wh, wy = oracle.gate_residual_rms_adaln(_o(h.view(-1, D)), _o(br.view(-1, D)), _o(g), _o(sc),
+                                            _o(sh), L, nv, 1e-6)
+    # residual stream updated in place
+    hi = h.clone()
+    _, y = api.gate_residual_rms_adaln(hi, br, g, sc, sh, nv, h_out=hi)
+    assert_close(hi.view(-1, D), wh, "fused in place h_out")
+    assert_close(y.view(-1, D), wy, "fused in place y")
+    # outputs inside guarded buffers
+    pad = 4096
+    n = B * L * D
+    bh = torch.full((n + 2 * pad,), 3.0, dtype=dt, device=DEV)
+    by = torch.full((n + 2 * pad,), -3.0, dtype=dt, device=DEV)
+    ho, y = api.gate_residual_rms_adaln(h, br, g, sc, sh, nv, h_out=bh[pad:pad + n].view(B, L, D),
+                                        y=by[pad:pad + n].view(B, L, D))
+    torch.cuda.synchronize()
+    assert torch.all(bh[:pad] == 3.0) and torch.all(bh[-pad:] == 3.0)
+    assert torch.all(by[:pad] == -3.0) and torch.all(by[-pad:] == -3.0)
+    assert_close(ho.view(-1, D), wh, "fused guarded h_out")
+    assert_close(y.view(-1, D), wy, "fused guarded y")
+    # gate = 0: h_out is h bit for bit and y equals sol_rms_adaln(h)
+    z = torch.zeros_like(g)
+    ho, y = api.gate_residual_rms_adaln(h, br, z, sc, sh, nv)
+    assert torch.equal(ho, h)
+    assert torch.equal(y, api.rms_adaln(h, sc, sh, nv))
+
+
+# ----------------------------------------------------------------------------
 # QKNorm + 3D RoPE
 # ----------------------------------------------------------------------------
 

@@ -9,7 +9,8 @@ per-head QKNorm + 3D multimodal RoPE, as CUDA kernels behind a C ABI
 The CUDA library is loaded on first use and must be built; there is no CPU
 path.
 """
-from ._abi import (SOL_BF16, SOL_F32, SolError, sol_gate_residual, sol_last_error,  # noqa: F401
-                   sol_qknorm_rope3d, sol_rms_adaln, sol_status_string, sol_version)
+from ._abi import (SOL_BF16, SOL_F32, SolError, sol_gate_residual,  # noqa: F401
+                   sol_gate_residual_rms_adaln, sol_last_error, sol_qknorm_rope3d,
+                   sol_rms_adaln, sol_status_string, sol_version)
 
 __version__ = "1.0"

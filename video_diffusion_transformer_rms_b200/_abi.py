@@ -52,6 +52,9 @@ def lib() -> ctypes.CDLL:
         L.sol_rms_adaln.restype = i
         L.sol_gate_residual.argtypes = [p, p, p, p, i64, i64, i64, i64, i, p]
         L.sol_gate_residual.restype = i
+        L.sol_gate_residual_rms_adaln.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, f,
+                                                  i, p]
+        L.sol_gate_residual_rms_adaln.restype = i
         L.sol_qknorm_rope3d.argtypes = [p, i64, p, p, i64, p, p, i64, i64, i64, i64, i64,
                                         i64, i64, i64, i64, i64, f, f, i, p]
         L.sol_qknorm_rope3d.restype = i
@@ -91,6 +94,12 @@ def sol_rms_adaln(x, y, scale, shift, gamma, B, L, n_video, D, eps, dtype, strea
 
 def sol_gate_residual(h, branch, gate, out, B, L, n_video, D, dtype, stream) -> int:
     return lib().sol_gate_residual(h, branch, gate, out, B, L, n_video, D, dtype, stream)
+
+
+def sol_gate_residual_rms_adaln(h, branch, gate, h_out, y, scale, shift, gamma, B, L, n_video,
+                                D, eps, dtype, stream) -> int:
+    return lib().sol_gate_residual_rms_adaln(h, branch, gate, h_out, y, scale, shift, gamma, B,
+                                             L, n_video, D, eps, dtype, stream)
 
 
 def sol_qknorm_rope3d(qkv, ld_qkv, q_out, k_out, ld_out, gamma_q, gamma_k, B, T, H, W,

@@ -64,6 +64,26 @@ def gate_residual(h: torch.Tensor, branch: torch.Tensor, gate: torch.Tensor, n_v
     return o
 
 
+def gate_residual_rms_adaln(h: torch.Tensor, branch: torch.Tensor, gate: torch.Tensor,
+                            scale: torch.Tensor, shift: torch.Tensor, n_video: int,
+                            gamma: Optional[torch.Tensor] = None, eps: float = 1e-6,
+                            h_out: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                            stream: Optional[torch.cuda.Stream] = None
+                            ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """h_out = h + gate[b, m] * branch; y = RMS-AdaLN(h_out) with scale/shift;
+    returns (h_out, y).  Pass h_out=h to update the residual stream in place."""
+    if h.dim() != 3 or not h.is_contiguous() or branch.shape != h.shape:
+        raise ValueError("h and branch must be contiguous [B, L, D] tensors of one shape")
+    B, L, D = h.shape
+    ho = torch.empty_like(h) if h_out is None else h_out
+    yo = torch.empty_like(h) if y is None else y
+    _abi.check(_abi.sol_gate_residual_rms_adaln(
+        _ptr(h), _ptr(branch), _ptr(gate), _ptr(ho), _ptr(yo), _ptr(scale), _ptr(shift),
+        _ptr(gamma), B, L, n_video, D, eps, _dtype(h, branch, gate, ho, yo, scale, shift, gamma),
+        _stream(stream)))
+    return ho, yo
+
+
 def qknorm_rope3d(qkv: torch.Tensor, T: int, H: int, W: int, n_audio: int, n_heads: int,
                   head_dim: int, sections: Sequence[int] = (16, 24, 24),
                   gamma_q: Optional[torch.Tensor] = None,

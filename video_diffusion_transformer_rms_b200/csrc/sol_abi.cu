@@ -258,6 +258,73 @@ sol_status sol_gate_residual(const void *h, const void *branch, const void *gate
   return ok();
 }
 
+sol_status sol_gate_residual_rms_adaln(const void *h, const void *branch, const void *gate,
+                                       void *h_out, void *y, const void *scale,
+                                       const void *shift, const void *gamma, int64_t B, int64_t L,
+                                       int64_t n_video, int64_t D, float eps, sol_dtype dtype,
+                                       sol_stream_t stream) {
+  const char *fn = "sol_gate_residual_rms_adaln";
+  if (dtype != SOL_F32 && dtype != SOL_BF16)
+    return fail(SOL_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
+  if (B < 0 || L < 0 || D <= 0 || n_video < 0 || n_video > L)
+    return fail(SOL_ERR_INVALID_ARG,
+                "%s: need B >= 0, L >= 0, D > 0, 0 <= n_video <= L "
+                "(B=%lld L=%lld n_video=%lld D=%lld)",
+                fn, (long long)B, (long long)L, (long long)n_video, (long long)D);
+  if (!(eps >= 0.f)) return fail(SOL_ERR_INVALID_ARG, "%s: eps must be >= 0", fn);
+  if (B > kMaxRows || L > kMaxRows || B * L > kMaxRows)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: B*L must be below 2^31 rows", fn);
+  const int64_t rows = B * L;
+  if (rows == 0) return ok();
+  if (!h || !branch || !gate || !h_out || !y || !scale || !shift)
+    return fail(SOL_ERR_INVALID_ARG,
+                "%s: h, branch, gate, h_out, y, scale and shift must be non-null", fn);
+  const int es = esize_of(dtype);
+  const int64_t row_bytes = D * es;
+  if (row_bytes % 16 != 0)
+    return fail(SOL_ERR_MISALIGNED, "%s: D*%d bytes must be a multiple of 16 (D=%lld)", fn, es,
+                (long long)D);
+  if (!aligned16(h) || !aligned16(branch) || !aligned16(gate) || !aligned16(h_out) ||
+      !aligned16(y) || !aligned16(scale) || !aligned16(shift) || (gamma && !aligned16(gamma)))
+    return fail(SOL_ERR_MISALIGNED, "%s: every pointer must be 16-byte aligned", fn);
+  if (row_bytes > kMaxRowBytesRms)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: D=%lld exceeds %lld elements", fn, (long long)D,
+                (long long)(kMaxRowBytesRms / es));
+  const int64_t act = rows * row_bytes, mod = B * 2 * row_bytes;
+  const Span hs = span_of(h, 1, 0, act), bs = span_of(branch, 1, 0, act),
+             hos = span_of(h_out, 1, 0, act), ys = span_of(y, 1, 0, act);
+  if (!same_or_disjoint(h_out, h, act) || spans_overlap(hos, bs))
+    return fail(SOL_ERR_INVALID_ARG, "%s: h_out must equal h or overlap neither h nor branch",
+                fn);
+  if (spans_overlap(ys, hs) || spans_overlap(ys, bs) || spans_overlap(ys, hos))
+    return fail(SOL_ERR_INVALID_ARG, "%s: y must not overlap h, branch or h_out", fn);
+  for (const Span &o : {hos, ys}) {
+    if (spans_overlap(o, span_of(gate, 1, 0, mod)) || spans_overlap(o, span_of(scale, 1, 0, mod)) ||
+        spans_overlap(o, span_of(shift, 1, 0, mod)) ||
+        (gamma && spans_overlap(o, span_of(gamma, 1, 0, row_bytes))))
+      return fail(SOL_ERR_INVALID_ARG, "%s: an output overlaps gate, scale, shift or gamma", fn);
+  }
+
+  RmsArgs a{};
+  a.x = h;
+  a.y = y;
+  a.scale = scale;
+  a.shift = shift;
+  a.gamma = gamma;
+  a.branch = branch;
+  a.gate = gate;
+  a.h_out = h_out;
+  a.rows = rows;
+  a.L = static_cast<int>(L);
+  a.n_video = static_cast<int>(n_video);
+  a.nvec = static_cast<int>(row_bytes / 16);
+  a.eps = eps;
+  a.inv_D = static_cast<float>(1.0 / static_cast<double>(D));
+  cudaError_t e = launch_gate_residual_rms_adaln(a, dtype == SOL_F32 ? 0 : 1, stream, nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_gate_residual_rms_adaln launch");
+  return ok();
+}
+
 sol_status sol_qknorm_rope3d(const void *qkv, int64_t ld_qkv, void *q_out, void *k_out,
                              int64_t ld_out, const void *gamma_q, const void *gamma_k, int64_t B,
                              int64_t T, int64_t H, int64_t W, int64_t n_audio, int64_t n_heads,

@@ -40,11 +40,14 @@ bool pick_split(int64_t nvec, int *threads, int *vpt);
   X(128, 4) X(128, 5) X(128, 6) X(256, 4) X(256, 5) X(256, 6) X(256, 7) X(256, 8)
 
 struct RmsArgs {
-  const void *x;
+  const void *x;       // input rows; with a residual: h
   void *y;
   const void *scale;
   const void *shift;
-  const void *gamma;  // may be null
+  const void *gamma;   // may be null
+  const void *branch;  // residual only: h_out = h + gate * branch feeds the norm
+  const void *gate;    // residual only
+  void *h_out;         // residual only
   int64_t rows;       // B * L
   int L;              // < 2^31
   int n_video;
@@ -91,6 +94,8 @@ struct QkArgs {
 // dtype: 0 = fp32, 1 = bf16 (sol_dtype).  Each returns the launch error
 // (cudaSuccess if the kernel was enqueued) and fills `geo` if non-null.
 cudaError_t launch_rms_adaln(const RmsArgs &a, int dtype, cudaStream_t stream, Geometry *geo);
+cudaError_t launch_gate_residual_rms_adaln(const RmsArgs &a, int dtype, cudaStream_t stream,
+                                           Geometry *geo);
 cudaError_t launch_gate_residual(const GateArgs &a, int dtype, cudaStream_t stream,
                                  Geometry *geo);
 cudaError_t launch_qknorm_rope3d_f32(const QkArgs &a, cudaStream_t stream, Geometry *geo);
