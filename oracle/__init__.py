@@ -38,6 +38,8 @@ def _load():
         lib.oracle_gate_residual_rms_adaln.argtypes = [p, p, p, p, p, p, p, i64, i64, i64, i64,
                                                        d, i, p, p]
         lib.oracle_gate_residual_rms_adaln.restype = i
+        lib.oracle_residual_change.argtypes = [p, p, i64, i64, i64, i, p]
+        lib.oracle_residual_change.restype = i
         lib.oracle_qknorm_rope3d.argtypes = [p, i64, p, p, p, i64, i64, i64, i64,
                                              i64, i64, i64, i64, i64, i64, d, d,
                                              i, p, p]
@@ -127,6 +129,23 @@ def gate_residual_rms_adaln(h, branch, gate, scale, shift, L, n_video, eps, gamm
     if rc != 0:
         raise ValueError("oracle_gate_residual_rms_adaln rejected its arguments")
     return h_out.reshape(h.shape), y.reshape(h.shape)
+
+
+def residual_change(cur, prev, B, L):
+    """cur, prev: [B*L, D] (or [B, L, D]); returns [B + 1, 3] (num, den, rel),
+    the last row for the whole batch."""
+    cur, prev = _c(cur), _c(prev)
+    if cur.shape != prev.shape:
+        raise ValueError("cur and prev must have one shape")
+    D = cur.shape[-1]
+    if cur.size != B * L * D:
+        raise ValueError("cur must hold B*L rows")
+    out = np.empty((B + 1, 3), dtype=np.float64)
+    rc = _load().oracle_residual_change(_ptr(cur), _ptr(prev), B, L, D, _dtype_code(cur, prev),
+                                        _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_residual_change rejected its arguments")
+    return out
 
 
 def qknorm_rope3d(qkv, T, H, W, n_audio, n_heads, head_dim, sections, eps, theta,

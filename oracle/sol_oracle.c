@@ -190,6 +190,46 @@ int oracle_gate_residual_rms_adaln(const void *h, const void *branch, const void
 }
 
 /*
+ * First-Block-Cache change detector: how far the first block's residual
+ * moved since the previous denoising step (the cache gate of the Sol Video
+ * Inference Engine MiniMax-H3 page, cross-step caching paragraph: skip the
+ * remaining blocks when the first block's residual has barely changed).
+ * Relative L1 difference, per sample b over its L*D elements and over the
+ * whole batch:
+ *   num_b = sum |cur - prev|,  den_b = sum |prev|,
+ *   rel_b = num_b / den_b  (0 if num_b == den_b == 0, +inf if only den_b == 0)
+ * cur, prev: [B, L, D].  out: [B + 1][3] doubles (num, den, rel), row B for
+ * the whole batch (sums of the per-sample num and den).
+ */
+int oracle_residual_change(const void *cur, const void *prev, int64_t B, int64_t L,
+                           int64_t D, int dtype, double *out)
+{
+    if (B < 0 || L < 0 || D <= 0)
+        return -1;
+    double tn = 0.0, td = 0.0;
+    for (int64_t b = 0; b <= B; ++b) {
+        double num = 0.0, den = 0.0;
+        if (b < B) {
+            for (int64_t i = b * L * D; i < (b + 1) * L * D; ++i) {
+                double c = in_val(cur, i, dtype);
+                double p = in_val(prev, i, dtype);
+                num += fabs(c - p);
+                den += fabs(p);
+            }
+            tn += num;
+            td += den;
+        } else {
+            num = tn;
+            den = td;
+        }
+        out[3 * b + 0] = num;
+        out[3 * b + 1] = den;
+        out[3 * b + 2] = den > 0.0 ? num / den : (num > 0.0 ? INFINITY : 0.0);
+    }
+    return 0;
+}
+
+/*
  * Position of row r of a sample on the three rotary axes.
  * Video rows r < T*H*W are the latent grid in raster order, t-major:
  *   t = r / (H*W), h = (r / W) mod H, w = r mod W.

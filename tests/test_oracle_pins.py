@@ -455,3 +455,50 @@ def test_fused_residual_norm_closed_forms():
     h1, _ = oracle.gate_residual_rms_adaln(hh, br, g, z, z, L=L, n_video=nv, eps=1e-6)
     h2, _ = oracle.gate_residual_rms_adaln(hh, br, f32(2 * g), z, z, L=L, n_video=nv, eps=1e-6)
     np.testing.assert_allclose(h2 - h1, h1 - hh.astype(np.float64), rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# First-Block-Cache change detector
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("conv", [f32, bf16_bits], ids=["f32", "bf16"])
+def test_residual_change_hand_worked(conv):
+    # sample 0: cur = [1, 2, -3, 4], prev = [1, 1, -1, 2]: |c-p| = 0,1,2,2 -> 5;
+    #           |p| = 1+1+1+2 = 5 -> rel 1.0
+    # sample 1: cur = prev = [0.5, -0.5, 0.25, 0] -> num 0, den 1.25, rel 0
+    # batch: num 5, den 6.25, rel 0.8
+    cur = conv([[1, 2, -3, 4], [0.5, -0.5, 0.25, 0]])
+    prev = conv([[1, 1, -1, 2], [0.5, -0.5, 0.25, 0]])
+    out = oracle.residual_change(cur, prev, B=2, L=1)
+    np.testing.assert_array_equal(out, [[5, 5, 1.0], [0, 1.25, 0.0], [5, 6.25, 0.8]])
+
+
+def test_residual_change_closed_forms():
+    B, L, D = 3, 7, 16
+    prev = f32(RNG.standard_normal((B * L, D)))
+    # identical steps: zero change
+    out = oracle.residual_change(prev, prev, B, L)
+    np.testing.assert_array_equal(out[:, 0], 0.0)
+    np.testing.assert_array_equal(out[:, 2], 0.0)
+    # cur = (1 + a) * prev changes every element by |a * p|: rel = |a|; with
+    # 1 + a a power of two the scaled values stay exact
+    out = oracle.residual_change(f32(prev * 2.0), prev, B, L)
+    np.testing.assert_allclose(out[:, 2], 1.0, rtol=1e-15)
+    out = oracle.residual_change(f32(prev * 0.5), prev, B, L)
+    np.testing.assert_allclose(out[:, 2], 0.5, rtol=1e-15)
+    # cur = -prev: rel = 2
+    out = oracle.residual_change(f32(-prev), prev, B, L)
+    np.testing.assert_allclose(out[:, 2], 2.0, rtol=1e-15)
+    # batch row sums the per-sample rows
+    cur = f32(RNG.standard_normal((B * L, D)))
+    out = oracle.residual_change(cur, prev, B, L)
+    np.testing.assert_allclose(out[B, :2], out[:B, :2].sum(axis=0), rtol=1e-14)
+
+
+def test_residual_change_zero_denominator():
+    z = f32(np.zeros((2, 4)))
+    o = f32(np.ones((2, 4)))
+    out = oracle.residual_change(z, z, 2, 1)
+    assert np.all(out[:, 2] == 0.0)
+    out = oracle.residual_change(o, z, 2, 1)
+    assert np.all(np.isinf(out[:, 2]))
