@@ -53,6 +53,7 @@
 #ifndef SOL_H
 #define SOL_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -185,6 +186,46 @@ sol_status sol_qknorm_rope3d(const void *qkv, int64_t ld_qkv, void *q_out,
                              int64_t sec_h, int64_t sec_w, float eps,
                              float theta, sol_dtype dtype,
                              sol_stream_t stream);
+
+/*
+ * First-Block-Cache change detector (Sol Video Inference Engine MiniMax-H3
+ * page, cross-step caching paragraph: the first block's residual is compared
+ * with the previous denoising step's, and the remaining blocks are skipped
+ * when it has barely moved, against one residual-difference threshold).
+ * Relative L1 difference per sample b and over the whole batch:
+ *
+ *   num_b = sum_{r,c} |cur[b][r][c] - prev[b][r][c]|
+ *   den_b = sum_{r,c} |prev[b][r][c]|
+ *   rel_b = num_b / den_b   (0 if num_b = den_b = 0; +inf if only den_b = 0)
+ *
+ * and, if prev_out is non-null, prev_out = cur in the same pass (the cache
+ * refresh a step that does not skip performs).
+ *
+ *   cur, prev    [B, L, D] device, contiguous, 16-byte aligned.
+ *   prev_out     [B, L, D] device or NULL; may equal prev (in place), else
+ *                must not overlap cur or prev.
+ *   out          device, (B + 1) * 3 doubles, 8-byte aligned: row b is
+ *                (num_b, den_b, rel_b), row B the batch (sum of num, sum of
+ *                den, their ratio).  Sums are accumulated in fp32 per row
+ *                (at most 64 terms) and fp64 beyond, in a fixed order: the
+ *                result is deterministic.
+ *   workspace    device scratch of at least
+ *                sol_residual_change_workspace_bytes(B) bytes, 16-byte
+ *                aligned, owned by the caller; its contents on entry do not
+ *                matter and are overwritten.  Calls that share a workspace
+ *                must be ordered on one stream.
+ *   D            as for sol_rms_adaln (same limit); B <= 65535, B*L < 2^31.
+ * Two kernels are enqueued (partial sums, then a one-CTA finalisation).
+ */
+sol_status sol_residual_change(const void *cur, const void *prev,
+                               void *prev_out, int64_t B, int64_t L, int64_t D,
+                               double *out, void *workspace,
+                               size_t workspace_bytes, sol_dtype dtype,
+                               sol_stream_t stream);
+
+/* Workspace bytes sol_residual_change needs for B samples (a pure function
+ * of B; 16 KiB per sample). */
+size_t sol_residual_change_workspace_bytes(int64_t B);
 
 /* Static, human-readable name of a status code. */
 const char *sol_status_string(sol_status status);

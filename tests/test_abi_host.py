@@ -18,7 +18,8 @@ def built():
 def test_header_declares_the_entry_points():
     syms = _abi.header_symbols()
     for name in ("sol_rms_adaln", "sol_gate_residual", "sol_qknorm_rope3d",
-                 "sol_gate_residual_rms_adaln",
+                 "sol_gate_residual_rms_adaln", "sol_residual_change",
+                 "sol_residual_change_workspace_bytes",
                  "sol_status_string", "sol_last_error", "sol_version"):
         assert name in syms
 
@@ -135,6 +136,44 @@ def test_gate_residual_rms_adaln_rejects(kw, status):
 
 def test_gate_residual_rms_adaln_zero_rows_noop():
     assert fused(h=None, y=None, B=0) == _abi.SOL_OK
+
+
+def change(c=A, p=A + (1 << 30), po=None, B=2, L=4, D=64, out=A + (3 << 30),
+           ws=A + (4 << 30), wsb=None, dt=BF):
+    if wsb is None:
+        wsb = _abi.sol_residual_change_workspace_bytes(B)
+    return _abi.sol_residual_change(c, p, po, B, L, D, out, ws, wsb, dt, None)
+
+
+def test_residual_change_workspace_size():
+    assert _abi.sol_residual_change_workspace_bytes(0) == 0
+    assert _abi.sol_residual_change_workspace_bytes(1) == 16384
+    assert _abi.sol_residual_change_workspace_bytes(3) == 3 * 16384
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(c=None), _abi.SOL_ERR_INVALID_ARG),
+    (dict(out=None), _abi.SOL_ERR_INVALID_ARG),
+    (dict(ws=None), _abi.SOL_ERR_INVALID_ARG),
+    (dict(wsb=1000), _abi.SOL_ERR_INVALID_ARG),
+    (dict(D=12), _abi.SOL_ERR_MISALIGNED),
+    (dict(out=A + (3 << 30) + 4), _abi.SOL_ERR_MISALIGNED),
+    (dict(ws=A + (4 << 30) + 8), _abi.SOL_ERR_MISALIGNED),
+    (dict(B=70000, L=1), _abi.SOL_ERR_UNSUPPORTED),
+    (dict(D=16400), _abi.SOL_ERR_UNSUPPORTED),
+    (dict(po=A + 128), _abi.SOL_ERR_INVALID_ARG),           # prev_out overlaps cur
+    (dict(po=A + (1 << 30) + 16), _abi.SOL_ERR_INVALID_ARG),  # partial overlap with prev
+    (dict(out=A + 64), _abi.SOL_ERR_INVALID_ARG),           # out inside cur
+    (dict(ws=A + (1 << 30)), _abi.SOL_ERR_INVALID_ARG),     # workspace on prev
+    (dict(out=A + (4 << 30) + 64), _abi.SOL_ERR_INVALID_ARG),  # out inside workspace
+])
+def test_residual_change_rejects(kw, status):
+    assert change(**kw) == status
+
+
+def test_residual_change_zero_rows_noop():
+    assert change(c=None, out=None, B=0) == _abi.SOL_OK
+    assert change(c=None, L=0) == _abi.SOL_OK
 
 
 @pytest.mark.parametrize("kw,status", [

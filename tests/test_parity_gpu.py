@@ -291,6 +291,93 @@ def test_gate_residual_rms_adaln_in_place_and_guards():
 
 
 # ----------------------------------------------------------------------------
+# First-Block-Cache change detector
+# ----------------------------------------------------------------------------
+
+def _change_close(got, want, what):
+    """Relative error <= 1e-5 on num, den and rel (fp32 row partials of at most
+    64 terms, fp64 beyond); exact zeros and infinities must match."""
+    g = got.detach().cpu().numpy()
+    assert g.shape == want.shape, what
+    inf = np.isinf(want)
+    assert np.array_equal(np.isinf(g), inf), what
+    fin = ~inf
+    np.testing.assert_allclose(g[fin], want[fin], rtol=1e-5, atol=1e-30, err_msg=what)
+
+
+def _next_step(prev, rel_noise, seed):
+    """A 'next step' residual: prev plus relative noise (a few percent)."""
+    g = torch.Generator(device=prev.device).manual_seed(seed)
+    n = torch.randn(prev.shape, generator=g, device=prev.device, dtype=torch.float32)
+    return (prev.float() * (1.0 + rel_noise * n)).to(prev.dtype)
+
+
+@pytest.mark.parametrize("name", SMALL + ("clip5s", "clip15s", "cfg5s", "cfg5s_d3072"))
+def test_residual_change_workload(name):
+    w = WORKLOADS[name]
+    prev = activation(w.rows, w.D, w.torch_dtype, DEV, seed_for_change(w), w.outliers)
+    cur = _next_step(prev, 0.05, 7)
+    out = api.residual_change(cur.view(w.B, w.L, w.D), prev.view(w.B, w.L, w.D))
+    want = oracle.residual_change(_o(cur), _o(prev), w.B, w.L)
+    _change_close(out, want, f"residual_change[{name}]")
+    assert 0.01 < want[-1, 2] < 0.2
+
+
+def seed_for_change(w):
+    return 77_000 + w.index
+
+
+RC_SHAPES = [
+    (1, 1, 8, torch.bfloat16), (3, 37, 5128, torch.bfloat16), (2, 1000, 256, torch.float32),
+    (5, 999, 3072, torch.bfloat16), (1, 33, 16384, torch.bfloat16), (2, 17, 8192, torch.float32),
+    (70, 3, 512, torch.bfloat16), (1, 50001, 128, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("B,L,D,dt", RC_SHAPES)
+def test_residual_change_shapes(B, L, D, dt):
+    prev = activation(B * L, D, dt, DEV, 91, outliers=True)
+    cur = _next_step(prev, 0.1, 92)
+    out = api.residual_change(cur.view(B, L, D), prev.view(B, L, D))
+    _change_close(out, oracle.residual_change(_o(cur), _o(prev), B, L), f"rc B={B} L={L} D={D}")
+
+
+def test_residual_change_refresh_zero_and_determinism():
+    B, L, D, dt = 2, 3001, 5120, torch.bfloat16
+    prev = activation(B * L, D, dt, DEV, 93, outliers=True).view(B, L, D)
+    cur = _next_step(prev, 0.03, 94)
+    want = oracle.residual_change(_o(cur.view(-1, D)), _o(prev.view(-1, D)), B, L)
+    # cache refresh into a separate, guarded buffer
+    pad = 4096
+    n = B * L * D
+    buf = torch.full((n + 2 * pad,), 9.0, dtype=dt, device=DEV)
+    po = buf[pad:pad + n].view(B, L, D)
+    out = api.residual_change(cur, prev, prev_out=po)
+    torch.cuda.synchronize()
+    assert torch.equal(po, cur)
+    assert torch.all(buf[:pad] == 9.0) and torch.all(buf[-pad:] == 9.0)
+    _change_close(out, want, "rc refresh")
+    # refresh in place over prev; then the next comparison sees no change
+    p2 = prev.clone()
+    out = api.residual_change(cur, p2, prev_out=p2)
+    _change_close(out, want, "rc in-place refresh")
+    assert torch.equal(p2, cur)
+    out = api.residual_change(cur, p2)
+    assert torch.all(out[:, 0] == 0) and torch.all(out[:, 2] == 0)
+    # zero previous residual: rel is +inf where anything changed, 0 otherwise
+    z = torch.zeros_like(prev)
+    out = api.residual_change(cur, z)
+    assert torch.all(torch.isinf(out[:, 2]))
+    out = api.residual_change(z, z)
+    assert torch.all(out == 0)
+    # deterministic: same bits on every call
+    ws = torch.empty(_abi.sol_residual_change_workspace_bytes(B), dtype=torch.uint8, device=DEV)
+    a = api.residual_change(cur, prev, workspace=ws)
+    b = api.residual_change(cur, prev, workspace=ws)
+    assert torch.equal(a, b)
+
+
+# ----------------------------------------------------------------------------
 # QKNorm + 3D RoPE
 # ----------------------------------------------------------------------------
 

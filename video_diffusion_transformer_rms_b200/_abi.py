@@ -55,6 +55,10 @@ def lib() -> ctypes.CDLL:
         L.sol_gate_residual_rms_adaln.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, f,
                                                   i, p]
         L.sol_gate_residual_rms_adaln.restype = i
+        L.sol_residual_change.argtypes = [p, p, p, i64, i64, i64, p, p, ctypes.c_size_t, i, p]
+        L.sol_residual_change.restype = i
+        L.sol_residual_change_workspace_bytes.argtypes = [i64]
+        L.sol_residual_change_workspace_bytes.restype = ctypes.c_size_t
         L.sol_qknorm_rope3d.argtypes = [p, i64, p, p, i64, p, p, i64, i64, i64, i64, i64,
                                         i64, i64, i64, i64, i64, f, f, i, p]
         L.sol_qknorm_rope3d.restype = i
@@ -100,6 +104,16 @@ def sol_gate_residual_rms_adaln(h, branch, gate, h_out, y, scale, shift, gamma, 
                                 D, eps, dtype, stream) -> int:
     return lib().sol_gate_residual_rms_adaln(h, branch, gate, h_out, y, scale, shift, gamma, B,
                                              L, n_video, D, eps, dtype, stream)
+
+
+def sol_residual_change(cur, prev, prev_out, B, L, D, out, workspace, workspace_bytes, dtype,
+                        stream) -> int:
+    return lib().sol_residual_change(cur, prev, prev_out, B, L, D, out, workspace,
+                                     workspace_bytes, dtype, stream)
+
+
+def sol_residual_change_workspace_bytes(B) -> int:
+    return lib().sol_residual_change_workspace_bytes(B)
 
 
 def sol_qknorm_rope3d(qkv, ld_qkv, q_out, k_out, ld_out, gamma_q, gamma_k, B, T, H, W,

@@ -84,6 +84,30 @@ def gate_residual_rms_adaln(h: torch.Tensor, branch: torch.Tensor, gate: torch.T
     return ho, yo
 
 
+def residual_change(cur: torch.Tensor, prev: torch.Tensor,
+                    prev_out: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None,
+                    out: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """First-Block-Cache change of a [B, L, D] residual against the previous
+    step's: returns a [B + 1, 3] float64 CUDA tensor of (sum |cur - prev|,
+    sum |prev|, their ratio) per sample and, in the last row, for the batch.
+    With prev_out (may be prev itself) the cache is refreshed to cur in the
+    same pass.  The workspace is allocated by PyTorch unless given."""
+    if cur.dim() != 3 or not cur.is_contiguous() or prev.shape != cur.shape:
+        raise ValueError("cur and prev must be contiguous [B, L, D] tensors of one shape")
+    B, L, D = cur.shape
+    need = _abi.sol_residual_change_workspace_bytes(B)
+    ws = workspace if workspace is not None else torch.empty(
+        max(need, 16), dtype=torch.uint8, device=cur.device)
+    o = out if out is not None else torch.empty((B + 1, 3), dtype=torch.float64,
+                                                device=cur.device)
+    _abi.check(_abi.sol_residual_change(
+        _ptr(cur), _ptr(prev), _ptr(prev_out), B, L, D, _ptr(o), _ptr(ws),
+        ws.numel() * ws.element_size(), _dtype(cur, prev, prev_out), _stream(stream)))
+    return o
+
+
 def qknorm_rope3d(qkv: torch.Tensor, T: int, H: int, W: int, n_audio: int, n_heads: int,
                   head_dim: int, sections: Sequence[int] = (16, 24, 24),
                   gamma_q: Optional[torch.Tensor] = None,

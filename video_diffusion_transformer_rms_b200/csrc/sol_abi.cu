@@ -325,6 +325,70 @@ sol_status sol_gate_residual_rms_adaln(const void *h, const void *branch, const 
   return ok();
 }
 
+size_t sol_residual_change_workspace_bytes(int64_t B) {
+  return B <= 0 ? 0 : static_cast<size_t>(B) * kMaxChangeCtas * 2 * sizeof(double);
+}
+
+sol_status sol_residual_change(const void *cur, const void *prev, void *prev_out, int64_t B,
+                               int64_t L, int64_t D, double *out, void *workspace,
+                               size_t workspace_bytes, sol_dtype dtype, sol_stream_t stream) {
+  const char *fn = "sol_residual_change";
+  if (dtype != SOL_F32 && dtype != SOL_BF16)
+    return fail(SOL_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
+  if (B < 0 || L < 0 || D <= 0)
+    return fail(SOL_ERR_INVALID_ARG, "%s: need B >= 0, L >= 0, D > 0", fn);
+  if (B > 65535 || L > kMaxRows || B * L > kMaxRows)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: need B <= 65535 and B*L below 2^31 rows", fn);
+  const int64_t rows = B * L;
+  if (rows == 0) return ok();
+  if (!cur || !prev || !out || !workspace)
+    return fail(SOL_ERR_INVALID_ARG, "%s: cur, prev, out and workspace must be non-null", fn);
+  const int es = esize_of(dtype);
+  const int64_t row_bytes = D * es;
+  if (row_bytes % 16 != 0)
+    return fail(SOL_ERR_MISALIGNED, "%s: D*%d bytes must be a multiple of 16 (D=%lld)", fn, es,
+                (long long)D);
+  if (!aligned16(cur) || !aligned16(prev) || (prev_out && !aligned16(prev_out)) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(out) & 7u))
+    return fail(SOL_ERR_MISALIGNED,
+                "%s: tensors and workspace must be 16-byte aligned, out 8-byte aligned", fn);
+  if (row_bytes > kMaxRowBytesRms)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: D=%lld exceeds %lld elements", fn, (long long)D,
+                (long long)(kMaxRowBytesRms / es));
+  const size_t need = sol_residual_change_workspace_bytes(B);
+  if (workspace_bytes < need)
+    return fail(SOL_ERR_INVALID_ARG, "%s: workspace has %zu bytes, needs %zu", fn,
+                workspace_bytes, need);
+  const int64_t act = rows * row_bytes;
+  const Span cs = span_of(cur, 1, 0, act), ps = span_of(prev, 1, 0, act);
+  const Span os = span_of(out, 1, 0, (B + 1) * 3 * 8), ws = span_of(workspace, 1, 0, need);
+  if (prev_out) {
+    const Span pos = span_of(prev_out, 1, 0, act);
+    if (!same_or_disjoint(prev_out, prev, act) || spans_overlap(pos, cs))
+      return fail(SOL_ERR_INVALID_ARG, "%s: prev_out must equal prev or overlap neither input",
+                  fn);
+    if (spans_overlap(os, pos) || spans_overlap(ws, pos))
+      return fail(SOL_ERR_INVALID_ARG, "%s: out or workspace overlaps prev_out", fn);
+  }
+  if (spans_overlap(os, cs) || spans_overlap(os, ps) || spans_overlap(ws, cs) ||
+      spans_overlap(ws, ps) || spans_overlap(os, ws))
+    return fail(SOL_ERR_INVALID_ARG, "%s: out and workspace must not overlap the tensors or "
+                "each other", fn);
+
+  ChangeArgs a{};
+  a.cur = cur;
+  a.prev = prev;
+  a.prev_out = prev_out;
+  a.out = out;
+  a.partial = static_cast<double *>(workspace);
+  a.B = static_cast<int>(B);
+  a.L = static_cast<int>(L);
+  a.nvec = static_cast<int>(row_bytes / 16);
+  cudaError_t e = launch_residual_change(a, dtype == SOL_F32 ? 0 : 1, stream, nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_residual_change launch");
+  return ok();
+}
+
 sol_status sol_qknorm_rope3d(const void *qkv, int64_t ld_qkv, void *q_out, void *k_out,
                              int64_t ld_out, const void *gamma_q, const void *gamma_k, int64_t B,
                              int64_t T, int64_t H, int64_t W, int64_t n_audio, int64_t n_heads,

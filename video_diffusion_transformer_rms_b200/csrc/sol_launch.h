@@ -91,6 +91,21 @@ struct QkArgs {
   float theta;
 };
 
+// First-Block-Cache change detector.  `partial` is the caller's workspace:
+// [B][kMaxChangeCtas][2] doubles, every slot a CTA uses rewritten per call.
+constexpr int kMaxChangeCtas = 1024;
+struct ChangeArgs {
+  const void *cur;
+  const void *prev;
+  void *prev_out;   // may be null (no cache refresh)
+  double *out;      // [B + 1][3]: num, den, rel
+  double *partial;  // workspace
+  int B;
+  int L;
+  int nvec;
+  int ctas_per_sample;  // set by the launcher
+};
+
 // dtype: 0 = fp32, 1 = bf16 (sol_dtype).  Each returns the launch error
 // (cudaSuccess if the kernel was enqueued) and fills `geo` if non-null.
 cudaError_t launch_rms_adaln(const RmsArgs &a, int dtype, cudaStream_t stream, Geometry *geo);
@@ -98,6 +113,8 @@ cudaError_t launch_gate_residual_rms_adaln(const RmsArgs &a, int dtype, cudaStre
                                            Geometry *geo);
 cudaError_t launch_gate_residual(const GateArgs &a, int dtype, cudaStream_t stream,
                                  Geometry *geo);
+cudaError_t launch_residual_change(const ChangeArgs &a, int dtype, cudaStream_t stream,
+                                   Geometry *geo);
 cudaError_t launch_qknorm_rope3d_f32(const QkArgs &a, cudaStream_t stream, Geometry *geo);
 cudaError_t launch_qknorm_rope3d_bf16(const QkArgs &a, cudaStream_t stream, Geometry *geo);
 inline cudaError_t launch_qknorm_rope3d(const QkArgs &a, int dtype, cudaStream_t stream,
