@@ -227,6 +227,35 @@ sol_status sol_residual_change(const void *cur, const void *prev,
  * of B; 16 KiB per sample). */
 size_t sol_residual_change_workspace_bytes(int64_t B);
 
+/*
+ * sol_residual_change without a workspace argument.  This entry point has no
+ * counterpart on the pages; it exists for callers that cannot call
+ * cudaMalloc: a host that has already handed the device's memory to its own
+ * pool or framework allocator (so a raw cudaMalloc would fail or fragment
+ * it), a hot loop that must not pay cudaMalloc/cudaFree's implicit device
+ * synchronisation, or a plain-C plug-in with no allocator to borrow from.
+ *
+ * It computes exactly what sol_residual_change computes (same kernels, same
+ * fixed summation order) and allocates nothing.  The partial sums live in
+ * one device array inside libsol, 256 KiB, enough for B <= 16 samples; every
+ * GPU that loads the library holds that array until the process exits.
+ * Larger B returns SOL_ERR_UNSUPPORTED (use sol_residual_change).
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  Every call shares the one array and it keeps
+ * the last call's contents; each call rewrites every slot it later reads,
+ * so nothing needs clearing, but calls whose kernels overlap on the GPU
+ * (different streams, or different host threads on one device) race on it:
+ * order them on one stream.
+ *
+ *   cur, prev, prev_out, B, L, D, out, dtype: as for sol_residual_change.
+ */
+sol_status sol_residual_change_noalloc(const void *cur, const void *prev,
+                                       void *prev_out, int64_t B, int64_t L,
+                                       int64_t D, double *out, sol_dtype dtype,
+                                       sol_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char *sol_status_string(sol_status status);
 

@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.sol_residual_change.restype = i
         L.sol_residual_change_workspace_bytes.argtypes = [i64]
         L.sol_residual_change_workspace_bytes.restype = ctypes.c_size_t
+        L.sol_residual_change_noalloc.argtypes = [p, p, p, i64, i64, i64, p, i, p]
+        L.sol_residual_change_noalloc.restype = i
         L.sol_qknorm_rope3d.argtypes = [p, i64, p, p, i64, p, p, i64, i64, i64, i64, i64,
                                         i64, i64, i64, i64, i64, f, f, i, p]
         L.sol_qknorm_rope3d.restype = i
@@ -114,6 +116,12 @@ def sol_residual_change(cur, prev, prev_out, B, L, D, out, workspace, workspace_
 
 def sol_residual_change_workspace_bytes(B) -> int:
     return lib().sol_residual_change_workspace_bytes(B)
+
+
+def sol_residual_change_noalloc(cur, prev, prev_out, B, L, D, out, dtype, stream) -> int:
+    """sol_residual_change with its scratch inside libsol (B <= 16): for
+    callers that cannot allocate device memory."""
+    return lib().sol_residual_change_noalloc(cur, prev, prev_out, B, L, D, out, dtype, stream)
 
 
 def sol_qknorm_rope3d(qkv, ld_qkv, q_out, k_out, ld_out, gamma_q, gamma_k, B, T, H, W,

@@ -20,6 +20,9 @@
 // 2*D*esize bytes read, plus D*esize written with the cache refresh.
 #include <math.h>
 
+#include <map>
+#include <mutex>
+
 #include "sol_device.cuh"
 #include "sol_launch.h"
 
@@ -226,6 +229,49 @@ cudaError_t launch_residual_change(const ChangeArgs &a, int dtype, cudaStream_t 
                 : dispatch<float, false>(a, threads, vpt, stream, geo);
   return copy ? dispatch<__nv_bfloat16, true>(a, threads, vpt, stream, geo)
               : dispatch<__nv_bfloat16, false>(a, threads, vpt, stream, geo);
+}
+
+// ---------------------------------------------------------------------------
+// Variant for callers that cannot allocate device memory: the partial sums go
+// to this file-scope array instead of a caller workspace.  It is sized for
+// kNoAllocMaxSamples samples (256 KiB) and every device that loads the
+// library holds it until the process exits.  Host code must not pass the
+// symbol itself to a kernel (in host code it is only a stand-in): the device
+// address is looked up with cudaGetSymbolAddress, once per device, with that
+// device current, on the first call made on it.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) double g_change_scratch[kNoAllocMaxSamples * kMaxChangeCtas * 2];
+
+namespace {
+
+cudaError_t noalloc_scratch(double **ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static std::mutex mu;
+  static std::map<int, double *> addr;
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = addr.find(dev);
+  if (it == addr.end()) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_change_scratch);
+    if (e != cudaSuccess) return e;
+    it = addr.emplace(dev, static_cast<double *>(p)).first;
+  }
+  *ptr = it->second;
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_residual_change_noalloc(ChangeArgs a, int dtype, cudaStream_t stream,
+                                           Geometry *geo) {
+  if (a.B > kNoAllocMaxSamples) return cudaErrorInvalidValue;
+  double *scratch = nullptr;
+  cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  a.partial = scratch;
+  return launch_residual_change(a, dtype, stream, geo);
 }
 
 }  // namespace sol

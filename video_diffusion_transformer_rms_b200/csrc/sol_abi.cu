@@ -389,6 +389,64 @@ sol_status sol_residual_change(const void *cur, const void *prev, void *prev_out
   return ok();
 }
 
+sol_status sol_residual_change_noalloc(const void *cur, const void *prev, void *prev_out,
+                                       int64_t B, int64_t L, int64_t D, double *out,
+                                       sol_dtype dtype, sol_stream_t stream) {
+  const char *fn = "sol_residual_change_noalloc";
+  if (dtype != SOL_F32 && dtype != SOL_BF16)
+    return fail(SOL_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
+  if (B < 0 || L < 0 || D <= 0)
+    return fail(SOL_ERR_INVALID_ARG, "%s: need B >= 0, L >= 0, D > 0", fn);
+  if (B > kNoAllocMaxSamples)
+    return fail(SOL_ERR_UNSUPPORTED,
+                "%s: B=%lld exceeds the %d samples its built-in scratch holds; use "
+                "sol_residual_change with a workspace",
+                fn, (long long)B, kNoAllocMaxSamples);
+  if (L > kMaxRows || B * L > kMaxRows)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: B*L must be below 2^31 rows", fn);
+  const int64_t rows = B * L;
+  if (rows == 0) return ok();
+  if (!cur || !prev || !out)
+    return fail(SOL_ERR_INVALID_ARG, "%s: cur, prev and out must be non-null", fn);
+  const int es = esize_of(dtype);
+  const int64_t row_bytes = D * es;
+  if (row_bytes % 16 != 0)
+    return fail(SOL_ERR_MISALIGNED, "%s: D*%d bytes must be a multiple of 16 (D=%lld)", fn, es,
+                (long long)D);
+  if (!aligned16(cur) || !aligned16(prev) || (prev_out && !aligned16(prev_out)) ||
+      (reinterpret_cast<uintptr_t>(out) & 7u))
+    return fail(SOL_ERR_MISALIGNED, "%s: tensors must be 16-byte aligned, out 8-byte aligned",
+                fn);
+  if (row_bytes > kMaxRowBytesRms)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: D=%lld exceeds %lld elements", fn, (long long)D,
+                (long long)(kMaxRowBytesRms / es));
+  const int64_t act = rows * row_bytes;
+  const Span cs = span_of(cur, 1, 0, act), ps = span_of(prev, 1, 0, act);
+  const Span os = span_of(out, 1, 0, (B + 1) * 3 * 8);
+  if (prev_out) {
+    const Span pos = span_of(prev_out, 1, 0, act);
+    if (!same_or_disjoint(prev_out, prev, act) || spans_overlap(pos, cs))
+      return fail(SOL_ERR_INVALID_ARG, "%s: prev_out must equal prev or overlap neither input",
+                  fn);
+    if (spans_overlap(os, pos))
+      return fail(SOL_ERR_INVALID_ARG, "%s: out overlaps prev_out", fn);
+  }
+  if (spans_overlap(os, cs) || spans_overlap(os, ps))
+    return fail(SOL_ERR_INVALID_ARG, "%s: out must not overlap cur or prev", fn);
+
+  ChangeArgs a{};
+  a.cur = cur;
+  a.prev = prev;
+  a.prev_out = prev_out;
+  a.out = out;
+  a.B = static_cast<int>(B);
+  a.L = static_cast<int>(L);
+  a.nvec = static_cast<int>(row_bytes / 16);
+  cudaError_t e = launch_residual_change_noalloc(a, dtype == SOL_F32 ? 0 : 1, stream, nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_residual_change_noalloc launch");
+  return ok();
+}
+
 sol_status sol_qknorm_rope3d(const void *qkv, int64_t ld_qkv, void *q_out, void *k_out,
                              int64_t ld_out, const void *gamma_q, const void *gamma_k, int64_t B,
                              int64_t T, int64_t H, int64_t W, int64_t n_audio, int64_t n_heads,

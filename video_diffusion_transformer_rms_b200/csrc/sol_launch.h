@@ -115,6 +115,11 @@ cudaError_t launch_gate_residual(const GateArgs &a, int dtype, cudaStream_t stre
                                  Geometry *geo);
 cudaError_t launch_residual_change(const ChangeArgs &a, int dtype, cudaStream_t stream,
                                    Geometry *geo);
+// Same, with the partial sums in the library's own device array (no
+// workspace): at most kNoAllocMaxSamples samples.
+constexpr int kNoAllocMaxSamples = 16;
+cudaError_t launch_residual_change_noalloc(ChangeArgs a, int dtype, cudaStream_t stream,
+                                           Geometry *geo);
 cudaError_t launch_qknorm_rope3d_f32(const QkArgs &a, cudaStream_t stream, Geometry *geo);
 cudaError_t launch_qknorm_rope3d_bf16(const QkArgs &a, cudaStream_t stream, Geometry *geo);
 inline cudaError_t launch_qknorm_rope3d(const QkArgs &a, int dtype, cudaStream_t stream,
