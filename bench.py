@@ -308,6 +308,44 @@ def run_ours(args):
     value, total_units, slowest = dist.job_throughput(w.rows * K, elapsed_s)
     per_kernel_ms = {k: dist.max_over_ranks(v) for k, v in per_kernel_ms.items()}
 
+    # ---- next-row kernels, timed on their own after the step -------------
+    ws = torch.empty(_abi.sol_residual_change_workspace_bytes(w.B), dtype=torch.uint8,
+                     device=dev)
+    rc_out = torch.empty((w.B + 1, 3), dtype=torch.float64, device=dev)
+    extra = {
+        # h_out = h + gate*branch and y = RMS-AdaLN(h_out) in one pass: 4 D elements / row
+        "gate_residual_rms_adaln": (4, lambda: _abi.sol_gate_residual_rms_adaln(
+            p["h"], p["branch"], p["gate"], out.data_ptr(), y.data_ptr(), p["scale"],
+            p["shift"], None, w.B, w.L, w.n_video, D, w.eps, dt, s)),
+        # First-Block-Cache change of h against branch (stand-ins for two steps'
+        # residuals): 2 D elements read per row; with the cache refresh 3 D
+        "residual_change": (2, lambda: _abi.sol_residual_change(
+            p["h"], p["branch"], None, w.B, w.L, D, rc_out.data_ptr(), ws.data_ptr(),
+            ws.numel(), dt, s)),
+        "residual_change_refresh": (3, lambda: _abi.sol_residual_change(
+            p["h"], p["branch"], out.data_ptr(), w.B, w.L, D, rc_out.data_ptr(),
+            ws.data_ptr(), ws.numel(), dt, s)),
+    }
+    next_rows = {}
+    for name, (elems, fn) in extra.items():
+        for _ in range(5):
+            _abi.check(fn())
+        n_it = 200
+        ea = torch.cuda.Event(enable_timing=True)
+        eb = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        ea.record(stream)
+        for _ in range(n_it):
+            _abi.check(fn())
+        eb.record(stream)
+        torch.cuda.synchronize()
+        ms = dist.max_over_ranks(ea.elapsed_time(eb) / n_it)
+        nbytes = elems * D * w.esize * w.rows
+        next_rows[name] = {"ms": round(ms, 4), "tokens_per_s": round(w.rows / (ms / 1e3)),
+                           "bytes_per_token": elems * D * w.esize,
+                           "GB_per_s": round(nbytes / (ms / 1e3) / 1e9, 1)}
+    del ws
+
     # ---- end to end through the public API, host buffers ------------------
     e2e = run_e2e(args, w, t, stream, api)
     e2e_value, _, _ = dist.job_throughput(w.rows * e2e["steps"], e2e["seconds"])
@@ -344,7 +382,8 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; no dataset or weights involved)",
             "config": workload_config(w, world),
-            "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu,
+            "roofline": roofline, "kernels": kernels, "next_rows": next_rows,
+            "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                     "steps": e2e["steps"],

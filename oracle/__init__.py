@@ -40,6 +40,12 @@ def _load():
         lib.oracle_gate_residual_rms_adaln.restype = i
         lib.oracle_residual_change.argtypes = [p, p, i64, i64, i64, i, p]
         lib.oracle_residual_change.restype = i
+        lib.oracle_qknorm_rope3d_ex.argtypes = [p, i64, p, p, p, i64, i64, i64, i64,
+                                                i64, i64, i64, i64, i64, i64, d, d,
+                                                i, i, p, p]
+        lib.oracle_qknorm_rope3d_ex.restype = i
+        lib.oracle_quantize_heads.argtypes = [p, i64, i64, i64, p, p]
+        lib.oracle_quantize_heads.restype = i
         lib.oracle_qknorm_rope3d.argtypes = [p, i64, p, p, p, i64, i64, i64, i64,
                                              i64, i64, i64, i64, i64, i64, d, d,
                                              i, p, p]
@@ -168,6 +174,41 @@ def qknorm_rope3d(qkv, T, H, W, n_audio, n_heads, head_dim, sections, eps, theta
     if rc != 0:
         raise ValueError("oracle_qknorm_rope3d rejected its arguments")
     return q, k
+
+
+def qknorm_rope3d_ex(qkv, T, H, W, n_audio, n_heads, head_dim, sections, eps, theta,
+                     half_split, gamma_q=None, gamma_k=None, row_ids=None):
+    """qknorm_rope3d with a rotary pair layout flag (half_split: pair i is
+    elements (i, i + head_dim/2))."""
+    qkv, gamma_q, gamma_k = _c(qkv), _c(gamma_q), _c(gamma_k)
+    D = n_heads * head_dim
+    q2 = qkv.reshape(-1, qkv.shape[-1])
+    rid, n = _rows(row_ids, q2.shape[0])
+    if n != q2.shape[0]:
+        raise ValueError("row_ids length must match the rows of qkv")
+    q = np.empty((n, D), dtype=np.float64)
+    k = np.empty((n, D), dtype=np.float64)
+    st, sh, sw = sections
+    rc = _load().oracle_qknorm_rope3d_ex(_ptr(q2), q2.shape[1], _ptr(gamma_q), _ptr(gamma_k),
+                                         _ptr(rid), n, T, H, W, n_audio, n_heads, head_dim, st,
+                                         sh, sw, eps, theta, int(bool(half_split)),
+                                         _dtype_code(qkv, gamma_q, gamma_k), _ptr(q), _ptr(k))
+    if rc != 0:
+        raise ValueError("oracle_qknorm_rope3d_ex rejected its arguments")
+    return q, k
+
+
+def quantize_heads(x, n_heads, head_dim):
+    """Symmetric per-head INT8 codes of x [n_rows, n_heads*head_dim] (fp64):
+    returns (codes int32 [n_rows, D], scales fp64 [n_rows, n_heads])."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    n = x.shape[0]
+    code = np.empty(x.shape, dtype=np.int32)
+    scale = np.empty((n, n_heads), dtype=np.float64)
+    rc = _load().oracle_quantize_heads(_ptr(x), n, n_heads, head_dim, _ptr(code), _ptr(scale))
+    if rc != 0:
+        raise ValueError("oracle_quantize_heads rejected its arguments")
+    return code, scale
 
 
 def ulp(v, dtype):

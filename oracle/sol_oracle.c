@@ -321,3 +321,98 @@ int oracle_qknorm_rope3d(const void *qkv, int64_t ld_qkv, const void *gamma_q,
     }
     return 0;
 }
+
+/*
+ * QKNorm + 3D RoPE with a choice of rotary pair layout.  half_split = 0 is
+ * oracle_qknorm_rope3d (pair i = elements (2i, 2i+1)); half_split = 1 pairs
+ * element i with element i + head_dim/2 (the "rotate half" layout of GPT-NeoX
+ * style implementations):
+ *   out[i]              = n[i] cos(phi_i) - n[i + hd/2] sin(phi_i)
+ *   out[i + hd/2]       = n[i] sin(phi_i) + n[i + hd/2] cos(phi_i)
+ * with the same phi_i, sections and positions.  Arguments as for
+ * oracle_qknorm_rope3d.
+ */
+int oracle_qknorm_rope3d_ex(const void *qkv, int64_t ld_qkv, const void *gamma_q,
+                            const void *gamma_k, const int64_t *row_ids, int64_t n_rows,
+                            int64_t T, int64_t H, int64_t W, int64_t n_audio,
+                            int64_t n_heads, int64_t head_dim, int64_t sec_t,
+                            int64_t sec_h, int64_t sec_w, double eps, double theta,
+                            int half_split, int dtype, double *q_out, double *k_out)
+{
+    if (!half_split)
+        return oracle_qknorm_rope3d(qkv, ld_qkv, gamma_q, gamma_k, row_ids, n_rows, T, H,
+                                    W, n_audio, n_heads, head_dim, sec_t, sec_h, sec_w, eps,
+                                    theta, dtype, q_out, k_out);
+    int64_t D = n_heads * head_dim;
+    int64_t L = T * H * W + n_audio;
+    int64_t half = head_dim / 2;
+    if (n_rows < 0 || T < 0 || H < 0 || W < 0 || n_audio < 0 || L <= 0 ||
+        n_heads <= 0 || head_dim <= 0 || head_dim % 2 != 0 || sec_t < 0 ||
+        sec_h < 0 || sec_w < 0 || sec_t + sec_h + sec_w != half || ld_qkv < 2 * D)
+        return -1;
+    for (int64_t k = 0; k < n_rows; ++k) {
+        int64_t r = row_id(row_ids, k) % L;
+        int64_t pos[3];
+        row_position(r, T, H, W, pos);
+        for (int part = 0; part < 2; ++part) {
+            const void *gam = part == 0 ? gamma_q : gamma_k;
+            double *out = part == 0 ? q_out : k_out;
+            for (int64_t hd = 0; hd < n_heads; ++hd) {
+                int64_t src = k * ld_qkv + part * D + hd * head_dim;
+                int64_t dst = k * D + hd * head_dim;
+                double ss = 0.0;
+                for (int64_t j = 0; j < head_dim; ++j) {
+                    double v = in_val(qkv, src + j, dtype);
+                    ss += v * v;
+                }
+                double denom = sqrt(ss / (double)head_dim + eps);
+                for (int64_t i = 0; i < half; ++i) {
+                    double a = in_val(qkv, src + i, dtype) / denom;
+                    double b = in_val(qkv, src + i + half, dtype) / denom;
+                    if (gam) {
+                        a = a * in_val(gam, i, dtype);
+                        b = b * in_val(gam, i + half, dtype);
+                    }
+                    int axis = i < sec_t ? 0 : (i < sec_t + sec_h ? 1 : 2);
+                    double phi = (double)pos[axis] *
+                                 pow(theta, -2.0 * (double)i / (double)head_dim);
+                    double c = cos(phi), s = sin(phi);
+                    out[dst + i] = a * c - b * s;
+                    out[dst + i + half] = a * s + b * c;
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Symmetric INT8 quantisation of each head vector (for the INT8 Q/K
+ * exchange between GPUs in the KOCPC article's 4x/8x B300 runs):
+ *   scale = max_j |x[j]| / 127,  code[j] = round_half_even(x[j] / scale)
+ * (scale 0 and all codes 0 for an all-zero head).  x: [n_rows, n_heads *
+ * head_dim] doubles; code: same shape (int32 holding values in -127..127);
+ * scale: [n_rows, n_heads].
+ */
+int oracle_quantize_heads(const double *x, int64_t n_rows, int64_t n_heads,
+                          int64_t head_dim, int32_t *code, double *scale)
+{
+    if (n_rows < 0 || n_heads <= 0 || head_dim <= 0)
+        return -1;
+    for (int64_t k = 0; k < n_rows; ++k) {
+        for (int64_t h = 0; h < n_heads; ++h) {
+            const double *v = x + (k * n_heads + h) * head_dim;
+            int32_t *c = code + (k * n_heads + h) * head_dim;
+            double amax = 0.0;
+            for (int64_t j = 0; j < head_dim; ++j)
+                if (fabs(v[j]) > amax)
+                    amax = fabs(v[j]);
+            double s = amax / 127.0;
+            scale[k * n_heads + h] = s;
+            for (int64_t j = 0; j < head_dim; ++j)
+                c[j] = s > 0.0 ? (int32_t)nearbyint(v[j] / s) : 0;
+        }
+    }
+    return 0;
+}
+

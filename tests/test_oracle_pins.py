@@ -502,3 +502,78 @@ def test_residual_change_zero_denominator():
     assert np.all(out[:, 2] == 0.0)
     out = oracle.residual_change(o, z, 2, 1)
     assert np.all(np.isinf(out[:, 2]))
+
+
+# ----------------------------------------------------------------------------
+# QKNorm + RoPE epilogue variants: half-split pairs, INT8 heads
+# ----------------------------------------------------------------------------
+
+def test_half_split_angles_match_hand_table():
+    # first half of every head = 1, second half = 0: with eps = 0 the head
+    # normalises to sqrt2 in the first half; pair i = (x[i], x[i+64]) becomes
+    # sqrt2 (cos phi_i, sin phi_i) at elements (i, i + 64).
+    pos, pairs = _positions()
+    rows = _grid_rows(**TINY)
+    hd = TINY["head_dim"]
+    qh = np.concatenate([np.ones(hd // 2), np.zeros(hd // 2)])
+    qkv = _qkv_same_every_row(qh, qh, rows, TINY["n_heads"])
+    q, k = oracle.qknorm_rope3d_ex(qkv, eps=0.0, half_split=True, **TINY)
+    s2 = math.sqrt(2.0)
+    for r, p in pos.items():
+        for i, (axis, freq) in pairs.items():
+            phi = p[axis] * freq
+            for out in (q, k):
+                for head in range(TINY["n_heads"]):
+                    a, b = out[r, head * hd + i], out[r, head * hd + i + hd // 2]
+                    assert abs(math.hypot(a, b) - s2) < 1e-13
+                    assert abs(_wrap(math.atan2(b, a) - phi)) < 1e-12, (r, i)
+
+
+def test_half_split_is_complex_multiplication_and_flag_off_is_interleaved():
+    rows = _grid_rows(**TINY)
+    qh, kh = RNG.standard_normal(128), RNG.standard_normal(128)
+    qkv = _qkv_same_every_row(qh, kh, rows, 2)
+    q, _ = oracle.qknorm_rope3d_ex(qkv, eps=1e-6, half_split=True, **TINY)
+    z0 = q[0, :64] + 1j * q[0, 64:128]
+    for r in range(rows):
+        rot = z0 * np.exp(1j * _closed_form_angles(r))
+        np.testing.assert_allclose(q[r, :64], rot.real, atol=1e-12)
+        np.testing.assert_allclose(q[r, 64:128], rot.imag, atol=1e-12)
+    qi, ki = oracle.qknorm_rope3d_ex(qkv, eps=1e-6, half_split=False, **TINY)
+    q0, k0 = oracle.qknorm_rope3d(qkv, eps=1e-6, **TINY)
+    np.testing.assert_array_equal(qi, q0)
+    np.testing.assert_array_equal(ki, k0)
+
+
+def test_quantize_heads_hand_worked():
+    # head 0: max |x| = 127 -> scale 1; -63.5 rounds half to even (-64),
+    # 0.5 -> 0, 1.5 -> 2.  head 1: all zero -> scale 0, codes 0.
+    x = np.array([[127.0, -63.5, 0.5, 1.5, 0.0, 0.0, 0.0, 0.0]])
+    code, scale = oracle.quantize_heads(x, n_heads=2, head_dim=4)
+    np.testing.assert_array_equal(code, [[127, -64, 0, 2, 0, 0, 0, 0]])
+    np.testing.assert_array_equal(scale, [[1.0, 0.0]])
+    # a head scaled by 2: same codes, scale 2/127 * 127 / 2... -> scale doubles
+    code2, scale2 = oracle.quantize_heads(2 * x, n_heads=2, head_dim=4)
+    np.testing.assert_array_equal(code2, code)
+    np.testing.assert_array_equal(scale2, 2 * scale)
+
+
+def test_quantize_heads_bounds_and_error():
+    x = RNG.standard_normal((9, 3 * 16)) * np.linspace(0.1, 40, 9)[:, None]
+    code, scale = oracle.quantize_heads(x, n_heads=3, head_dim=16)
+    assert code.min() >= -127 and code.max() <= 127
+    deq = code.reshape(9, 3, 16) * scale[:, :, None]
+    err = np.abs(deq - x.reshape(9, 3, 16))
+    assert np.all(err <= scale[:, :, None] / 2 + 1e-12)
+    assert np.all(np.abs(code.reshape(9, 3, 16)).max(axis=2) == 127)
+
+
+def test_half_split_identity_at_origin_gives_gamma():
+    hd = 128
+    gq = f32(1.0 + 0.1 * RNG.standard_normal(hd))
+    gk = f32(1.0 + 0.1 * RNG.standard_normal(hd))
+    qkv = _qkv_same_every_row(np.full(hd, 2.0), np.full(hd, -0.5), 1, 2)
+    q, k = oracle.qknorm_rope3d_ex(qkv, 1, 1, 1, 0, 2, hd, (16, 24, 24), 0.0, 1e4, True,
+                                   gamma_q=gq, gamma_k=gk)
+    np.testing.assert_allclose(q[0], np.tile(gq.astype(np.float64), 2), rtol=1e-15)
+    np.testing.assert_allclose(k[0], np.tile(-gk.astype(np.float64), 2), rtol=1e-15)
