@@ -188,6 +188,53 @@ sol_status sol_qknorm_rope3d(const void *qkv, int64_t ld_qkv, void *q_out,
                              sol_stream_t stream);
 
 /*
+ * Output layout and epilogue of sol_qknorm_rope3d_ex.
+ *
+ * Element (sample b, token row r, head h, channel c) of q (k) goes to
+ * q_out (k_out) + b*stride_b + r*stride_row + h*stride_head + c, strides in
+ * elements of the output type, channels contiguous.  [B, L, H, hd] is
+ * (L*H*hd, H*hd, hd); attention's [B, H, L, hd] is (H*L*hd, hd, L*hd).
+ * The strides must address distinct elements (not checked).
+ */
+typedef struct sol_qk_layout {
+    int64_t stride_b;
+    int64_t stride_row;
+    int64_t stride_head;
+    int32_t half_split; /* 0: pair i = (2i, 2i+1); 1: pair i = (i, i + hd/2) */
+    int32_t int8_out;   /* 1: q_out/k_out receive int8 codes, and q_scale /
+                           k_scale [B, L, H] fp32 receive max|x| / 127 per head */
+    float *q_scale;     /* int8_out only: device, 4-byte aligned */
+    float *k_scale;
+} sol_qk_layout;
+
+/*
+ * QKNorm + 3D RoPE (as sol_qknorm_rope3d) with the epilogue variants its
+ * consumers need: any head-strided output layout (attention's [B, H, L, hd]
+ * directly), the half-split rotary pair layout, and INT8 output with
+ * symmetric per-(row, head) scales, code = round_half_even(x * 127 /
+ * max|x|) in fp32 (the quantised Q/K the KOCPC Sol-H3 article's 4x/8x B300
+ * runs exchange between GPUs).  The rotation angles, sections, positions,
+ * gamma and eps are those of sol_qknorm_rope3d.
+ *
+ *   dtype       SOL_BF16 input (SOL_ERR_UNSUPPORTED otherwise); output bf16,
+ *               or int8 with int8_out.
+ *   head_dim    64, 128 or 256.
+ *   q_out, k_out, layout   see sol_qk_layout; outputs must not overlap qkv,
+ *               each other or the scales (no in-place form).  Each output
+ *               vector start (16 bytes, 8 for int8) must be aligned to its
+ *               size: base and strides * element size multiples of it.
+ *   other arguments as for sol_qknorm_rope3d.
+ */
+sol_status sol_qknorm_rope3d_ex(const void *qkv, int64_t ld_qkv, void *q_out,
+                                void *k_out, const sol_qk_layout *layout,
+                                const void *gamma_q, const void *gamma_k,
+                                int64_t B, int64_t T, int64_t H, int64_t W,
+                                int64_t n_audio, int64_t n_heads,
+                                int64_t head_dim, int64_t sec_t, int64_t sec_h,
+                                int64_t sec_w, float eps, float theta,
+                                sol_dtype dtype, sol_stream_t stream);
+
+/*
  * First-Block-Cache change detector (Sol Video Inference Engine MiniMax-H3
  * page, cross-step caching paragraph: the first block's residual is compared
  * with the previous denoising step's, and the remaining blocks are skipped

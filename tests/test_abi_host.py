@@ -19,7 +19,8 @@ def test_header_declares_the_entry_points():
     syms = _abi.header_symbols()
     for name in ("sol_rms_adaln", "sol_gate_residual", "sol_qknorm_rope3d",
                  "sol_gate_residual_rms_adaln", "sol_residual_change",
-                 "sol_residual_change_workspace_bytes",
+                 "sol_residual_change_workspace_bytes", "sol_qknorm_rope3d_ex",
+                 "sol_residual_change_noalloc",
                  "sol_status_string", "sol_last_error", "sol_version"):
         assert name in syms
 
@@ -223,3 +224,34 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     with pytest.raises(ImportError):
         _abi.lib()
     assert isinstance(ctypes.CDLL, type)
+
+
+def qkex(qkv=A, ldq=3 * 1024, qo=A + (1 << 30), ko=A + (2 << 30), sb=None, sr=1024, sh=128,
+         half=0, int8=0, qs=None, ks=None, B=1, T=2, H=4, W=6, na=8, nh=8, hd=128,
+         secs=(16, 24, 24), dt=BF):
+    L = T * H * W + na
+    lay = _abi.QkLayout(L * nh * hd if sb is None else sb, sr, sh, half, int8, qs, ks)
+    return _abi.sol_qknorm_rope3d_ex(qkv, ldq, qo, ko, lay, None, None, B, T, H, W, na, nh, hd,
+                                     *secs, 1e-6, 1e4, dt, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dt=F32), _abi.SOL_ERR_UNSUPPORTED),
+    (dict(hd=32, secs=(4, 6, 6), nh=32), _abi.SOL_ERR_UNSUPPORTED),
+    (dict(sr=-1), _abi.SOL_ERR_INVALID_ARG),
+    (dict(sh=4), _abi.SOL_ERR_MISALIGNED),                      # 8-byte head stride
+    (dict(qo=A + (1 << 30) + 8), _abi.SOL_ERR_MISALIGNED),
+    (dict(int8=1), _abi.SOL_ERR_INVALID_ARG),                   # scales missing
+    (dict(int8=1, qs=A + (3 << 30) + 2, ks=A + (4 << 30)), _abi.SOL_ERR_MISALIGNED),
+    (dict(qo=A + 4096), _abi.SOL_ERR_INVALID_ARG),              # q_out inside qkv
+    (dict(ko=A + (1 << 30) + 1024), _abi.SOL_ERR_INVALID_ARG),  # k_out overlaps q_out
+    (dict(int8=1, qs=A + (1 << 30), ks=A + (4 << 30)), _abi.SOL_ERR_INVALID_ARG),  # scale on q
+])
+def test_qknorm_rope3d_ex_rejects(kw, status):
+    assert qkex(**kw) == status
+
+
+def test_qknorm_rope3d_ex_null_layout():
+    assert _abi.sol_qknorm_rope3d_ex(A, 3 * 1024, A + (1 << 30), A + (2 << 30), None, None,
+                                     None, 1, 2, 4, 6, 8, 8, 128, 16, 24, 24, 1e-6, 1e4, BF,
+                                     None) == _abi.SOL_ERR_INVALID_ARG

@@ -495,3 +495,100 @@ def test_qknorm_rope3d_large_positions_are_accurate():
                                   (16, 24, 24), 1e-6, 1e4, row_ids=ids)
     assert_close(take_rows_gpu(q.reshape(L, -1), ids), wq, "q far positions")
     assert_close(take_rows_gpu(k.reshape(L, -1), ids), wk, "k far positions")
+
+
+
+# ----------------------------------------------------------------------------
+# QKNorm + RoPE epilogue variants: layouts, half-split pairs, INT8 output
+# ----------------------------------------------------------------------------
+
+def _bshd(t, layout):
+    """[B, L, H, hd] view of a q/k output in either layout."""
+    return t if layout == "bshd" else t.permute(0, 2, 1, 3)
+
+
+def _check_int8(codes, scales, want, n_heads, hd, what):
+    """scale = max|x| / 127 per (row, head) within fp32 error, and every code
+    dequantises to within half a step of the oracle value (plus 1% of a step
+    for the fp32 arithmetic before the rounding)."""
+    c = codes.detach().cpu().numpy().astype(np.float64).reshape(-1, n_heads, hd)
+    sc = scales.detach().cpu().numpy().astype(np.float64).reshape(-1, n_heads)
+    x = want.reshape(-1, n_heads, hd)
+    np.testing.assert_allclose(sc, np.abs(x).max(axis=2) / 127.0, rtol=1e-5, atol=1e-12,
+                               err_msg=f"{what} scales")
+    err = np.abs(c * sc[:, :, None] - x)
+    bound = sc[:, :, None] * 0.51 + 1e-9
+    bad = err > bound
+    assert not bad.any(), f"{what}: {int(bad.sum())} codes off by more than half a step"
+    assert np.abs(c).max() <= 127
+
+
+@pytest.mark.parametrize("name", ("medium", "clip5s"))
+@pytest.mark.parametrize("half", [False, True])
+@pytest.mark.parametrize("layout", ["bshd", "bhsd"])
+@pytest.mark.parametrize("int8", [False, True])
+def test_qknorm_rope3d_ex_workload(name, half, layout, int8):
+    w = WORKLOADS[name]
+    t = make_inputs(w, DEV, which=("qknorm_rope3d",))
+    qkv = t["qkv"].view(w.B, w.L, 3 * w.D)
+    res = api.qknorm_rope3d_ex(qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim,
+                               w.sections, t["gamma_q"], t["gamma_k"], w.eps, w.theta,
+                               layout=layout, half_split=half, int8=int8)
+    torch.cuda.synchronize()
+    q, k = (_bshd(r, layout).reshape(w.rows, w.D) for r in res[:2])
+    ids = None if name == "medium" else _ids(w, 512)
+    qkv2 = qkv.view(-1, 3 * w.D)
+    src = _o(qkv2) if ids is None else take_rows(qkv2[:, :2 * w.D], ids)
+    wq, wk = oracle.qknorm_rope3d_ex(src, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim,
+                                     w.sections, w.eps, w.theta, half, _o(t["gamma_q"]),
+                                     _o(t["gamma_k"]), row_ids=ids)
+    if ids is not None:
+        q, k = take_rows_gpu(q, ids), take_rows_gpu(k, ids)
+    tag = f"ex[{name} half={half} {layout} int8={int8}]"
+    if int8:
+        qs, ks = (r.reshape(w.rows, w.n_heads) for r in res[2:])
+        if ids is not None:
+            qs, ks = take_rows_gpu(qs, ids), take_rows_gpu(ks, ids)
+        _check_int8(q, qs, wq, w.n_heads, w.head_dim, tag + " q")
+        _check_int8(k, ks, wk, w.n_heads, w.head_dim, tag + " k")
+    else:
+        assert_close(q, wq, tag + " q")
+        assert_close(k, wk, tag + " k")
+
+
+def test_qknorm_rope3d_ex_interleaved_matches_default_entry_point():
+    # same arithmetic as sol_qknorm_rope3d, only the addressing differs:
+    # bit-identical results in both layouts
+    w = WORKLOADS["medium"]
+    t = make_inputs(w, DEV, which=("qknorm_rope3d",))
+    qkv = t["qkv"].view(w.B, w.L, 3 * w.D)
+    args = (w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections, t["gamma_q"],
+            t["gamma_k"], w.eps, w.theta)
+    q0, k0 = api.qknorm_rope3d(qkv, *args)
+    for layout in ("bshd", "bhsd"):
+        q1, k1 = api.qknorm_rope3d_ex(qkv, *args, layout=layout)
+        assert torch.equal(_bshd(q1, layout).reshape(q0.shape), q0)
+        assert torch.equal(_bshd(k1, layout).reshape(k0.shape), k0)
+
+
+@pytest.mark.parametrize("hd,secs", [(64, (8, 12, 12)), (256, (32, 48, 48))])
+@pytest.mark.parametrize("half", [False, True])
+def test_qknorm_rope3d_ex_head_dims(hd, secs, half):
+    B, T, H, W, na, nh = 2, 3, 5, 7, 11, 6
+    L = T * H * W + na
+    D = nh * hd
+    qkv = activation(B * L, 3 * D, torch.bfloat16, DEV, 61, outliers=True).view(B, L, 3 * D)
+    gq = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 62)
+    gk = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 63)
+    for int8 in (False, True):
+        res = api.qknorm_rope3d_ex(qkv, T, H, W, na, nh, hd, secs, gq, gk, layout="bhsd",
+                                   half_split=half, int8=int8)
+        wq, wk = oracle.qknorm_rope3d_ex(_o(qkv.view(B * L, 3 * D)), T, H, W, na, nh, hd, secs,
+                                         1e-6, 1e4, half, _o(gq), _o(gk))
+        q, k = (_bshd(r, "bhsd").reshape(B * L, D) for r in res[:2])
+        if int8:
+            _check_int8(q, res[2], wq, nh, hd, f"hd={hd} q")
+            _check_int8(k, res[3], wk, nh, hd, f"hd={hd} k")
+        else:
+            assert_close(q, wq, f"hd={hd} half={half} q")
+            assert_close(k, wk, f"hd={hd} half={half} k")

@@ -24,6 +24,14 @@ SOL_ERR_CUDA = 4
 SOL_F32 = 0
 SOL_BF16 = 1
 
+class QkLayout(ctypes.Structure):
+    """sol_qk_layout of include/sol.h."""
+    _fields_ = [("stride_b", ctypes.c_int64), ("stride_row", ctypes.c_int64),
+                ("stride_head", ctypes.c_int64), ("half_split", ctypes.c_int32),
+                ("int8_out", ctypes.c_int32), ("q_scale", ctypes.c_void_p),
+                ("k_scale", ctypes.c_void_p)]
+
+
 _lock = threading.Lock()
 _lib = None
 
@@ -61,6 +69,10 @@ def lib() -> ctypes.CDLL:
         L.sol_residual_change_workspace_bytes.restype = ctypes.c_size_t
         L.sol_residual_change_noalloc.argtypes = [p, p, p, i64, i64, i64, p, i, p]
         L.sol_residual_change_noalloc.restype = i
+        L.sol_qknorm_rope3d_ex.argtypes = [p, i64, p, p, ctypes.POINTER(QkLayout), p, p, i64,
+                                           i64, i64, i64, i64, i64, i64, i64, i64, i64, f, f,
+                                           i, p]
+        L.sol_qknorm_rope3d_ex.restype = i
         L.sol_qknorm_rope3d.argtypes = [p, i64, p, p, i64, p, p, i64, i64, i64, i64, i64,
                                         i64, i64, i64, i64, i64, f, f, i, p]
         L.sol_qknorm_rope3d.restype = i
@@ -130,6 +142,16 @@ def sol_qknorm_rope3d(qkv, ld_qkv, q_out, k_out, ld_out, gamma_q, gamma_k, B, T,
     return lib().sol_qknorm_rope3d(qkv, ld_qkv, q_out, k_out, ld_out, gamma_q, gamma_k, B, T,
                                    H, W, n_audio, n_heads, head_dim, sec_t, sec_h, sec_w,
                                    eps, theta, dtype, stream)
+
+
+def sol_qknorm_rope3d_ex(qkv, ld_qkv, q_out, k_out, layout, gamma_q, gamma_k, B, T, H, W,
+                         n_audio, n_heads, head_dim, sec_t, sec_h, sec_w, eps, theta, dtype,
+                         stream) -> int:
+    """layout: a QkLayout (or None, which the library rejects)."""
+    ref = ctypes.byref(layout) if layout is not None else None
+    return lib().sol_qknorm_rope3d_ex(qkv, ld_qkv, q_out, k_out, ref, gamma_q, gamma_k, B, T,
+                                      H, W, n_audio, n_heads, head_dim, sec_t, sec_h, sec_w,
+                                      eps, theta, dtype, stream)
 
 
 def sol_status_string(status: int) -> str:

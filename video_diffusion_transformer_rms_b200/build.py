@@ -21,8 +21,9 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsol.so")
 
 SOURCES = ["sol_abi.cu", "rms_adaln.cu", "gate_residual.cu", "qknorm_rope3d_bf16.cu",
-           "qknorm_rope3d_f32.cu", "residual_change.cu"]
-HEADERS = ["sol_device.cuh", "sol_launch.h", "qknorm_rope3d.cuh"]
+           "qknorm_rope3d_f32.cu", "qknorm_rope3d_ex_bf16.cu", "qknorm_rope3d_ex_int8.cu",
+           "residual_change.cu"]
+HEADERS = ["sol_device.cuh", "sol_launch.h", "qknorm_rope3d.cuh", "qknorm_rope3d_ex.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",

@@ -1,0 +1,321 @@
+// QKNorm + 3D RoPE epilogue variants (bf16 input), for what consumes q and k
+// next:
+//   - any output layout with unit element stride: per (sample, token row,
+//     head) strides, e.g. attention's [B, H, L, head_dim] straight away;
+//   - the half-split rotary pair layout, pair i = elements (i, i + hd/2);
+//   - INT8 output: symmetric per-(row, head) codes round(x * 127 / max|x|)
+//     with fp32 scales max|x| / 127, the quantised Q/K that the KOCPC Sol-H3
+//     article's 4x/8x B300 runs send between GPUs ("INT8 QKV ... transfer").
+// Same structure as qknorm_rope3d.cuh (ring, cursors, per-row angle tables,
+// G lanes per head).  With the half-split layout a thread's partner elements
+// (i + hd/2, or i - hd/2) sit in lane gl ^ G/2 of the same head: one 16-byte
+// shuffle per vector brings them over, and each thread writes only its own
+// elements.  With INT8 output the head's max |x| is a G-lane shuffle max;
+// the codes are rounded half to even from the fp32 value (one FMA with a
+// magic constant, then byte permutes).
+#pragma once
+#include "qknorm_rope3d.cuh"
+
+namespace sol {
+namespace qk {
+
+// Round-half-even of x*s for |x*s| <= 127 by adding 1.5 * 2^23: the fp32
+// sum has an ulp of 1, so one FMA rounds the exact product to an integer and
+// leaves it, as a two's-complement byte, in the low byte of the bit pattern.
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+__device__ __forceinline__ uint32_t code_bits(float x, float s) {
+  return __float_as_uint(fmaf(x, s, kRoundMagic));
+}
+// Low bytes of four words, in order, as one word.
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+__device__ __forceinline__ void st_stream8(void *gmem_dst, uint32_t lo, uint32_t hi) {
+  asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};\n" ::"l"(gmem_dst), "r"(lo), "r"(hi)
+               : "memory");
+}
+
+template <int G>
+__device__ __forceinline__ float group_max(float v) {
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+template <int G, int NT, int VPT, int R, int S, bool HALF, bool OUT8>
+__global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
+  using IO = Io<__nv_bfloat16>;
+  constexpr int E = IO::E;    // 8 elements per 16-byte vector
+  constexpr int P = E / 2;    // natural pairs (2e, 2e+1)
+  constexpr int Q = P / 2;    // float2 lanes of two rotary pairs (interleaved layout)
+  constexpr int VB = OUT8 ? 8 : 16;  // output bytes per vector
+  constexpr int TAB = 2 * R * kMaxPairs;
+  extern __shared__ __align__(16) unsigned char smem[];
+  double *freq = reinterpret_cast<double *>(smem);
+  float *cosb = reinterpret_cast<float *>(smem + kMaxPairs * 8);
+  float *sinb = cosb + TAB;
+  uint4 *ring = reinterpret_cast<uint4 *>(smem + header_bytes<R>());
+
+  const int tid = threadIdx.x;
+  const int gl = tid % G;
+  // first rotary pair of this thread's elements: interleaved, E/2 pairs per
+  // vector; half-split, one pair per element, positions mod hd/2
+  const int p0 = HALF ? (gl % (G / 2)) * E : gl * (E / 2);
+  const int64_t part_bytes = static_cast<int64_t>(a.nvec_q) * 16;
+
+  bool ok[VPT];
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) ok[k] = k * NT + tid < a.nvec_q;
+
+  // gamma: interleaved as in qknorm_rope3d.cuh; half-split as own / partner
+  // elements in natural pairs
+  float2 gev[2][Q], god[2][Q];   // interleaved
+  float2 gown[2][P], gpar[2][P]; // half-split
+#pragma unroll
+  for (int part = 0; part < 2; ++part) {
+    const uint4 *g = static_cast<const uint4 *>(part == 0 ? a.gamma_q : a.gamma_k);
+    if constexpr (HALF) {
+      if (g) {
+        IO::unpack(ld_shared_vec(g + gl), gown[part]);
+        IO::unpack(ld_shared_vec(g + (gl ^ (G / 2))), gpar[part]);
+      } else {
+#pragma unroll
+        for (int m = 0; m < P; ++m) gown[part][m] = gpar[part][m] = splat2(1.f);
+      }
+    } else {
+      if (g) {
+        IO::unpack_eo(ld_shared_vec(g + gl), gev[part], god[part]);
+      } else {
+#pragma unroll
+        for (int m = 0; m < Q; ++m) gev[part][m] = god[part][m] = splat2(1.f);
+      }
+    }
+  }
+  for (int p = tid; p < a.npairs; p += NT)
+    freq[p] = pow(static_cast<double>(a.theta), -2.0 * p / a.head_dim);
+
+  int64_t begin;
+  int count;
+  cta_rows(a.rows, blockIdx.x, gridDim.x, begin, count);
+  const int iters = (count + R - 1) / R;
+  const unsigned char *src_c = static_cast<const unsigned char *>(a.qkv) + begin * a.ld_qkv_bytes;
+  auto slot = [&](int s, int q, int part, int k) -> uint4 * {
+    return &ring[(((s * R + q) * 2 + part) * VPT + k) * NT + tid];
+  };
+  auto issue = [&](int it, int s) {
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      const int j = it * R + q;
+      if (j < count) {
+        const unsigned char *src = src_c + j * a.ld_qkv_bytes;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          const uint4 *ps = reinterpret_cast<const uint4 *>(src + part * part_bytes) + tid;
+#pragma unroll
+          for (int k = 0; k < VPT; ++k)
+            if (ok[k]) cp_async16(slot(s, q, part, k), ps + k * NT);
+        }
+      }
+    }
+    cp_async_commit();
+  };
+
+#pragma unroll
+  for (int s = 0; s < S - 1; ++s) issue(s, s);
+  __syncthreads();
+
+  TokenCursor tok;
+  tok.init(begin, a.L);
+  GridCursor pos;
+  pos.init(tok.r, a.n_video, a.HW, a.W);
+  int cons = 0;
+  int buf = 0;
+  for (int it = 0; it < iters; ++it) {
+    issue(it + S - 1, cons == 0 ? S - 1 : cons - 1);
+    int pt[R], ph[R], pw[R];
+    {
+      TokenCursor t2 = tok;
+      GridCursor g2 = pos;
+#pragma unroll
+      for (int q = 0; q < R; ++q) {
+        pt[q] = g2.t;
+        ph[q] = g2.h;
+        pw[q] = g2.w;
+        t2.next(a.L);
+        g2.next(t2.r, a.n_video, a.H, a.W);
+      }
+    }
+    for (int idx = tid; idx < R * a.npairs; idx += NT) {
+      int q = 0, p = idx;
+#pragma unroll
+      for (int qq = 1; qq < R; ++qq)
+        if (p >= a.npairs) {
+          p -= a.npairs;
+          q = qq;
+        }
+      int at = pw[0];
+#pragma unroll
+      for (int qq = 0; qq < R; ++qq)
+        if (q == qq) at = p < a.sec_t ? pt[qq] : (p < a.sec_th ? ph[qq] : pw[qq]);
+      const double ang = static_cast<double>(at) * freq[p];
+      const double turns = rint(ang * kInv2Pi);
+      const float red = static_cast<float>(fma(-turns, k2Pi, ang));
+      float sv, cv;
+      sincosf(red, &sv, &cv);
+      cosb[(buf * R + q) * kMaxPairs + p] = cv;
+      sinb[(buf * R + q) * kMaxPairs + p] = sv;
+    }
+
+    cp_async_wait<S - 1>();
+    __syncthreads();
+
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      const int j = it * R + q;
+      if (j < count) {
+        const float *ct = &cosb[(buf * R + q) * kMaxPairs + p0];
+        const float *st = &sinb[(buf * R + q) * kMaxPairs + p0];
+        const int64_t row_off = static_cast<int64_t>(tok.b) * a.out_sb +
+                                static_cast<int64_t>(tok.r) * a.out_sr;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          // rotation coefficients of this thread's elements, gamma folded in
+          float2 c0[Q], ns1[Q], s0[Q], c1[Q];  // interleaved
+          float2 ca[P], sb[P];                 // half-split: own*c + partner*(+-s)
+          if constexpr (HALF) {
+            const float sgn = gl >= G / 2 ? 1.f : -1.f;
+#pragma unroll
+            for (int m = 0; m < P; ++m) {
+              const float2 cc = *reinterpret_cast<const float2 *>(ct + 2 * m);
+              const float2 ss = *reinterpret_cast<const float2 *>(st + 2 * m);
+              ca[m] = mul2(gown[part][m], cc);
+              sb[m] = mul2(gpar[part][m], make_float2(sgn * ss.x, sgn * ss.y));
+            }
+          } else {
+#pragma unroll
+            for (int m = 0; m < Q; ++m) {
+              const float2 cs = *reinterpret_cast<const float2 *>(ct + 2 * m);
+              const float2 sn = *reinterpret_cast<const float2 *>(st + 2 * m);
+              c0[m] = mul2(gev[part][m], cs);
+              s0[m] = mul2(gev[part][m], sn);
+              ns1[m] = mul2(god[part][m], make_float2(-sn.x, -sn.y));
+              c1[m] = mul2(god[part][m], cs);
+            }
+          }
+          unsigned char *obase = static_cast<unsigned char *>(part == 0 ? a.q_out : a.k_out) +
+                                 row_off;
+          float *scale_row = OUT8 ? (part == 0 ? a.q_scale : a.k_scale) +
+                                        (begin + j) * static_cast<int64_t>(a.n_heads)
+                                  : nullptr;
+#pragma unroll
+          for (int k = 0; k < VPT; ++k) {
+            const int v = k * NT + tid;
+            uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+            if (ok[k]) xv = *slot(cons, q, part, k);
+            float o[E];  // rotated outputs in element order
+            if constexpr (HALF) {
+              uint4 pv;
+              pv.x = __shfl_xor_sync(0xffffffffu, xv.x, G / 2);
+              pv.y = __shfl_xor_sync(0xffffffffu, xv.y, G / 2);
+              pv.z = __shfl_xor_sync(0xffffffffu, xv.z, G / 2);
+              pv.w = __shfl_xor_sync(0xffffffffu, xv.w, G / 2);
+              float2 own[P], par[P];
+              IO::unpack(xv, own);
+              IO::unpack(pv, par);
+              float2 acc = mul2(own[0], own[0]);
+#pragma unroll
+              for (int m = 1; m < P; ++m) acc = fma2(own[m], own[m], acc);
+              const float ssq = group_sum<G>(acc.x + acc.y);
+              const float2 inv2 = splat2(rsqrtf(fmaf(ssq, a.inv_hd, a.eps)));
+#pragma unroll
+              for (int m = 0; m < P; ++m) {
+                const float2 u = mul2(fma2(own[m], ca[m], mul2(par[m], sb[m])), inv2);
+                o[2 * m] = u.x;
+                o[2 * m + 1] = u.y;
+              }
+            } else {
+              float2 ev[Q], od[Q];
+              IO::unpack_eo(xv, ev, od);
+              float2 acc = mul2(ev[0], ev[0]);
+              acc = fma2(od[0], od[0], acc);
+#pragma unroll
+              for (int m = 1; m < Q; ++m) {
+                acc = fma2(ev[m], ev[m], acc);
+                acc = fma2(od[m], od[m], acc);
+              }
+              const float ssq = group_sum<G>(acc.x + acc.y);
+              const float2 inv2 = splat2(rsqrtf(fmaf(ssq, a.inv_hd, a.eps)));
+#pragma unroll
+              for (int m = 0; m < Q; ++m) {
+                const float2 u0 = mul2(fma2(od[m], ns1[m], mul2(ev[m], c0[m])), inv2);
+                const float2 u1 = mul2(fma2(od[m], c1[m], mul2(ev[m], s0[m])), inv2);
+                o[4 * m + 0] = u0.x;
+                o[4 * m + 1] = u1.x;
+                o[4 * m + 2] = u0.y;
+                o[4 * m + 3] = u1.y;
+              }
+            }
+            const int head = v / G;
+            unsigned char *dst = obase + static_cast<int64_t>(head) * a.out_sh + (v % G) * VB;
+            if constexpr (OUT8) {
+              float amax = 0.f;
+#pragma unroll
+              for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(o[e]));
+              amax = group_max<G>(amax);
+              const float is = amax > 0.f ? 127.f / amax : 0.f;
+              uint32_t c[E];
+#pragma unroll
+              for (int e = 0; e < E; ++e) c[e] = code_bits(o[e], is);
+              if (ok[k]) {
+                st_stream8(dst, pack_low_bytes(c[0], c[1], c[2], c[3]),
+                           pack_low_bytes(c[4], c[5], c[6], c[7]));
+                if (gl == 0) scale_row[head] = amax / 127.f;
+              }
+            } else {
+              float2 pr[P];
+#pragma unroll
+              for (int m = 0; m < P; ++m) pr[m] = make_float2(o[2 * m], o[2 * m + 1]);
+              if (ok[k]) st_stream16(dst, IO::pack(pr));
+            }
+          }
+        }
+        tok.next(a.L);
+        pos.next(tok.r, a.n_video, a.H, a.W);
+      }
+    }
+    buf ^= 1;
+    cons = (cons + 1 == S) ? 0 : cons + 1;
+  }
+  cp_async_wait<0>();
+}
+
+template <int G, int NT, int VPT, bool HALF, bool OUT8>
+cudaError_t launch_ex(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
+  constexpr int R = VPT <= 6 ? 2 : 1;
+  constexpr int S = 2;
+  const void *fn =
+      reinterpret_cast<const void *>(&qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8>);
+  const size_t smem = header_bytes<R>() + static_cast<size_t>(S) * R * 2 * VPT * NT * 16;
+  const int per_sm = resident_blocks(fn, NT, smem);
+  if (per_sm <= 0) return cudaErrorInvalidConfiguration;
+  int64_t grid = static_cast<int64_t>(per_sm) * device_sms();
+  if (grid > a.rows) grid = a.rows;
+  if (geo) *geo = Geometry{NT, VPT, S, smem, static_cast<int>(grid)};
+  qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8>
+      <<<static_cast<unsigned>(grid), NT, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int G, bool HALF, bool OUT8>
+cudaError_t dispatch_ex(const QkArgs &a, int threads, int vpt, cudaStream_t stream,
+                        Geometry *geo) {
+#define SOL_CASE(NT, V) \
+  if (threads == NT && vpt == V) return launch_ex<G, NT, V, HALF, OUT8>(a, stream, geo);
+  SOL_SPLITS(SOL_CASE)
+#undef SOL_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace qk
+}  // namespace sol

@@ -1,0 +1,29 @@
+// QKNorm + 3D RoPE epilogue variants with bf16 output, for
+// head_dim 64, 128 or 256 (G = 8, 16, 32 lanes per head) and either rotary
+// pair layout.
+#include "qknorm_rope3d_ex.cuh"
+
+namespace sol {
+
+cudaError_t launch_qknorm_rope3d_ex_bf16out(const QkArgs &a, bool half_split, cudaStream_t stream,
+                                           Geometry *geo) {
+  const int G = a.head_dim * 2 / 16;
+  if (a.npairs > qk::kMaxPairs) return cudaErrorInvalidValue;
+  int threads = 0, vpt = 0;
+  if (!pick_split(a.nvec_q, &threads, &vpt)) return cudaErrorInvalidValue;
+  switch (G) {
+    case 8:
+      return half_split ? qk::dispatch_ex<8, true, false>(a, threads, vpt, stream, geo)
+                        : qk::dispatch_ex<8, false, false>(a, threads, vpt, stream, geo);
+    case 16:
+      return half_split ? qk::dispatch_ex<16, true, false>(a, threads, vpt, stream, geo)
+                        : qk::dispatch_ex<16, false, false>(a, threads, vpt, stream, geo);
+    case 32:
+      return half_split ? qk::dispatch_ex<32, true, false>(a, threads, vpt, stream, geo)
+                        : qk::dispatch_ex<32, false, false>(a, threads, vpt, stream, geo);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace sol

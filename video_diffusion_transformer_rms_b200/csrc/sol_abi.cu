@@ -325,6 +325,111 @@ sol_status sol_gate_residual_rms_adaln(const void *h, const void *branch, const 
   return ok();
 }
 
+sol_status sol_qknorm_rope3d_ex(const void *qkv, int64_t ld_qkv, void *q_out, void *k_out,
+                                const sol_qk_layout *layout, const void *gamma_q,
+                                const void *gamma_k, int64_t B, int64_t T, int64_t H, int64_t W,
+                                int64_t n_audio, int64_t n_heads, int64_t head_dim, int64_t sec_t,
+                                int64_t sec_h, int64_t sec_w, float eps, float theta,
+                                sol_dtype dtype, sol_stream_t stream) {
+  const char *fn = "sol_qknorm_rope3d_ex";
+  if (!layout) return fail(SOL_ERR_INVALID_ARG, "%s: layout must be non-null", fn);
+  if (dtype != SOL_BF16)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: bf16 input only", fn);
+  if (B < 0 || T < 0 || H < 0 || W < 0 || n_audio < 0 || n_heads <= 0)
+    return fail(SOL_ERR_INVALID_ARG, "%s: B, T, H, W, n_audio must be >= 0, n_heads > 0", fn);
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: head_dim must be 64, 128 or 256 (got %lld)", fn,
+                (long long)head_dim);
+  if (sec_t < 0 || sec_h < 0 || sec_w < 0 || sec_t + sec_h + sec_w != head_dim / 2)
+    return fail(SOL_ERR_INVALID_ARG, "%s: sections must sum to head_dim/2", fn);
+  if (!(eps >= 0.f) || !(theta > 0.f))
+    return fail(SOL_ERR_INVALID_ARG, "%s: need eps >= 0 and theta > 0", fn);
+  if (layout->stride_b < 0 || layout->stride_row < 0 || layout->stride_head < 0)
+    return fail(SOL_ERR_INVALID_ARG, "%s: strides must be >= 0", fn);
+  if (T > kMaxRows || H > kMaxRows || W > kMaxRows || n_audio > kMaxRows || B > kMaxRows ||
+      H * W > kMaxRows || T * H * W > kMaxRows || T * H * W + n_audio > kMaxRows ||
+      B * (T * H * W + n_audio) > kMaxRows)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: B*L and H*W must be below 2^31", fn);
+  const int64_t n_video = T * H * W;
+  const int64_t L = n_video + n_audio;
+  const int64_t rows = B * L;
+  const int64_t D = n_heads * head_dim;
+  if (ld_qkv < 2 * D) return fail(SOL_ERR_INVALID_ARG, "%s: need ld_qkv >= 2*D", fn);
+  if (rows == 0) return ok();
+  const bool int8 = layout->int8_out != 0;
+  if (!qkv || !q_out || !k_out || (int8 && (!layout->q_scale || !layout->k_scale)))
+    return fail(SOL_ERR_INVALID_ARG, "%s: qkv, q_out, k_out (and scales) must be non-null", fn);
+  if (2 * D * 2 > kMaxRowBytesQk)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: 2*D=%lld exceeds %lld elements", fn, (long long)(2 * D),
+                (long long)(kMaxRowBytesQk / 2));
+  const int oes = int8 ? 1 : 2;     // output element size
+  const int vb = int8 ? 8 : 16;     // output bytes per thread vector
+  const int64_t sb = layout->stride_b * oes, sr = layout->stride_row * oes,
+                sh = layout->stride_head * oes;
+  if (!aligned16(qkv) || (ld_qkv * 2) % 16 || (gamma_q && !aligned16(gamma_q)) ||
+      (gamma_k && !aligned16(gamma_k)) || reinterpret_cast<uintptr_t>(q_out) % vb ||
+      reinterpret_cast<uintptr_t>(k_out) % vb || sb % vb || sr % vb || sh % vb ||
+      (int8 && ((reinterpret_cast<uintptr_t>(layout->q_scale) & 3u) ||
+                (reinterpret_cast<uintptr_t>(layout->k_scale) & 3u))))
+    return fail(SOL_ERR_MISALIGNED, "%s: pointers and strides must be aligned", fn);
+  // byte extent of one output: last element + 1
+  const int64_t ext = (B - 1) * sb + (L - 1) * sr + (n_heads - 1) * sh + head_dim * oes;
+  const Span qs = span_of(q_out, 1, 0, ext), ks = span_of(k_out, 1, 0, ext);
+  const Span in = span_of(qkv, rows, ld_qkv * 2, 2 * D * 2);
+  if (spans_overlap(qs, in) || spans_overlap(ks, in) || spans_overlap(qs, ks))
+    return fail(SOL_ERR_INVALID_ARG, "%s: q_out and k_out must overlap neither qkv nor each other",
+                fn);
+  if (int8) {
+    const int64_t sc = rows * n_heads * 4;
+    const Span a1 = span_of(layout->q_scale, 1, 0, sc), a2 = span_of(layout->k_scale, 1, 0, sc);
+    for (const Span &z : {a1, a2})
+      if (spans_overlap(z, qs) || spans_overlap(z, ks) || spans_overlap(z, in))
+        return fail(SOL_ERR_INVALID_ARG, "%s: a scale array overlaps a tensor", fn);
+    if (spans_overlap(a1, a2))
+      return fail(SOL_ERR_INVALID_ARG, "%s: q_scale and k_scale overlap", fn);
+  }
+  for (const void *g : {gamma_q, gamma_k}) {
+    if (!g) continue;
+    const Span gs = span_of(g, 1, 0, head_dim * 2);
+    if (spans_overlap(gs, qs) || spans_overlap(gs, ks))
+      return fail(SOL_ERR_INVALID_ARG, "%s: an output overlaps gamma", fn);
+  }
+
+  QkArgs a{};
+  a.qkv = qkv;
+  a.q_out = q_out;
+  a.k_out = k_out;
+  a.gamma_q = gamma_q;
+  a.gamma_k = gamma_k;
+  a.ld_qkv_bytes = ld_qkv * 2;
+  a.ld_out_bytes = 0;
+  a.rows = rows;
+  a.L = static_cast<int>(L);
+  a.n_video = static_cast<int>(n_video);
+  a.HW = static_cast<int>(H * W);
+  a.H = static_cast<int>(H);
+  a.W = static_cast<int>(W);
+  a.nvec_q = static_cast<int>(D * 2 / 16);
+  a.npairs = static_cast<int>(head_dim / 2);
+  a.sec_t = static_cast<int>(sec_t);
+  a.sec_th = static_cast<int>(sec_t + sec_h);
+  a.head_dim = static_cast<int>(head_dim);
+  a.eps = eps;
+  a.inv_hd = static_cast<float>(1.0 / static_cast<double>(head_dim));
+  a.theta = theta;
+  a.out_sb = sb;
+  a.out_sr = sr;
+  a.out_sh = sh;
+  a.q_scale = layout->q_scale;
+  a.k_scale = layout->k_scale;
+  a.n_heads = static_cast<int>(n_heads);
+  const bool half = layout->half_split != 0;
+  cudaError_t e = int8 ? launch_qknorm_rope3d_ex_int8out(a, half, stream, nullptr)
+                       : launch_qknorm_rope3d_ex_bf16out(a, half, stream, nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_qknorm_rope3d_ex launch");
+  return ok();
+}
+
 size_t sol_residual_change_workspace_bytes(int64_t B) {
   return B <= 0 ? 0 : static_cast<size_t>(B) * kMaxChangeCtas * 2 * sizeof(double);
 }

@@ -89,6 +89,14 @@ struct QkArgs {
   float eps;
   float inv_hd;
   float theta;
+  // epilogue variants only (sol_qknorm_rope3d_ex): output byte strides per
+  // sample, token row and head; per-(row, head) fp32 scales for INT8 output
+  int64_t out_sb;
+  int64_t out_sr;
+  int64_t out_sh;
+  float *q_scale;
+  float *k_scale;
+  int n_heads;
 };
 
 // First-Block-Cache change detector.  `partial` is the caller's workspace:
@@ -122,6 +130,10 @@ cudaError_t launch_residual_change_noalloc(ChangeArgs a, int dtype, cudaStream_t
                                            Geometry *geo);
 cudaError_t launch_qknorm_rope3d_f32(const QkArgs &a, cudaStream_t stream, Geometry *geo);
 cudaError_t launch_qknorm_rope3d_bf16(const QkArgs &a, cudaStream_t stream, Geometry *geo);
+cudaError_t launch_qknorm_rope3d_ex_bf16out(const QkArgs &a, bool half_split, cudaStream_t stream,
+                                           Geometry *geo);
+cudaError_t launch_qknorm_rope3d_ex_int8out(const QkArgs &a, bool half_split, cudaStream_t stream,
+                                           Geometry *geo);
 inline cudaError_t launch_qknorm_rope3d(const QkArgs &a, int dtype, cudaStream_t stream,
                                         Geometry *geo) {
   return dtype == 0 ? launch_qknorm_rope3d_f32(a, stream, geo)
