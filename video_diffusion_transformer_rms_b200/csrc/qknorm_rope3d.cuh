@@ -239,7 +239,7 @@ template <typename T, int G>
 cudaError_t dispatch(const QkArgs &a, int threads, int vpt, cudaStream_t stream, Geometry *geo) {
 #define SOL_CASE(NT, V) \
   if (threads == NT && vpt == V) return launch<T, G, NT, V>(a, stream, geo);
-  SOL_SPLITS(SOL_CASE)
+  SOL_QK_SPLITS(SOL_CASE)
 #undef SOL_CASE
   return cudaErrorInvalidValue;
 }

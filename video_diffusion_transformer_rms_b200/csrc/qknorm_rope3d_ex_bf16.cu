@@ -10,7 +10,7 @@ cudaError_t launch_qknorm_rope3d_ex_bf16out(const QkArgs &a, bool half_split, cu
   const int G = a.head_dim * 2 / 16;
   if (a.npairs > qk::kMaxPairs) return cudaErrorInvalidValue;
   int threads = 0, vpt = 0;
-  if (!pick_split(a.nvec_q, &threads, &vpt)) return cudaErrorInvalidValue;
+  if (!pick_split_qk(a.nvec_q, &threads, &vpt)) return cudaErrorInvalidValue;
   switch (G) {
     case 8:
       return half_split ? qk::dispatch_ex<8, true, false>(a, threads, vpt, stream, geo)

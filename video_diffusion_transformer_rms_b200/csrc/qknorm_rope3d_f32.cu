@@ -9,7 +9,7 @@ cudaError_t launch_qknorm_rope3d_f32(const QkArgs &a, cudaStream_t stream, Geome
   const int G = a.head_dim * esize / 16;  // lanes per head
   if (a.npairs > qk::kMaxPairs) return cudaErrorInvalidValue;
   int threads = 0, vpt = 0;
-  if (!pick_split(a.nvec_q, &threads, &vpt)) return cudaErrorInvalidValue;
+  if (!pick_split_qk(a.nvec_q, &threads, &vpt)) return cudaErrorInvalidValue;
   switch (G) {
     case 2: return qk::dispatch<T, 2>(a, threads, vpt, stream, geo);
     case 4: return qk::dispatch<T, 4>(a, threads, vpt, stream, geo);

@@ -136,6 +136,19 @@ bool pick_split(int64_t nvec, int *threads, int *vpt) {
   return false;
 }
 
+bool pick_split_qk(int64_t nvec, int *threads, int *vpt) {
+  if (nvec <= 0) return false;
+  for (int t = 32; t <= kMaxThreads; t *= 2) {
+    const int64_t v = (nvec + t - 1) / t;
+    if (v <= 3 || (t == kMaxThreads && v <= kMaxVpt)) {
+      *threads = t;
+      *vpt = static_cast<int>(v);
+      return true;
+    }
+  }
+  return false;
+}
+
 }  // namespace sol
 
 using namespace sol;
