@@ -50,6 +50,8 @@ KERNEL_SOURCES = {
 }
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 ORACLE_SECONDS_PER_ROW = 0.4e-3  # all three oracle ops on one clip row (estimate)
 
 
@@ -345,6 +347,7 @@ def run_ours(args):
                            "bytes_per_token": elems * D * w.esize,
                            "GB_per_s": round(nbytes / (ms / 1e3) / 1e9, 1)}
     del ws
+    next_rows["gemm_gelu"] = time_gemm_gelu(w, D, dev, stream)
 
     # ---- end to end through the public API, host buffers ------------------
     e2e = run_e2e(args, w, t, stream, api)
@@ -395,6 +398,58 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     dist.barrier()
     dist.shutdown()
+
+
+def load_tensor_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback"
+
+
+def time_gemm_gelu(w, D, dev, stream):
+    """The MLP up-projection of one block, GELU fused in the epilogue: A = the
+    step's normalised tokens [rows, D], W1 [4D, D], bias [4D].  Compute bound:
+    2*rows*4D*D flops per launch, against the bf16 tensor peak."""
+    from video_diffusion_transformer_rms_b200 import _abi
+    M, N, K = w.rows, 4 * D, D
+    g = torch.Generator(device=dev).manual_seed(77)
+    A = torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16)
+    Wt = (torch.randn((N, K), generator=g, device=dev) * K ** -0.5).to(torch.bfloat16)
+    bias = (0.1 * torch.randn((N,), generator=g, device=dev)).to(torch.bfloat16)
+    C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    need = _abi.sol_gemm_gelu_workspace_bytes(M, N, K)
+    gws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    s = stream.cuda_stream
+
+    def fn():
+        return _abi.sol_gemm_gelu(A.data_ptr(), Wt.data_ptr(), bias.data_ptr(), C.data_ptr(),
+                                  M, N, K, gws.data_ptr(), need, s)
+
+    for _ in range(3):
+        _abi.check(fn())
+    n_it = 10
+    ea = torch.cuda.Event(enable_timing=True)
+    eb = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    ea.record(stream)
+    for _ in range(n_it):
+        _abi.check(fn())
+    eb.record(stream)
+    torch.cuda.synchronize()
+    ms = dist.max_over_ranks(ea.elapsed_time(eb) / n_it)
+    flops = 2.0 * M * N * K
+    tflops = flops / (ms / 1e3) / 1e12
+    burst, sustained, kind = load_tensor_peaks()
+    del A, Wt, bias, C, gws
+    return {"ms": round(ms, 3), "M": M, "N": N, "K": K, "flops_per_launch": flops,
+            "TFLOP_per_s": round(tflops, 1), "bound": "tensor",
+            f"frac_of_{kind}_bf16_burst": round(tflops / burst, 4),
+            f"frac_of_{kind}_bf16_sustained": round(tflops / sustained, 4),
+            "tokens_per_s": round(M / (ms / 1e3))}
 
 
 def run_e2e(args, w, t, stream, api):

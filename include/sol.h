@@ -303,6 +303,35 @@ sol_status sol_residual_change_noalloc(const void *cur, const void *prev,
                                        int64_t D, double *out, sol_dtype dtype,
                                        sol_stream_t stream);
 
+/*
+ * GEMM + bias + GELU in one kernel (Sol Video Inference Engine MiniMax-H3
+ * page, fusion table, row "GEMM + GELU": the MLP's activation-sized HBM round
+ * trip removed by applying GELU in the GEMM epilogue):
+ *
+ *   C[m][n] = gelu(sum_k A[m][k] * B[n][k] + bias[n]),
+ *   gelu(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))
+ *
+ * on the 5th-generation tensor cores (tcgen05 MMA, fp32 accumulators in
+ * tensor memory, TMA-staged operands).
+ *
+ *   A        [M, K] bf16 device, row-major (tokens).
+ *   B        [N, K] bf16 device, row-major (a Linear layer's weight).
+ *   bias     [N] bf16 device, or NULL.
+ *   C        [M, N] bf16 device, row-major; must not overlap A, B or bias.
+ *   M >= 0 (0 is a no-op), N, K > 0, each below 2^31; N and K multiples of
+ *   8 (16-byte rows); pointers 16-byte aligned.
+ *   workspace, workspace_bytes  device scratch of at least
+ *            sol_gemm_gelu_workspace_bytes(M, N, K) bytes (may be NULL/0 when
+ *            that is 0), owned by the caller.
+ */
+sol_status sol_gemm_gelu(const void *A, const void *B, const void *bias,
+                         void *C, int64_t M, int64_t N, int64_t K,
+                         void *workspace, size_t workspace_bytes,
+                         sol_stream_t stream);
+
+/* Workspace bytes sol_gemm_gelu needs for this problem on the current device. */
+size_t sol_gemm_gelu_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
 /* Static, human-readable name of a status code. */
 const char *sol_status_string(sol_status status);
 

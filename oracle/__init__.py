@@ -211,6 +211,31 @@ def quantize_heads(x, n_heads, head_dim):
     return code, scale
 
 
+def widen(a):
+    """Exact float64 values of an oracle input array (float32, or uint16 bf16 bits)."""
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    if a.dtype == np.float32:
+        return a.astype(np.float64)
+    raise TypeError(f"unsupported oracle input dtype {a.dtype}")
+
+
+def gelu_tanh(x):
+    """GELU, tanh form (Hendrycks & Gimpel): 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))."""
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)))
+
+
+def gemm_gelu(A, B, bias=None):
+    """gelu_tanh(A @ B.T + bias) in fp64; A [M, K], B [N, K], bias [N]; the
+    matmul is numpy's (a library primitive), everything else is spelled out."""
+    x = widen(A) @ widen(B).T
+    if bias is not None:
+        x = x + widen(bias)[None, :]
+    return gelu_tanh(x)
+
+
 def ulp(v, dtype):
     """Unit in the last place of the I/O dtype at the (fp64) value v.
 

@@ -577,3 +577,50 @@ def test_half_split_identity_at_origin_gives_gamma():
                                    gamma_q=gq, gamma_k=gk)
     np.testing.assert_allclose(q[0], np.tile(gq.astype(np.float64), 2), rtol=1e-15)
     np.testing.assert_allclose(k[0], np.tile(-gk.astype(np.float64), 2), rtol=1e-15)
+
+
+# ----------------------------------------------------------------------------
+# GEMM + GELU
+# ----------------------------------------------------------------------------
+
+def test_gelu_tanh_closed_forms():
+    x = np.array([0.0, 0.5, 1.0, 2.0, 3.0, 10.0])
+    g = oracle.gelu_tanh(x)
+    assert g[0] == 0.0
+    # odd part: gelu(x) - gelu(-x) = x exactly for the tanh form
+    np.testing.assert_allclose(g - oracle.gelu_tanh(-x), x, rtol=1e-15, atol=1e-15)
+    # saturation: gelu(10) ~ 10, gelu(-10) ~ 0
+    assert abs(g[-1] - 10.0) < 1e-7 and abs(oracle.gelu_tanh(-10.0)) < 1e-7
+    # x = 1: sqrt(2/pi) * 1.044715 = 0.833554...; 0.5 * (1 + tanh(that)) = 0.841192
+    assert abs(g[2] - 0.841192) < 1e-6
+
+
+def test_gemm_gelu_brute_force_and_layout():
+    rng = np.random.default_rng(5)
+    M, N, K = 3, 4, 5
+    A = f32(rng.standard_normal((M, K)))
+    B = f32(rng.standard_normal((N, K)))
+    bias = f32(rng.standard_normal(N))
+    C = oracle.gemm_gelu(A, B, bias)
+    for m in range(M):
+        for n in range(N):
+            s = sum(float(A[m, k]) * float(B[n, k]) for k in range(K)) + float(bias[n])
+            g = 0.5 * s * (1 + math.tanh(math.sqrt(2 / math.pi) * (s + 0.044715 * s ** 3)))
+            assert abs(C[m, n] - g) < 1e-12
+    # B a permutation: C = gelu(A[:, perm] + bias) -- a transposed operand fails
+    K = N = 6
+    A = f32(rng.standard_normal((4, K)))
+    perm = np.array([3, 0, 5, 1, 4, 2])
+    P = np.zeros((N, K), dtype=np.float32)
+    P[np.arange(N), perm] = 1.0
+    np.testing.assert_allclose(oracle.gemm_gelu(A, P), oracle.gelu_tanh(A[:, perm]),
+                               rtol=1e-15, atol=1e-15)
+    # bias runs along N (one value per output column)
+    z = f32(np.zeros((2, K)))
+    b = f32(np.arange(N) - 2.5)
+    np.testing.assert_allclose(oracle.gemm_gelu(z, P, b), np.tile(oracle.gelu_tanh(b), (2, 1)))
+
+
+def test_widen_bf16_bits():
+    np.testing.assert_array_equal(oracle.widen(np.array([0x3F80, 0xC000, 0x4049], np.uint16)),
+                                  [1.0, -2.0, 3.140625])

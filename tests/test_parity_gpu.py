@@ -592,3 +592,46 @@ def test_qknorm_rope3d_ex_head_dims(hd, secs, half):
         else:
             assert_close(q, wq, f"hd={hd} half={half} q")
             assert_close(k, wk, f"hd={hd} half={half} k")
+
+
+
+# ----------------------------------------------------------------------------
+# GEMM + bias + GELU (tcgen05)
+# ----------------------------------------------------------------------------
+
+def _weights(N, K, seed):
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    return (torch.randn((N, K), generator=g, device=DEV) / K ** 0.5).to(torch.bfloat16)
+
+
+GEMM_SHAPES = [
+    (1, 8, 8), (127, 256, 64), (300, 520, 1032), (257, 384, 256), (1000, 1024, 5120),
+    (129, 264, 72),
+]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_gemm_gelu_shapes(M, N, K):
+    A = activation(M, K, torch.bfloat16, DEV, 101 + M, outliers=True)
+    Bw = _weights(N, K, 102 + N)
+    bias = vectors((N,), 0.0, 0.5, torch.bfloat16, DEV, 103)
+    for b in (None, bias):
+        C = api.gemm_gelu(A, Bw, b)
+        want = oracle.gemm_gelu(_o(A), _o(Bw), None if b is None else _o(b))
+        assert_close(C, want, f"gemm_gelu M={M} N={N} K={K} bias={b is not None}")
+
+
+def test_gemm_gelu_clip_mlp_shape_sampled():
+    # the 5 s clip's MLP up-projection: 126,552 tokens x (5120 -> 4 x 5120)
+    w = WORKLOADS["clip5s"]
+    M, K, N = w.rows, w.D, 4 * w.D
+    A = activation(M, K, torch.bfloat16, DEV, 104, outliers=True)
+    Bw = _weights(N, K, 105)
+    bias = vectors((N,), 0.0, 0.5, torch.bfloat16, DEV, 106)
+    C = api.gemm_gelu(A, Bw, bias)
+    torch.cuda.synchronize()
+    ids = sample_rows(M, w.L, w.n_video, w.B, 192, seed=107)
+    want = oracle.gemm_gelu(take_rows(A, ids), _o(Bw), _o(bias))
+    assert_close(take_rows_gpu(C, ids), want, "gemm_gelu clip MLP sampled")
+    C2 = api.gemm_gelu(A[:4096], Bw, bias)
+    assert torch.equal(C2, C[:4096])  # same tiles, same order: deterministic

@@ -73,6 +73,10 @@ def lib() -> ctypes.CDLL:
                                            i64, i64, i64, i64, i64, i64, i64, i64, i64, f, f,
                                            i, p]
         L.sol_qknorm_rope3d_ex.restype = i
+        L.sol_gemm_gelu.argtypes = [p, p, p, p, i64, i64, i64, p, ctypes.c_size_t, p]
+        L.sol_gemm_gelu.restype = i
+        L.sol_gemm_gelu_workspace_bytes.argtypes = [i64, i64, i64]
+        L.sol_gemm_gelu_workspace_bytes.restype = ctypes.c_size_t
         L.sol_qknorm_rope3d.argtypes = [p, i64, p, p, i64, p, p, i64, i64, i64, i64, i64,
                                         i64, i64, i64, i64, i64, f, f, i, p]
         L.sol_qknorm_rope3d.restype = i
@@ -152,6 +156,14 @@ def sol_qknorm_rope3d_ex(qkv, ld_qkv, q_out, k_out, layout, gamma_q, gamma_k, B,
     return lib().sol_qknorm_rope3d_ex(qkv, ld_qkv, q_out, k_out, ref, gamma_q, gamma_k, B, T,
                                       H, W, n_audio, n_heads, head_dim, sec_t, sec_h, sec_w,
                                       eps, theta, dtype, stream)
+
+
+def sol_gemm_gelu(A, B, bias, C, M, N, K, workspace, workspace_bytes, stream) -> int:
+    return lib().sol_gemm_gelu(A, B, bias, C, M, N, K, workspace, workspace_bytes, stream)
+
+
+def sol_gemm_gelu_workspace_bytes(M, N, K) -> int:
+    return lib().sol_gemm_gelu_workspace_bytes(M, N, K)
 
 
 def sol_status_string(status: int) -> str:

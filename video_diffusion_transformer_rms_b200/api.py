@@ -178,3 +178,25 @@ def qknorm_rope3d_ex(qkv: torch.Tensor, T: int, H: int, W: int, n_audio: int, n_
         W, n_audio, n_heads, head_dim, st, sh, sw, eps, theta,
         _dtype(qkv, gamma_q, gamma_k), _stream(stream)))
     return (q, k, qs, ks) if int8 else (q, k)
+
+
+def gemm_gelu(A: torch.Tensor, B: torch.Tensor, bias: Optional[torch.Tensor] = None,
+              out: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """C = gelu_tanh(A @ B.T + bias) on the tensor cores; A [M, K], B [N, K]
+    (a Linear weight), bias [N], all bf16; returns C [M, N] bf16."""
+    if A.dim() != 2 or B.dim() != 2 or A.shape[1] != B.shape[1]:
+        raise ValueError("A must be [M, K] and B [N, K]")
+    if not (A.is_contiguous() and B.is_contiguous()):
+        raise ValueError("A and B must be contiguous")
+    M, K = A.shape
+    N = B.shape[0]
+    C = torch.empty((M, N), dtype=A.dtype, device=A.device) if out is None else out
+    need = _abi.sol_gemm_gelu_workspace_bytes(M, N, K)
+    ws = torch.empty(need, dtype=torch.uint8, device=A.device) if need else None
+    _dtype(A, B, bias, C)
+    if A.dtype != torch.bfloat16:
+        raise TypeError("sol_gemm_gelu takes bf16 tensors")
+    _abi.check(_abi.sol_gemm_gelu(_ptr(A), _ptr(B), _ptr(bias), _ptr(C), M, N, K, _ptr(ws),
+                                  need, _stream(stream)))
+    return C

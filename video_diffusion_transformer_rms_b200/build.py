@@ -22,7 +22,9 @@ LIB = os.path.join(PKG, "libsol.so")
 
 SOURCES = ["sol_abi.cu", "rms_adaln.cu", "gate_residual.cu", "qknorm_rope3d_bf16.cu",
            "qknorm_rope3d_f32.cu", "qknorm_rope3d_ex_bf16.cu", "qknorm_rope3d_ex_int8.cu",
-           "residual_change.cu"]
+           "residual_change.cu", "gemm_gelu.cu"]
+# sources built against the CUTLASS / CuTe headers (the sm100 GEMM templates)
+CUTLASS_SOURCES = {"gemm_gelu.cu"}
 HEADERS = ["sol_device.cuh", "sol_launch.h", "qknorm_rope3d.cuh", "qknorm_rope3d_ex.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -35,6 +37,17 @@ def _nvcc():
         if c and os.path.exists(c):
             return c
     raise RuntimeError("nvcc not found: the CUDA toolkit is required to build libsol")
+
+
+def _cutlass_root():
+    """The CUTLASS tree vendored with flashinfer (headers only; no import)."""
+    import importlib.util
+    spec = importlib.util.find_spec("flashinfer")
+    for base in (spec.submodule_search_locations if spec else []) or []:
+        root = os.path.join(base, "data", "cutlass")
+        if os.path.isdir(os.path.join(root, "include", "cute")):
+            return root
+    raise RuntimeError("CUTLASS headers not found (expected flashinfer/data/cutlass)")
 
 
 def _digest():
@@ -64,6 +77,11 @@ def build(force: bool = False, verbose: bool = False) -> str:
         obj = os.path.join(BUILD, src.replace(".cu", ".o"))
         cmd = [nvcc, *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-c",
                os.path.join(CSRC, src), "-o", obj]
+        if src in CUTLASS_SOURCES:
+            cut = _cutlass_root()
+            cmd[1:1] = ["-I", os.path.join(cut, "include"), "-I",
+                        os.path.join(cut, "tools", "util", "include"),
+                        "-diag-suppress", "20012"]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE,

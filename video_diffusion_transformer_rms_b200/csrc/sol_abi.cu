@@ -443,6 +443,43 @@ sol_status sol_qknorm_rope3d_ex(const void *qkv, int64_t ld_qkv, void *q_out, vo
   return ok();
 }
 
+size_t sol_gemm_gelu_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0 || M > kMaxRows || N > kMaxRows || K > kMaxRows) return 0;
+  GemmArgs g{nullptr, nullptr, nullptr, nullptr, M, N, K};
+  return gemm_gelu_workspace_bytes(g);
+}
+
+sol_status sol_gemm_gelu(const void *A, const void *B, const void *bias, void *C, int64_t M,
+                         int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
+                         sol_stream_t stream) {
+  const char *fn = "sol_gemm_gelu";
+  if (M < 0 || N <= 0 || K <= 0)
+    return fail(SOL_ERR_INVALID_ARG, "%s: need M >= 0, N > 0, K > 0", fn);
+  if (M > kMaxRows || N > kMaxRows || K > kMaxRows)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: M, N, K must be below 2^31", fn);
+  if (M == 0) return ok();
+  if (!A || !B || !C) return fail(SOL_ERR_INVALID_ARG, "%s: A, B and C must be non-null", fn);
+  if (N % 8 || K % 8)
+    return fail(SOL_ERR_MISALIGNED, "%s: N and K must be multiples of 8 (N=%lld K=%lld)", fn,
+                (long long)N, (long long)K);
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C) || (bias && !aligned16(bias)))
+    return fail(SOL_ERR_MISALIGNED, "%s: pointers must be 16-byte aligned", fn);
+  const Span cs = span_of(C, 1, 0, M * N * 2);
+  if (spans_overlap(cs, span_of(A, 1, 0, M * K * 2)) ||
+      spans_overlap(cs, span_of(B, 1, 0, N * K * 2)) ||
+      (bias && spans_overlap(cs, span_of(bias, 1, 0, N * 2))))
+    return fail(SOL_ERR_INVALID_ARG, "%s: C must not overlap A, B or bias", fn);
+  GemmArgs g{A, B, bias, C, M, N, K};
+  const size_t need = gemm_gelu_workspace_bytes(g);
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return fail(SOL_ERR_INVALID_ARG, "%s: workspace needs %zu bytes", fn, need);
+  if (gemm_gelu_check(g) != 0)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: the GEMM templates reject this problem", fn);
+  cudaError_t e = launch_gemm_gelu(g, workspace, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_gemm_gelu launch");
+  return ok();
+}
+
 size_t sol_residual_change_workspace_bytes(int64_t B) {
   return B <= 0 ? 0 : static_cast<size_t>(B) * kMaxChangeCtas * 2 * sizeof(double);
 }

@@ -125,6 +125,18 @@ struct ChangeArgs {
   int ctas_per_sample;  // set by the launcher
 };
 
+// GEMM + bias + GELU: C[M, N] = gelu(A[M, K] . B[N, K]^T + bias[N]), bf16.
+struct GemmArgs {
+  const void *A;
+  const void *B;
+  const void *bias;  // may be null
+  void *C;
+  int64_t M, N, K;
+};
+size_t gemm_gelu_workspace_bytes(const GemmArgs &g);
+int gemm_gelu_check(const GemmArgs &g);
+cudaError_t launch_gemm_gelu(const GemmArgs &g, void *workspace, cudaStream_t stream);
+
 // dtype: 0 = fp32, 1 = bf16 (sol_dtype).  Each returns the launch error
 // (cudaSuccess if the kernel was enqueued) and fills `geo` if non-null.
 cudaError_t launch_rms_adaln(const RmsArgs &a, int dtype, cudaStream_t stream, Geometry *geo);
