@@ -2,13 +2,15 @@
 for profilers (ncu) that should capture a small, self-contained case.
 
     python -m video_diffusion_transformer_rms_b200.profile_case \
-        [--workload clip5s] [--frames 4] [--launches 1]
+        [--workload clip5s] [--frames 4] [--launches 1] [--kernel norm|gemm]
 
 The slice keeps the clip's H x W latent grid, D and head layout, takes the
 first `--frames` latent frames (T) and scales the audio rows by the same
 fraction.  Inputs are larger than L2 at the default 4 frames (16,384 rows:
 168 MB per activation, 503 MB of merged QKV), so DRAM counters stay
-meaningful while the device footprint stays near 1.5 GB.
+meaningful while the device footprint stays near 1.5 GB.  `--kernel gemm`
+runs the MLP up-projection with fused GELU on the same slice instead
+(A [rows, D], W1 [4D, D], C [rows, 4D]: about 1 GB at 4 frames).
 """
 import argparse
 import dataclasses
@@ -24,11 +26,14 @@ def main():
     ap.add_argument("--workload", default="clip5s", choices=sorted(WORKLOADS))
     ap.add_argument("--frames", type=int, default=4)
     ap.add_argument("--launches", type=int, default=1)
+    ap.add_argument("--kernel", default="norm", choices=["norm", "gemm"])
     args = ap.parse_args()
     full = WORKLOADS[args.workload]
     T = max(1, min(full.T, args.frames))
     n_audio = full.n_audio * T // full.T
     w = dataclasses.replace(full, name=f"{full.name}_slice{T}", T=T, n_audio=n_audio)
+    if args.kernel == "gemm":
+        return gemm_case(w, args.launches)
     t = make_inputs(w, "cuda")
     D = w.D
     x = t["x"].view(w.B, w.L, D)
@@ -46,6 +51,19 @@ def main():
         api.gate_residual(h, br, t["gate"], w.n_video, out=out)
     torch.cuda.synchronize()
     print(f"{w.name}: {w.rows} rows, D={D}, {args.launches} launch(es) of each kernel")
+
+
+def gemm_case(w, launches):
+    M, N, K = w.rows, 4 * w.D, w.D
+    g = torch.Generator(device="cuda").manual_seed(77)
+    A = torch.randn((M, K), generator=g, device="cuda").to(torch.bfloat16)
+    W1 = (torch.randn((N, K), generator=g, device="cuda") * K ** -0.5).to(torch.bfloat16)
+    bias = (0.1 * torch.randn((N,), generator=g, device="cuda")).to(torch.bfloat16)
+    C = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    for _ in range(launches):
+        api.gemm_gelu(A, W1, bias, out=C)
+    torch.cuda.synchronize()
+    print(f"{w.name}: gemm_gelu M={M} N={N} K={K}, {launches} launch(es)")
 
 
 if __name__ == "__main__":
