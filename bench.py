@@ -314,22 +314,48 @@ def run_ours(args):
     ws = torch.empty(_abi.sol_residual_change_workspace_bytes(w.B), dtype=torch.uint8,
                      device=dev)
     rc_out = torch.empty((w.B + 1, 3), dtype=torch.float64, device=dev)
+    # QKNorm+RoPE epilogue variants write into the step's q/k buffer (q in its
+    # first half, k in the second) or, for INT8, into code and scale buffers
+    half_bytes = w.rows * D * w.esize
+    q8 = torch.empty(2 * w.rows * D, dtype=torch.int8, device=dev)
+    s8 = torch.empty(2 * w.rows * w.n_heads, dtype=torch.float32, device=dev)
+    hd = w.head_dim
+    lay_bhsd = _abi.QkLayout(w.L * D, hd, w.L * hd, 0, 0, None, None)
+    lay_half = _abi.QkLayout(w.L * D, D, hd, 1, 0, None, None)
+    lay_int8 = _abi.QkLayout(w.L * D, D, hd, 0, 1, s8.data_ptr(),
+                             s8.data_ptr() + w.rows * w.n_heads * 4)
+
+    def k_qk_ex(lay, q_ptr, k_ptr):
+        return lambda: _abi.sol_qknorm_rope3d_ex(
+            p["qkv"], 3 * D, q_ptr, k_ptr, lay, p["gamma_q"], p["gamma_k"], w.B, w.T, w.H, w.W,
+            w.n_audio, w.n_heads, hd, st, sh_, sw, w.eps, w.theta, dt, s)
+
+    row = D * w.esize  # bytes of one D-wide bf16 row
     extra = {
-        # h_out = h + gate*branch and y = RMS-AdaLN(h_out) in one pass: 4 D elements / row
-        "gate_residual_rms_adaln": (4, lambda: _abi.sol_gate_residual_rms_adaln(
+        # h_out = h + gate*branch and y = RMS-AdaLN(h_out) in one pass: 4 D-wide rows
+        "gate_residual_rms_adaln": (4 * row, lambda: _abi.sol_gate_residual_rms_adaln(
             p["h"], p["branch"], p["gate"], out.data_ptr(), y.data_ptr(), p["scale"],
             p["shift"], None, w.B, w.L, w.n_video, D, w.eps, dt, s)),
         # First-Block-Cache change of h against branch (stand-ins for two steps'
-        # residuals): 2 D elements read per row; with the cache refresh 3 D
-        "residual_change": (2, lambda: _abi.sol_residual_change(
+        # residuals): 2 D-wide rows read; with the cache refresh 3
+        "residual_change": (2 * row, lambda: _abi.sol_residual_change(
             p["h"], p["branch"], None, w.B, w.L, D, rc_out.data_ptr(), ws.data_ptr(),
             ws.numel(), dt, s)),
-        "residual_change_refresh": (3, lambda: _abi.sol_residual_change(
+        "residual_change_refresh": (3 * row, lambda: _abi.sol_residual_change(
             p["h"], p["branch"], out.data_ptr(), w.B, w.L, D, rc_out.data_ptr(),
             ws.data_ptr(), ws.numel(), dt, s)),
+        # q, k read and written (4 rows) in attention's [B, H, L, hd] layout
+        "qknorm_rope3d_ex_bhsd": (4 * row, k_qk_ex(lay_bhsd, qk.data_ptr(),
+                                                   qk.data_ptr() + half_bytes)),
+        # half-split rotary pairs
+        "qknorm_rope3d_ex_half": (4 * row, k_qk_ex(lay_half, qk.data_ptr(),
+                                                   qk.data_ptr() + half_bytes)),
+        # INT8 codes (2D bytes) + fp32 scales per (row, head) for q and k
+        "qknorm_rope3d_ex_int8": (2 * row + 2 * D + 2 * w.n_heads * 4,
+                                  k_qk_ex(lay_int8, q8.data_ptr(), q8.data_ptr() + w.rows * D)),
     }
     next_rows = {}
-    for name, (elems, fn) in extra.items():
+    for name, (bytes_per_row, fn) in extra.items():
         for _ in range(5):
             _abi.check(fn())
         n_it = 200
@@ -342,11 +368,11 @@ def run_ours(args):
         eb.record(stream)
         torch.cuda.synchronize()
         ms = dist.max_over_ranks(ea.elapsed_time(eb) / n_it)
-        nbytes = elems * D * w.esize * w.rows
+        nbytes = bytes_per_row * w.rows
         next_rows[name] = {"ms": round(ms, 4), "tokens_per_s": round(w.rows / (ms / 1e3)),
-                           "bytes_per_token": elems * D * w.esize,
+                           "bytes_per_token": bytes_per_row,
                            "GB_per_s": round(nbytes / (ms / 1e3) / 1e9, 1)}
-    del ws
+    del ws, q8, s8
     next_rows["gemm_gelu"] = time_gemm_gelu(w, D, dev, stream)
 
     # ---- end to end through the public API, host buffers ------------------

@@ -635,3 +635,35 @@ def test_gemm_gelu_clip_mlp_shape_sampled():
     assert_close(take_rows_gpu(C, ids), want, "gemm_gelu clip MLP sampled")
     C2 = api.gemm_gelu(A[:4096], Bw, bias)
     assert torch.equal(C2, C[:4096])  # same tiles, same order: deterministic
+
+
+@pytest.mark.parametrize("half", [False, True])
+def test_qknorm_rope3d_ex_int8_edge_heads(half):
+    # per row: a normal head, an all-zero head, a head of tiny normal values
+    # (x * 2^-110, so max|u| < 2^-96 and the kernel rescales before dividing),
+    # and a head with one 1e4 outlier; q and k get different heads
+    T, H, W, na, nh, hd = 2, 3, 4, 5, 4, 128
+    L = T * H * W + na
+    D = nh * hd
+    base = activation(L, 3 * D, torch.float32, DEV, 71, outliers=False).view(L, 3, nh, hd)
+    x = base.clone()
+    for part, (zero, tiny, spike) in enumerate([(1, 2, 3), (2, 3, 1)]):
+        x[:, part, zero] = 0.0
+        x[:, part, tiny] = torch.sign(base[:, part, tiny]) * (1 + base[:, part, tiny].abs()) * 2.0 ** -110
+        x[:, part, spike, 17] = 1.0e4
+    qkv = x.to(torch.bfloat16).view(1, L, 3 * D)
+    gq = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 72)
+    gk = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 73)
+    res = api.qknorm_rope3d_ex(qkv, T, H, W, na, nh, hd, (16, 24, 24), gq, gk, layout="bshd",
+                               half_split=half, int8=True)
+    torch.cuda.synchronize()
+    wq, wk = oracle.qknorm_rope3d_ex(_o(qkv.view(L, 3 * D)), T, H, W, na, nh, hd, (16, 24, 24),
+                                     1e-6, 1e4, half, _o(gq), _o(gk))
+    q, k, qs, ks = res
+    _check_int8(q.reshape(L, D), qs, wq, nh, hd, f"edge half={half} q")
+    _check_int8(k.reshape(L, D), ks, wk, nh, hd, f"edge half={half} k")
+    # the zero heads: scale 0 and every code 0
+    assert torch.all(qs.view(L, nh)[:, 1] == 0) and torch.all(q.view(L, nh, hd)[:, 1] == 0)
+    assert torch.all(ks.view(L, nh)[:, 2] == 0) and torch.all(k.view(L, nh, hd)[:, 2] == 0)
+    # the tiny heads use the full code range
+    assert int(q.view(L, nh, hd)[:, 2].abs().amax()) == 127

@@ -10,9 +10,10 @@
 // G lanes per head).  With the half-split layout a thread's partner elements
 // (i + hd/2, or i - hd/2) sit in lane gl ^ G/2 of the same head: one 16-byte
 // shuffle per vector brings them over, and each thread writes only its own
-// elements.  With INT8 output the head's max |x| is a G-lane shuffle max;
-// the codes are rounded half to even from the fp32 value (one FMA with a
-// magic constant, then byte permutes).
+// elements.  With INT8 output the head's max |x| is a G-lane shuffle max,
+// run side by side with the sum of squares (the 1/rms factor cancels from
+// the codes); the codes are rounded half to even from the fp32 value (one FMA
+// with a magic constant, then byte permutes).
 #pragma once
 #include "qknorm_rope3d.cuh"
 
@@ -23,9 +24,6 @@ namespace qk {
 // sum has an ulp of 1, so one FMA rounds the exact product to an integer and
 // leaves it, as a two's-complement byte, in the low byte of the bit pattern.
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
-__device__ __forceinline__ uint32_t code_bits(float x, float s) {
-  return __float_as_uint(fmaf(x, s, kRoundMagic));
-}
 // Low bytes of four words, in order, as one word.
 __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
@@ -34,13 +32,6 @@ __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint3
 __device__ __forceinline__ void st_stream8(void *gmem_dst, uint32_t lo, uint32_t hi) {
   asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};\n" ::"l"(gmem_dst), "r"(lo), "r"(hi)
                : "memory");
-}
-
-template <int G>
-__device__ __forceinline__ float group_max(float v) {
-#pragma unroll
-  for (int o = G / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
 }
 
 template <int G, int NT, int VPT, int R, int S, bool HALF, bool OUT8>
@@ -213,7 +204,10 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
             const int v = k * NT + tid;
             uint4 xv = make_uint4(0u, 0u, 0u, 0u);
             if (ok[k]) xv = *slot(cons, q, part, k);
-            float o[E];  // rotated outputs in element order
+            // rotated outputs in element order, not yet multiplied by the
+            // head's 1/rms; acc: this thread's part of the sum of squares
+            float o[E];
+            float2 acc;
             if constexpr (HALF) {
               uint4 pv;
               pv.x = __shfl_xor_sync(0xffffffffu, xv.x, G / 2);
@@ -223,33 +217,29 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
               float2 own[P], par[P];
               IO::unpack(xv, own);
               IO::unpack(pv, par);
-              float2 acc = mul2(own[0], own[0]);
+              acc = mul2(own[0], own[0]);
 #pragma unroll
               for (int m = 1; m < P; ++m) acc = fma2(own[m], own[m], acc);
-              const float ssq = group_sum<G>(acc.x + acc.y);
-              const float2 inv2 = splat2(rsqrtf(fmaf(ssq, a.inv_hd, a.eps)));
 #pragma unroll
               for (int m = 0; m < P; ++m) {
-                const float2 u = mul2(fma2(own[m], ca[m], mul2(par[m], sb[m])), inv2);
+                const float2 u = fma2(own[m], ca[m], mul2(par[m], sb[m]));
                 o[2 * m] = u.x;
                 o[2 * m + 1] = u.y;
               }
             } else {
               float2 ev[Q], od[Q];
               IO::unpack_eo(xv, ev, od);
-              float2 acc = mul2(ev[0], ev[0]);
+              acc = mul2(ev[0], ev[0]);
               acc = fma2(od[0], od[0], acc);
 #pragma unroll
               for (int m = 1; m < Q; ++m) {
                 acc = fma2(ev[m], ev[m], acc);
                 acc = fma2(od[m], od[m], acc);
               }
-              const float ssq = group_sum<G>(acc.x + acc.y);
-              const float2 inv2 = splat2(rsqrtf(fmaf(ssq, a.inv_hd, a.eps)));
 #pragma unroll
               for (int m = 0; m < Q; ++m) {
-                const float2 u0 = mul2(fma2(od[m], ns1[m], mul2(ev[m], c0[m])), inv2);
-                const float2 u1 = mul2(fma2(od[m], c1[m], mul2(ev[m], s0[m])), inv2);
+                const float2 u0 = fma2(od[m], ns1[m], mul2(ev[m], c0[m]));
+                const float2 u1 = fma2(od[m], c1[m], mul2(ev[m], s0[m]));
                 o[4 * m + 0] = u0.x;
                 o[4 * m + 1] = u1.x;
                 o[4 * m + 2] = u0.y;
@@ -259,23 +249,50 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
             const int head = v / G;
             unsigned char *dst = obase + static_cast<int64_t>(head) * a.out_sh + (v % G) * VB;
             if constexpr (OUT8) {
-              float amax = 0.f;
+              // 1/rms is one positive factor per head, so it cancels from the
+              // codes: code = round(u * 127 / max|u|) on the un-normalised
+              // rotation u, and only the scale max|u| / rms / 127 needs it.
+              // The sum of squares and the max then reduce side by side.
+              float ssq = acc.x + acc.y;
+              float m4[E / 2];
 #pragma unroll
-              for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(o[e]));
-              amax = group_max<G>(amax);
-              const float is = amax > 0.f ? 127.f / amax : 0.f;
+              for (int e = 0; e < E / 2; ++e) m4[e] = fmaxf(fabsf(o[2 * e]), fabsf(o[2 * e + 1]));
+              float umax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+#pragma unroll
+              for (int off = G / 2; off > 0; off >>= 1) {
+                ssq += __shfl_xor_sync(0xffffffffu, ssq, off);
+                umax = fmaxf(umax, __shfl_xor_sync(0xffffffffu, umax, off));
+              }
+              const float inv = rsqrtf(fmaf(ssq, a.inv_hd, a.eps));
+              // |u * is| <= 127 up to the fast division's 2 ulp, which the
+              // round-to-nearest keeps at 127
+              float is = umax > 0.f ? __fdividef(127.f, umax) : 0.f;
+              if (umax > 0.f && umax < 0x1p-96f) {
+                // a head of (near-)denormal inputs: 127 / umax would overflow,
+                // so scale u and umax by 2^64 (exact) first; the codes are
+                // unchanged
+#pragma unroll
+                for (int e = 0; e < E; ++e) o[e] *= 0x1p64f;
+                is = __fdividef(127.f, umax * 0x1p64f);
+              }
               uint32_t c[E];
+              const float2 is2 = splat2(is), magic2 = splat2(kRoundMagic);
 #pragma unroll
-              for (int e = 0; e < E; ++e) c[e] = code_bits(o[e], is);
+              for (int m = 0; m < P; ++m) {
+                const float2 r = fma2(make_float2(o[2 * m], o[2 * m + 1]), is2, magic2);
+                c[2 * m] = __float_as_uint(r.x);
+                c[2 * m + 1] = __float_as_uint(r.y);
+              }
               if (ok[k]) {
                 st_stream8(dst, pack_low_bytes(c[0], c[1], c[2], c[3]),
                            pack_low_bytes(c[4], c[5], c[6], c[7]));
-                if (gl == 0) scale_row[head] = amax / 127.f;
+                if (gl == 0) scale_row[head] = umax * inv * (1.f / 127.f);
               }
             } else {
+              const float2 inv2 = splat2(rsqrtf(fmaf(group_sum<G>(acc.x + acc.y), a.inv_hd, a.eps)));
               float2 pr[P];
 #pragma unroll
-              for (int m = 0; m < P; ++m) pr[m] = make_float2(o[2 * m], o[2 * m + 1]);
+              for (int m = 0; m < P; ++m) pr[m] = mul2(make_float2(o[2 * m], o[2 * m + 1]), inv2);
               if (ok[k]) st_stream16(dst, IO::pack(pr));
             }
           }
@@ -292,7 +309,11 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
 
 template <int G, int NT, int VPT, bool HALF, bool OUT8>
 cudaError_t launch_ex(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
-  constexpr int R = VPT <= 6 ? 2 : 1;
+  // INT8: one row per stage halves the ring, so a third CTA (24 warps per
+  // SM) fits beside the register limit: 0.90 against 1.04 ms at the 5 s
+  // clip.  The bf16 variants keep two rows per stage (one barrier per two
+  // rows), which measured as fast or faster for them.
+  constexpr int R = OUT8 ? 1 : (VPT <= 6 ? 2 : 1);
   constexpr int S = 2;
   const void *fn =
       reinterpret_cast<const void *>(&qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8>);

@@ -2,7 +2,7 @@
 for profilers (ncu) that should capture a small, self-contained case.
 
     python -m video_diffusion_transformer_rms_b200.profile_case \
-        [--workload clip5s] [--frames 4] [--launches 1] [--kernel norm|gemm]
+        [--workload clip5s] [--frames 4] [--launches 1] [--kernel norm|gemm|qk_bhsd|qk_half|qk_int8]
 
 The slice keeps the clip's H x W latent grid, D and head layout, takes the
 first `--frames` latent frames (T) and scales the audio rows by the same
@@ -10,7 +10,9 @@ fraction.  Inputs are larger than L2 at the default 4 frames (16,384 rows:
 168 MB per activation, 503 MB of merged QKV), so DRAM counters stay
 meaningful while the device footprint stays near 1.5 GB.  `--kernel gemm`
 runs the MLP up-projection with fused GELU on the same slice instead
-(A [rows, D], W1 [4D, D], C [rows, 4D]: about 1 GB at 4 frames).
+(A [rows, D], W1 [4D, D], C [rows, 4D]: about 1 GB at 4 frames), and
+`--kernel qk_*` one QKNorm+RoPE epilogue variant ([B, H, L, hd] output,
+half-split pairs, INT8 output).
 """
 import argparse
 import dataclasses
@@ -26,7 +28,8 @@ def main():
     ap.add_argument("--workload", default="clip5s", choices=sorted(WORKLOADS))
     ap.add_argument("--frames", type=int, default=4)
     ap.add_argument("--launches", type=int, default=1)
-    ap.add_argument("--kernel", default="norm", choices=["norm", "gemm"])
+    ap.add_argument("--kernel", default="norm",
+                    choices=["norm", "gemm", "qk_bhsd", "qk_half", "qk_int8"])
     args = ap.parse_args()
     full = WORKLOADS[args.workload]
     T = max(1, min(full.T, args.frames))
@@ -43,6 +46,15 @@ def main():
     y = torch.empty_like(x)
     out = torch.empty_like(h)
     qk = torch.empty((w.B, w.L, 2 * D), dtype=qkv.dtype, device=qkv.device)
+    if args.kernel.startswith("qk_"):
+        opts = {"qk_bhsd": {"layout": "bhsd"}, "qk_half": {"half_split": True},
+                "qk_int8": {"int8": True}}[args.kernel]
+        for _ in range(args.launches):
+            api.qknorm_rope3d_ex(qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim,
+                                 w.sections, t["gamma_q"], t["gamma_k"], w.eps, w.theta, **opts)
+        torch.cuda.synchronize()
+        print(f"{w.name}: {w.rows} rows, D={D}, {args.launches} launch(es) of {args.kernel}")
+        return
     for _ in range(args.launches):
         api.rms_adaln(x, t["scale"], t["shift"], w.n_video, eps=w.eps, out=y)
         api.qknorm_rope3d(qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections,
