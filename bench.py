@@ -417,7 +417,8 @@ def run_ours(args):
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                     "steps": e2e["steps"],
                     "path": "pinned host inputs -> H2D -> api.rms_adaln / api.qknorm_rope3d / "
-                            "api.gate_residual -> D2H of y, q, k, out; CUDA events"},
+                            "api.gate_residual -> D2H of y, q, k, out; copy-in, kernels and "
+                            "copy-out on three streams ordered by events; CUDA events"},
             "gpu_launches": len(KERNELS) * K,
             "clocks": clock_info,
         }
@@ -480,9 +481,20 @@ def time_gemm_gelu(w, D, dev, stream):
 
 def run_e2e(args, w, t, stream, api):
     """Same step through the public tensor API, inputs copied every step
-    from pinned host memory and every output copied back."""
+    from pinned host memory and every output copied back.
+
+    Three streams: host-to-device copies, the kernels, device-to-host
+    copies.  Each kernel waits for its own inputs and each output copy for
+    its kernel, so the two PCIe directions and the kernels overlap; the
+    next step's copy into a buffer waits for the kernel that read it, and a
+    kernel's write waits for the copy-out of its previous result."""
     D = w.D
-    names = ("x", "scale", "shift", "qkv", "gamma_q", "gamma_k", "h", "branch", "gate")
+    groups = {  # inputs of each kernel, in launch order
+        "rms_adaln": ("scale", "shift", "x"),
+        "qknorm_rope3d": ("gamma_q", "gamma_k", "qkv"),
+        "gate_residual": ("gate", "h", "branch"),
+    }
+    names = [n for g in groups.values() for n in g]
     host = {n: torch.empty(t[n].shape, dtype=t[n].dtype, pin_memory=True) for n in names}
     for n in names:
         host[n].copy_(t[n])
@@ -490,25 +502,51 @@ def run_e2e(args, w, t, stream, api):
     y = torch.empty((w.B, w.L, D), dtype=t["x"].dtype, device=t["x"].device)
     qk = torch.empty((w.B, w.L, 2 * D), dtype=t["x"].dtype, device=t["x"].device)
     out = torch.empty_like(y)
-    host_out = {"y": torch.empty(y.shape, dtype=y.dtype, pin_memory=True),
-                "qk": torch.empty(qk.shape, dtype=qk.dtype, pin_memory=True),
-                "out": torch.empty(out.shape, dtype=out.dtype, pin_memory=True)}
+    results = {"rms_adaln": y, "qknorm_rope3d": qk, "gate_residual": out}
+    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+                for k, v in results.items()}
     h2d = sum(host[n].numel() * host[n].element_size() for n in names)
     d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    read_done = {k: None for k in groups}   # kernel k finished reading its inputs
+    copied_out = {k: None for k in groups}  # result of kernel k is on the host
+
+    def kernel(k):
+        if k == "rms_adaln":
+            api.rms_adaln(dev["x"].view(w.B, w.L, D), dev["scale"], dev["shift"], w.n_video,
+                          eps=w.eps, out=y, stream=stream)
+        elif k == "qknorm_rope3d":
+            api.qknorm_rope3d(dev["qkv"].view(w.B, w.L, 3 * D), w.T, w.H, w.W, w.n_audio,
+                              w.n_heads, w.head_dim, w.sections, dev["gamma_q"],
+                              dev["gamma_k"], w.eps, w.theta, q_out=qk[..., :D],
+                              k_out=qk[..., D:], stream=stream)
+        else:
+            api.gate_residual(dev["h"].view(w.B, w.L, D), dev["branch"].view(w.B, w.L, D),
+                              dev["gate"], w.n_video, out=out, stream=stream)
 
     def step():
-        for n in names:
-            dev[n].copy_(host[n], non_blocking=True)
-        api.rms_adaln(dev["x"].view(w.B, w.L, D), dev["scale"], dev["shift"], w.n_video,
-                      eps=w.eps, out=y)
-        api.qknorm_rope3d(dev["qkv"].view(w.B, w.L, 3 * D), w.T, w.H, w.W, w.n_audio,
-                          w.n_heads, w.head_dim, w.sections, dev["gamma_q"], dev["gamma_k"],
-                          w.eps, w.theta, q_out=qk[..., :D], k_out=qk[..., D:])
-        api.gate_residual(dev["h"].view(w.B, w.L, D), dev["branch"].view(w.B, w.L, D),
-                          dev["gate"], w.n_video, out=out)
-        host_out["y"].copy_(y, non_blocking=True)
-        host_out["qk"].copy_(qk, non_blocking=True)
-        host_out["out"].copy_(out, non_blocking=True)
+        for k, g in groups.items():
+            if read_done[k] is not None:
+                s_in.wait_event(read_done[k])
+            with torch.cuda.stream(s_in):
+                for n in g:
+                    dev[n].copy_(host[n], non_blocking=True)
+            arrived = ev()
+            arrived.record(s_in)
+            stream.wait_event(arrived)
+            if copied_out[k] is not None:
+                stream.wait_event(copied_out[k])
+            kernel(k)
+            done = ev()
+            done.record(stream)
+            read_done[k] = done
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                host_out[k].copy_(results[k], non_blocking=True)
+            c = ev()
+            c.record(s_out)
+            copied_out[k] = c
 
     step()
     torch.cuda.synchronize()
@@ -517,9 +555,11 @@ def run_e2e(args, w, t, stream, api):
     b = torch.cuda.Event(enable_timing=True)
     dist.barrier()
     torch.cuda.synchronize()
-    a.record(stream)
+    a.record(s_in)
     for _ in range(n):
         step()
+    for c in copied_out.values():
+        stream.wait_event(c)
     b.record(stream)
     torch.cuda.synchronize()
     dist.barrier()
