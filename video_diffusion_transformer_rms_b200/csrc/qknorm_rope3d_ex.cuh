@@ -333,7 +333,11 @@ cudaError_t dispatch_ex(const QkArgs &a, int threads, int vpt, cudaStream_t stre
                         Geometry *geo) {
 #define SOL_CASE(NT, V) \
   if (threads == NT && vpt == V) return launch_ex<G, NT, V, HALF, OUT8>(a, stream, geo);
-  SOL_QK_SPLITS(SOL_CASE)
+  if constexpr (OUT8 && !HALF) {
+    SOL_SPLITS(SOL_CASE)
+  } else {
+    SOL_QK_SPLITS(SOL_CASE)
+  }
 #undef SOL_CASE
   return cudaErrorInvalidValue;
 }
