@@ -42,7 +42,7 @@ def _load():
         lib.oracle_residual_change.restype = i
         lib.oracle_qknorm_rope3d_ex.argtypes = [p, i64, p, p, p, i64, i64, i64, i64,
                                                 i64, i64, i64, i64, i64, i64, d, d,
-                                                i, i, p, p]
+                                                i, i, i, p, p]
         lib.oracle_qknorm_rope3d_ex.restype = i
         lib.oracle_quantize_heads.argtypes = [p, i64, i64, i64, p, p]
         lib.oracle_quantize_heads.restype = i
@@ -177,9 +177,11 @@ def qknorm_rope3d(qkv, T, H, W, n_audio, n_heads, head_dim, sections, eps, theta
 
 
 def qknorm_rope3d_ex(qkv, T, H, W, n_audio, n_heads, head_dim, sections, eps, theta,
-                     half_split, gamma_q=None, gamma_k=None, row_ids=None):
+                     half_split, gamma_q=None, gamma_k=None, row_ids=None, per_axis=False):
     """qknorm_rope3d with a rotary pair layout flag (half_split: pair i is
-    elements (i, i + head_dim/2))."""
+    elements (i, i + head_dim/2)) and a frequency ladder flag (per_axis: pair
+    j of a section of s pairs turns at theta^(-j/s), each axis with a ladder
+    of its own)."""
     qkv, gamma_q, gamma_k = _c(qkv), _c(gamma_q), _c(gamma_k)
     D = n_heads * head_dim
     q2 = qkv.reshape(-1, qkv.shape[-1])
@@ -192,7 +194,8 @@ def qknorm_rope3d_ex(qkv, T, H, W, n_audio, n_heads, head_dim, sections, eps, th
     rc = _load().oracle_qknorm_rope3d_ex(_ptr(q2), q2.shape[1], _ptr(gamma_q), _ptr(gamma_k),
                                          _ptr(rid), n, T, H, W, n_audio, n_heads, head_dim, st,
                                          sh, sw, eps, theta, int(bool(half_split)),
-                                         _dtype_code(qkv, gamma_q, gamma_k), _ptr(q), _ptr(k))
+                                         int(bool(per_axis)), _dtype_code(qkv, gamma_q, gamma_k),
+                                         _ptr(q), _ptr(k))
     if rc != 0:
         raise ValueError("oracle_qknorm_rope3d_ex rejected its arguments")
     return q, k

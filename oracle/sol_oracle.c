@@ -323,23 +323,55 @@ int oracle_qknorm_rope3d(const void *qkv, int64_t ld_qkv, const void *gamma_q,
 }
 
 /*
- * QKNorm + 3D RoPE with a choice of rotary pair layout.  half_split = 0 is
- * oracle_qknorm_rope3d (pair i = elements (2i, 2i+1)); half_split = 1 pairs
- * element i with element i + head_dim/2 (the "rotate half" layout of GPT-NeoX
- * style implementations):
+ * Frequency of rotary pair i.
+ *   per_axis = 0: one ladder over all head_dim/2 pairs, theta^(-2i/head_dim),
+ *                 the sections only choose the position (M-RoPE style);
+ *   per_axis = 1: each section its own ladder over its own 2*s rotary
+ *                 dimensions: pair j of a section of s pairs (j counted from
+ *                 the section's first pair) has theta^(-2j/(2s)) = theta^(-j/s),
+ *                 as when t, h and w each get a RoPE of their own and the
+ *                 three are concatenated (an empty section holds no pair, so
+ *                 its size is never divided by).
+ */
+static double rope_freq(int64_t i, int64_t head_dim, int64_t sec_t, int64_t sec_h,
+                        double theta, int per_axis)
+{
+    if (!per_axis)
+        return pow(theta, -2.0 * (double)i / (double)head_dim);
+    int64_t start, size;
+    if (i < sec_t) {
+        start = 0;
+        size = sec_t;
+    } else if (i < sec_t + sec_h) {
+        start = sec_t;
+        size = sec_h;
+    } else {
+        start = sec_t + sec_h;
+        size = head_dim / 2 - sec_t - sec_h;
+    }
+    return pow(theta, -(double)(i - start) / (double)size);
+}
+
+/*
+ * QKNorm + 3D RoPE with a choice of rotary pair layout and of frequency
+ * ladder.  half_split = 0 pairs elements (2i, 2i+1) as oracle_qknorm_rope3d
+ * does; half_split = 1 pairs element i with element i + head_dim/2 (the
+ * "rotate half" layout of GPT-NeoX style implementations):
  *   out[i]              = n[i] cos(phi_i) - n[i + hd/2] sin(phi_i)
  *   out[i + hd/2]       = n[i] sin(phi_i) + n[i + hd/2] cos(phi_i)
- * with the same phi_i, sections and positions.  Arguments as for
- * oracle_qknorm_rope3d.
+ * with phi_i = pos[axis(i)] * rope_freq(i) (per_axis as for rope_freq) and the
+ * same sections and positions.  With half_split = 0 and per_axis = 0 this is
+ * oracle_qknorm_rope3d itself.  Other arguments as for oracle_qknorm_rope3d.
  */
 int oracle_qknorm_rope3d_ex(const void *qkv, int64_t ld_qkv, const void *gamma_q,
                             const void *gamma_k, const int64_t *row_ids, int64_t n_rows,
                             int64_t T, int64_t H, int64_t W, int64_t n_audio,
                             int64_t n_heads, int64_t head_dim, int64_t sec_t,
                             int64_t sec_h, int64_t sec_w, double eps, double theta,
-                            int half_split, int dtype, double *q_out, double *k_out)
+                            int half_split, int per_axis, int dtype, double *q_out,
+                            double *k_out)
 {
-    if (!half_split)
+    if (!half_split && !per_axis)
         return oracle_qknorm_rope3d(qkv, ld_qkv, gamma_q, gamma_k, row_ids, n_rows, T, H,
                                     W, n_audio, n_heads, head_dim, sec_t, sec_h, sec_w, eps,
                                     theta, dtype, q_out, k_out);
@@ -367,18 +399,21 @@ int oracle_qknorm_rope3d_ex(const void *qkv, int64_t ld_qkv, const void *gamma_q
                 }
                 double denom = sqrt(ss / (double)head_dim + eps);
                 for (int64_t i = 0; i < half; ++i) {
-                    double a = in_val(qkv, src + i, dtype) / denom;
-                    double b = in_val(qkv, src + i + half, dtype) / denom;
+                    /* the two elements of pair i */
+                    int64_t ia = half_split ? i : 2 * i;
+                    int64_t ib = half_split ? i + half : 2 * i + 1;
+                    double a = in_val(qkv, src + ia, dtype) / denom;
+                    double b = in_val(qkv, src + ib, dtype) / denom;
                     if (gam) {
-                        a = a * in_val(gam, i, dtype);
-                        b = b * in_val(gam, i + half, dtype);
+                        a = a * in_val(gam, ia, dtype);
+                        b = b * in_val(gam, ib, dtype);
                     }
                     int axis = i < sec_t ? 0 : (i < sec_t + sec_h ? 1 : 2);
                     double phi = (double)pos[axis] *
-                                 pow(theta, -2.0 * (double)i / (double)head_dim);
+                                 rope_freq(i, head_dim, sec_t, sec_h, theta, per_axis);
                     double c = cos(phi), s = sin(phi);
-                    out[dst + i] = a * c - b * s;
-                    out[dst + i + half] = a * s + b * c;
+                    out[dst + ia] = a * c - b * s;
+                    out[dst + ib] = a * s + b * c;
                 }
             }
         }

@@ -238,6 +238,61 @@ def test_rope_angles_match_hand_table():
                                            atol=1e-13)
 
 
+@pytest.mark.parametrize("half", [False, True])
+def test_rope_per_axis_angles_match_hand_table(half):
+    # per-axis ladder: every pair of q holds (1, 0) and of k holds (0, 1) in
+    # the chosen pair layout; with eps = 0 the rotated q pair is
+    # sqrt2 (cos phi, sin phi), phi = position on the pair's axis times the
+    # hand-written per-axis frequency
+    pos, _ = _positions()
+    g = read_golden("rope3d_per_axis_freqs.txt")
+    pairs = {int(r[0]): ("thw".index(r[1]), float(r[3])) for r in g["pair"]}
+    rows = _grid_rows(**TINY)
+    hd = TINY["head_dim"]
+    if half:
+        qh = np.concatenate([np.ones(hd // 2), np.zeros(hd // 2)])
+        kh = np.concatenate([np.zeros(hd // 2), np.ones(hd // 2)])
+    else:
+        qh, kh = np.tile([1.0, 0.0], hd // 2), np.tile([0.0, 1.0], hd // 2)
+    qkv = _qkv_same_every_row(qh, kh, rows, TINY["n_heads"])
+    q, k = oracle.qknorm_rope3d_ex(qkv, TINY["T"], TINY["H"], TINY["W"], TINY["n_audio"],
+                                   TINY["n_heads"], hd, TINY["sections"], 0.0, TINY["theta"],
+                                   half, per_axis=True)
+    s2 = math.sqrt(2.0)
+    for r, p in pos.items():
+        for i, (axis, freq) in pairs.items():
+            phi = p[axis] * freq
+            ia, ib = (i, i + hd // 2) if half else (2 * i, 2 * i + 1)
+            for head in range(TINY["n_heads"]):
+                a, b = q[r, head * hd + ia], q[r, head * hd + ib]
+                assert abs(math.hypot(a, b) - s2) < 1e-13
+                assert abs(_wrap(math.atan2(b, a) - phi)) < 1e-12, (r, i, head)
+                c, d = k[r, head * hd + ia], k[r, head * hd + ib]
+                np.testing.assert_allclose([c, d], [-s2 * math.sin(phi), s2 * math.cos(phi)],
+                                           atol=1e-13)
+
+
+def test_rope_per_axis_with_one_section_is_the_global_ladder():
+    # a single section of all 64 pairs: its own ladder theta^(-j/64) is the
+    # global theta^(-2i/128), so the per-axis flag changes nothing
+    rows = _grid_rows(**TINY)
+    qkv = f32(RNG.standard_normal((rows, 3 * 2 * 128)))
+    for secs in ((64, 0, 0), (0, 64, 0), (0, 0, 64)):
+        args = (qkv, TINY["T"], TINY["H"], TINY["W"], TINY["n_audio"], 2, 128, secs, 1e-6,
+                1e4)
+        for half in (False, True):
+            q0, k0 = oracle.qknorm_rope3d_ex(*args, half, per_axis=False)
+            q1, k1 = oracle.qknorm_rope3d_ex(*args, half, per_axis=True)
+            np.testing.assert_allclose(q1, q0, rtol=0, atol=1e-15)
+            np.testing.assert_allclose(k1, k0, rtol=0, atol=1e-15)
+    # and with three sections it differs (pair 16 is the h section's first)
+    args = (qkv, TINY["T"], TINY["H"], TINY["W"], TINY["n_audio"], 2, 128, (16, 24, 24), 1e-6,
+            1e4)
+    q0, _ = oracle.qknorm_rope3d_ex(*args, False, per_axis=False)
+    q1, _ = oracle.qknorm_rope3d_ex(*args, False, per_axis=True)
+    assert np.abs(q1 - q0).max() > 0.1
+
+
 def test_qknorm_identity_at_origin_gives_gamma():
     # a constant head at position (0,0,0) normalises to all ones (eps = 0) and
     # the rotation is the identity, so the output is gamma itself.
