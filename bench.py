@@ -324,6 +324,11 @@ def run_ours(args):
     lay_half = _abi.QkLayout(w.L * D, D, hd, 1, 0, None, None)
     lay_int8 = _abi.QkLayout(w.L * D, D, hd, 0, 1, s8.data_ptr(),
                              s8.data_ptr() + w.rows * w.n_heads * 4)
+    v8 = torch.empty(w.rows * D, dtype=torch.int8, device=dev)
+    vs8 = torch.empty(w.rows * w.n_heads, dtype=torch.float32, device=dev)
+    lay_int8_v = _abi.QkLayout(w.L * D, D, hd, 0, 1, s8.data_ptr(),
+                               s8.data_ptr() + w.rows * w.n_heads * 4, 0, 0, v8.data_ptr(),
+                               vs8.data_ptr())
 
     def k_qk_ex(lay, q_ptr, k_ptr):
         return lambda: _abi.sol_qknorm_rope3d_ex(
@@ -353,6 +358,11 @@ def run_ours(args):
         # INT8 codes (2D bytes) + fp32 scales per (row, head) for q and k
         "qknorm_rope3d_ex_int8": (2 * row + 2 * D + 2 * w.n_heads * 4,
                                   k_qk_ex(lay_int8, q8.data_ptr(), q8.data_ptr() + w.rows * D)),
+        # the same, plus v quantised as it stands (a second launch): q, k, v read,
+        # three sets of codes and scales written
+        "qknorm_rope3d_ex_int8_qkv": (3 * row + 3 * D + 3 * w.n_heads * 4,
+                                      k_qk_ex(lay_int8_v, q8.data_ptr(),
+                                              q8.data_ptr() + w.rows * D)),
     }
     next_rows = {}
     for name, (bytes_per_row, fn) in extra.items():
@@ -372,7 +382,7 @@ def run_ours(args):
         next_rows[name] = {"ms": round(ms, 4), "tokens_per_s": round(w.rows / (ms / 1e3)),
                            "bytes_per_token": bytes_per_row,
                            "GB_per_s": round(nbytes / (ms / 1e3) / 1e9, 1)}
-    del ws, q8, s8
+    del ws, q8, s8, v8, vs8
     next_rows["gemm_gelu"] = time_gemm_gelu(w, D, dev, stream)
 
     # ---- end to end through the public API, host buffers ------------------

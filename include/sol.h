@@ -205,6 +205,18 @@ typedef struct sol_qk_layout {
                            k_scale [B, L, H] fp32 receive max|x| / 127 per head */
     float *q_scale;     /* int8_out only: device, 4-byte aligned */
     float *k_scale;
+    int32_t per_axis_freq; /* 0: one frequency ladder over all head_dim/2
+                              pairs, theta^(-2i/head_dim), the sections only
+                              choosing the position; 1: each section a ladder
+                              of its own, local pair j of a section of s pairs
+                              at theta^(-j/s) (t, h and w each a RoPE over
+                              their own 2s dimensions) */
+    int32_t reserved;   /* must be 0 */
+    void *v_out;        /* int8_out only, may be NULL: if set, v (columns
+                           [2D, 3D) of qkv) is quantised as it stands (no
+                           norm, no rotation) to int8 codes here, in the
+                           layout of q_out/k_out, with scales in v_scale */
+    float *v_scale;     /* [B, L, H] fp32, with v_out */
 } sol_qk_layout;
 
 /*
@@ -223,7 +235,17 @@ typedef struct sol_qk_layout {
  *               each other or the scales (no in-place form).  Each output
  *               vector start (16 bytes, 8 for int8) must be aligned to its
  *               size: base and strides * element size multiples of it.
+ *               v_out / v_scale follow the int8 rules of q_out / q_scale and
+ *               must overlap none of the other buffers; with v_out set,
+ *               ld_qkv must be >= 3*D.  The quantisation of v is a second
+ *               kernel on the same stream (v is not read by the first).
  *   other arguments as for sol_qknorm_rope3d.
+ *
+ * The per-axis frequency ladder and the quantised v are options of this
+ * library (the pages name per-axis frequencies and INT8 Q/K/V transfer, not
+ * their exact form).  A layout with reserved != 0 or per_axis_freq outside
+ * {0, 1} returns SOL_ERR_INVALID_ARG; v_out without int8_out returns
+ * SOL_ERR_UNSUPPORTED.
  */
 sol_status sol_qknorm_rope3d_ex(const void *qkv, int64_t ld_qkv, void *q_out,
                                 void *k_out, const sol_qk_layout *layout,

@@ -226,11 +226,16 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     assert isinstance(ctypes.CDLL, type)
 
 
+# well-placed fp32 scale arrays for the INT8 cases (none overlaps another buffer)
+Q8S, K8S, V8S = A + (3 << 30), A + (4 << 30), A + (6 << 30)
+
+
 def qkex(qkv=A, ldq=3 * 1024, qo=A + (1 << 30), ko=A + (2 << 30), sb=None, sr=1024, sh=128,
          half=0, int8=0, qs=None, ks=None, B=1, T=2, H=4, W=6, na=8, nh=8, hd=128,
-         secs=(16, 24, 24), dt=BF):
+         secs=(16, 24, 24), dt=BF, per_axis=0, reserved=0, vo=None, vs=None):
     L = T * H * W + na
-    lay = _abi.QkLayout(L * nh * hd if sb is None else sb, sr, sh, half, int8, qs, ks)
+    lay = _abi.QkLayout(L * nh * hd if sb is None else sb, sr, sh, half, int8, qs, ks, per_axis,
+                        reserved, vo, vs)
     return _abi.sol_qknorm_rope3d_ex(qkv, ldq, qo, ko, lay, None, None, B, T, H, W, na, nh, hd,
                                      *secs, 1e-6, 1e4, dt, None)
 
@@ -246,6 +251,20 @@ def qkex(qkv=A, ldq=3 * 1024, qo=A + (1 << 30), ko=A + (2 << 30), sb=None, sr=10
     (dict(qo=A + 4096), _abi.SOL_ERR_INVALID_ARG),              # q_out inside qkv
     (dict(ko=A + (1 << 30) + 1024), _abi.SOL_ERR_INVALID_ARG),  # k_out overlaps q_out
     (dict(int8=1, qs=A + (1 << 30), ks=A + (4 << 30)), _abi.SOL_ERR_INVALID_ARG),  # scale on q
+    (dict(reserved=1), _abi.SOL_ERR_INVALID_ARG),
+    (dict(per_axis=2), _abi.SOL_ERR_INVALID_ARG),
+    (dict(vo=A + (5 << 30)), _abi.SOL_ERR_UNSUPPORTED),          # v_out needs int8
+    (dict(int8=1, qs=Q8S, ks=K8S, vo=A + (5 << 30)), _abi.SOL_ERR_INVALID_ARG),  # no v_scale
+    (dict(int8=1, qs=Q8S, ks=K8S, vo=A + (5 << 30), vs=V8S, ldq=2 * 1024),
+     _abi.SOL_ERR_INVALID_ARG),                                  # v not in the rows
+    (dict(int8=1, qs=Q8S, ks=K8S, vo=A + (5 << 30) + 4, vs=V8S), _abi.SOL_ERR_MISALIGNED),
+    (dict(int8=1, qs=Q8S, ks=K8S, vo=A + (5 << 30), vs=V8S + 2), _abi.SOL_ERR_MISALIGNED),
+    (dict(int8=1, qs=Q8S, ks=K8S, vo=A + 4096, vs=V8S),
+     _abi.SOL_ERR_INVALID_ARG),                                  # v_out on qkv's v columns
+    (dict(int8=1, qs=Q8S, ks=K8S, vo=A + (2 << 30) + 64, vs=V8S),
+     _abi.SOL_ERR_INVALID_ARG),                                  # v_out overlaps k_out
+    (dict(int8=1, qs=Q8S, ks=K8S, vo=A + (5 << 30), vs=Q8S + 64),
+     _abi.SOL_ERR_INVALID_ARG),                                  # v_scale overlaps q_scale
 ])
 def test_qknorm_rope3d_ex_rejects(kw, status):
     assert qkex(**kw) == status

@@ -556,6 +556,67 @@ def test_qknorm_rope3d_ex_workload(name, half, layout, int8):
         assert_close(k, wk, tag + " k")
 
 
+@pytest.mark.parametrize("name", ("medium", "clip5s"))
+@pytest.mark.parametrize("half", [False, True])
+@pytest.mark.parametrize("int8", [False, True])
+def test_qknorm_rope3d_ex_per_axis_freq(name, half, int8):
+    # each rotary section with a frequency ladder of its own, theta^(-j/s)
+    w = WORKLOADS[name]
+    t = make_inputs(w, DEV, which=("qknorm_rope3d",))
+    qkv = t["qkv"].view(w.B, w.L, 3 * w.D)
+    res = api.qknorm_rope3d_ex(qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim,
+                               w.sections, t["gamma_q"], t["gamma_k"], w.eps, w.theta,
+                               layout="bhsd", half_split=half, int8=int8, per_axis_freq=True)
+    torch.cuda.synchronize()
+    q, k = (_bshd(r, "bhsd").reshape(w.rows, w.D) for r in res[:2])
+    ids = None if name == "medium" else _ids(w, 384)
+    qkv2 = qkv.view(-1, 3 * w.D)
+    src = _o(qkv2) if ids is None else take_rows(qkv2[:, :2 * w.D], ids)
+    wq, wk = oracle.qknorm_rope3d_ex(src, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim,
+                                     w.sections, w.eps, w.theta, half, _o(t["gamma_q"]),
+                                     _o(t["gamma_k"]), row_ids=ids, per_axis=True)
+    if ids is not None:
+        q, k = take_rows_gpu(q, ids), take_rows_gpu(k, ids)
+    tag = f"per-axis[{name} half={half} int8={int8}]"
+    if int8:
+        qs, ks = (r.reshape(w.rows, w.n_heads) for r in res[2:4])
+        if ids is not None:
+            qs, ks = take_rows_gpu(qs, ids), take_rows_gpu(ks, ids)
+        _check_int8(q, qs, wq, w.n_heads, w.head_dim, tag + " q")
+        _check_int8(k, ks, wk, w.n_heads, w.head_dim, tag + " k")
+    else:
+        assert_close(q, wq, tag + " q")
+        assert_close(k, wk, tag + " k")
+
+
+@pytest.mark.parametrize("name", ("medium", "clip5s"))
+@pytest.mark.parametrize("layout", ["bshd", "bhsd"])
+def test_qknorm_rope3d_ex_quantized_v(name, layout):
+    # v quantised as it stands, per (row, head), next to the INT8 q and k
+    w = WORKLOADS[name]
+    t = make_inputs(w, DEV, which=("qknorm_rope3d",))
+    qkv = t["qkv"].view(w.B, w.L, 3 * w.D)
+    q, k, qs, ks, v, vs = api.qknorm_rope3d_ex(
+        qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections, t["gamma_q"],
+        t["gamma_k"], w.eps, w.theta, layout=layout, int8=True, quantize_v=True)
+    torch.cuda.synchronize()
+    ids = None if name == "medium" else _ids(w, 384)
+    qkv2 = qkv.view(-1, 3 * w.D)
+    v_rows = qkv2[:, 2 * w.D:]
+    want_v = oracle.widen(_o(v_rows.contiguous()) if ids is None else take_rows(v_rows, ids))
+    v = _bshd(v, layout).reshape(w.rows, w.D)
+    vs = vs.reshape(w.rows, w.n_heads)
+    if ids is not None:
+        v, vs = take_rows_gpu(v, ids), take_rows_gpu(vs, ids)
+    _check_int8(v, vs, want_v, w.n_heads, w.head_dim, f"v[{name} {layout}]")
+    # q and k are those of the INT8 entry point without v
+    q2, k2, qs2, ks2 = api.qknorm_rope3d_ex(
+        qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections, t["gamma_q"],
+        t["gamma_k"], w.eps, w.theta, layout=layout, int8=True)
+    assert torch.equal(q, q2) and torch.equal(k, k2)
+    assert torch.equal(qs, qs2) and torch.equal(ks, ks2)
+
+
 def test_qknorm_rope3d_ex_interleaved_matches_default_entry_point():
     # same arithmetic as sol_qknorm_rope3d, only the addressing differs:
     # bit-identical results in both layouts
@@ -641,13 +702,13 @@ def test_gemm_gelu_clip_mlp_shape_sampled():
 def test_qknorm_rope3d_ex_int8_edge_heads(half):
     # per row: a normal head, an all-zero head, a head of tiny normal values
     # (x * 2^-110, so max|u| < 2^-96 and the kernel rescales before dividing),
-    # and a head with one 1e4 outlier; q and k get different heads
+    # and a head with one 1e4 outlier; q, k and v get different heads
     T, H, W, na, nh, hd = 2, 3, 4, 5, 4, 128
     L = T * H * W + na
     D = nh * hd
     base = activation(L, 3 * D, torch.float32, DEV, 71, outliers=False).view(L, 3, nh, hd)
     x = base.clone()
-    for part, (zero, tiny, spike) in enumerate([(1, 2, 3), (2, 3, 1)]):
+    for part, (zero, tiny, spike) in enumerate([(1, 2, 3), (2, 3, 1), (3, 1, 2)]):
         x[:, part, zero] = 0.0
         x[:, part, tiny] = torch.sign(base[:, part, tiny]) * (1 + base[:, part, tiny].abs()) * 2.0 ** -110
         x[:, part, spike, 17] = 1.0e4
@@ -655,11 +716,15 @@ def test_qknorm_rope3d_ex_int8_edge_heads(half):
     gq = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 72)
     gk = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 73)
     res = api.qknorm_rope3d_ex(qkv, T, H, W, na, nh, hd, (16, 24, 24), gq, gk, layout="bshd",
-                               half_split=half, int8=True)
+                               half_split=half, int8=True, quantize_v=True)
     torch.cuda.synchronize()
     wq, wk = oracle.qknorm_rope3d_ex(_o(qkv.view(L, 3 * D)), T, H, W, na, nh, hd, (16, 24, 24),
                                      1e-6, 1e4, half, _o(gq), _o(gk))
-    q, k, qs, ks = res
+    q, k, qs, ks, v, vs = res
+    want_v = oracle.widen(_o(qkv.view(L, 3 * D)[:, 2 * D:].contiguous()))
+    _check_int8(v.reshape(L, D), vs, want_v, nh, hd, f"edge half={half} v")
+    assert torch.all(vs.view(L, nh)[:, 3] == 0) and torch.all(v.view(L, nh, hd)[:, 3] == 0)
+    assert int(v.view(L, nh, hd)[:, 1].abs().amax()) == 127
     _check_int8(q.reshape(L, D), qs, wq, nh, hd, f"edge half={half} q")
     _check_int8(k.reshape(L, D), ks, wk, nh, hd, f"edge half={half} k")
     # the zero heads: scale 0 and every code 0

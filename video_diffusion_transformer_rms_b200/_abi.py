@@ -29,7 +29,9 @@ class QkLayout(ctypes.Structure):
     _fields_ = [("stride_b", ctypes.c_int64), ("stride_row", ctypes.c_int64),
                 ("stride_head", ctypes.c_int64), ("half_split", ctypes.c_int32),
                 ("int8_out", ctypes.c_int32), ("q_scale", ctypes.c_void_p),
-                ("k_scale", ctypes.c_void_p)]
+                ("k_scale", ctypes.c_void_p), ("per_axis_freq", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("v_out", ctypes.c_void_p),
+                ("v_scale", ctypes.c_void_p)]
 
 
 _lock = threading.Lock()

@@ -145,13 +145,18 @@ def qknorm_rope3d_ex(qkv: torch.Tensor, T: int, H: int, W: int, n_audio: int, n_
                      gamma_q: Optional[torch.Tensor] = None,
                      gamma_k: Optional[torch.Tensor] = None, eps: float = 1e-6,
                      theta: float = 10000.0, layout: str = "bshd", half_split: bool = False,
-                     int8: bool = False, stream: Optional[torch.cuda.Stream] = None):
+                     int8: bool = False, per_axis_freq: bool = False, quantize_v: bool = False,
+                     stream: Optional[torch.cuda.Stream] = None):
     """QKNorm + 3D RoPE epilogue variants (bf16 input).  layout "bshd" gives
-    q, k as [B, L, H, hd]; "bhsd" gives attention's [B, H, L, hd].  With
-    int8=True returns (q_codes, k_codes, q_scale, k_scale), codes int8 in the
-    chosen layout and scales fp32 [B, L, H]; else (q, k) in bf16."""
+    q, k as [B, L, H, hd]; "bhsd" as attention's [B, H, L, hd].  half_split
+    pairs element i with i + hd/2; per_axis_freq gives each rotary section a
+    frequency ladder of its own.  int8 returns (q, k, q_scale, k_scale): int8
+    codes in the chosen layout and scales fp32 [B, L, H]; with quantize_v
+    also (v, v_scale), v quantised as it stands; else (q, k) in bf16."""
     if qkv.dim() != 3 or qkv.stride(2) != 1 or qkv.stride(0) != qkv.shape[1] * qkv.stride(1):
         raise ValueError("qkv must be [B, L, C] with unit column stride and packed rows")
+    if quantize_v and not int8:
+        raise ValueError("quantize_v needs int8=True")
     B, L, _ = qkv.shape
     if L != T * H * W + n_audio:
         raise ValueError("L must equal T*H*W + n_audio")
@@ -166,17 +171,23 @@ def qknorm_rope3d_ex(qkv: torch.Tensor, T: int, H: int, W: int, n_audio: int, n_
         raise ValueError("layout must be 'bshd' or 'bhsd'")
     q = torch.empty(shape, dtype=odt, device=qkv.device)
     k = torch.empty(shape, dtype=odt, device=qkv.device)
-    qs = ks = None
+    qs = ks = v = vs = None
     if int8:
         qs = torch.empty((B, L, n_heads), dtype=torch.float32, device=qkv.device)
         ks = torch.empty((B, L, n_heads), dtype=torch.float32, device=qkv.device)
+    if quantize_v:
+        v = torch.empty(shape, dtype=odt, device=qkv.device)
+        vs = torch.empty((B, L, n_heads), dtype=torch.float32, device=qkv.device)
     lay = _abi.QkLayout(strides[0], strides[1], strides[2], int(bool(half_split)),
-                        int(bool(int8)), _ptr(qs), _ptr(ks))
+                        int(bool(int8)), _ptr(qs), _ptr(ks), int(bool(per_axis_freq)), 0,
+                        _ptr(v), _ptr(vs))
     st, sh, sw = sections
     _abi.check(_abi.sol_qknorm_rope3d_ex(
         _ptr(qkv), qkv.stride(1), _ptr(q), _ptr(k), lay, _ptr(gamma_q), _ptr(gamma_k), B, T, H,
         W, n_audio, n_heads, head_dim, st, sh, sw, eps, theta,
         _dtype(qkv, gamma_q, gamma_k), _stream(stream)))
+    if quantize_v:
+        return q, k, qs, ks, v, vs
     return (q, k, qs, ks) if int8 else (q, k)
 
 

@@ -22,7 +22,7 @@ LIB = os.path.join(PKG, "libsol.so")
 
 SOURCES = ["sol_abi.cu", "rms_adaln.cu", "gate_residual.cu", "qknorm_rope3d_bf16.cu",
            "qknorm_rope3d_f32.cu", "qknorm_rope3d_ex_bf16.cu", "qknorm_rope3d_ex_int8.cu",
-           "residual_change.cu", "gemm_gelu.cu"]
+           "residual_change.cu", "quantize_heads.cu", "gemm_gelu.cu"]
 # sources built against the CUTLASS / CuTe headers (the sm100 GEMM templates)
 CUTLASS_SOURCES = {"gemm_gelu.cu"}
 HEADERS = ["sol_device.cuh", "sol_launch.h", "qknorm_rope3d.cuh", "qknorm_rope3d_ex.cuh"]

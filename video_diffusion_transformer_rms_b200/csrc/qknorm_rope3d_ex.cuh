@@ -5,7 +5,9 @@
 //   - the half-split rotary pair layout, pair i = elements (i, i + hd/2);
 //   - INT8 output: symmetric per-(row, head) codes round(x * 127 / max|x|)
 //     with fp32 scales max|x| / 127, the quantised Q/K that the KOCPC Sol-H3
-//     article's 4x/8x B300 runs send between GPUs ("INT8 QKV ... transfer").
+//     article's 4x/8x B300 runs send between GPUs ("INT8 QKV ... transfer");
+//   - a per-axis frequency ladder: each of the t/h/w sections a RoPE of its
+//     own, pair j of a section of s pairs at theta^(-j/s).
 // Same structure as qknorm_rope3d.cuh (ring, cursors, per-row angle tables,
 // G lanes per head).  With the half-split layout a thread's partner elements
 // (i + hd/2, or i - hd/2) sit in lane gl ^ G/2 of the same head: one 16-byte
@@ -19,20 +21,6 @@
 
 namespace sol {
 namespace qk {
-
-// Round-half-even of x*s for |x*s| <= 127 by adding 1.5 * 2^23: the fp32
-// sum has an ulp of 1, so one FMA rounds the exact product to an integer and
-// leaves it, as a two's-complement byte, in the low byte of the bit pattern.
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
-// Low bytes of four words, in order, as one word.
-__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
-}
-
-__device__ __forceinline__ void st_stream8(void *gmem_dst, uint32_t lo, uint32_t hi) {
-  asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};\n" ::"l"(gmem_dst), "r"(lo), "r"(hi)
-               : "memory");
-}
 
 template <int G, int NT, int VPT, int R, int S, bool HALF, bool OUT8>
 __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
@@ -83,8 +71,19 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
       }
     }
   }
-  for (int p = tid; p < a.npairs; p += NT)
-    freq[p] = pow(static_cast<double>(a.theta), -2.0 * p / a.head_dim);
+  // frequency of each rotary pair: one ladder over all pairs, or with
+  // per_axis one per section (local pair j of a section of s pairs at
+  // theta^(-j/s))
+  for (int p = tid; p < a.npairs; p += NT) {
+    double e = -2.0 * p / a.head_dim;
+    if (a.per_axis) {
+      const int start = p < a.sec_t ? 0 : (p < a.sec_th ? a.sec_t : a.sec_th);
+      const int size = p < a.sec_t ? a.sec_t : (p < a.sec_th ? a.sec_th - a.sec_t
+                                                             : a.npairs - a.sec_th);
+      e = -static_cast<double>(p - start) / size;
+    }
+    freq[p] = pow(static_cast<double>(a.theta), e);
+  }
 
   int64_t begin;
   int count;

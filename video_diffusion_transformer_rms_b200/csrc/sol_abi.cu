@@ -370,8 +370,16 @@ sol_status sol_qknorm_rope3d_ex(const void *qkv, int64_t ld_qkv, void *q_out, vo
   if (ld_qkv < 2 * D) return fail(SOL_ERR_INVALID_ARG, "%s: need ld_qkv >= 2*D", fn);
   if (rows == 0) return ok();
   const bool int8 = layout->int8_out != 0;
-  if (!qkv || !q_out || !k_out || (int8 && (!layout->q_scale || !layout->k_scale)))
+  if (layout->reserved != 0 || (layout->per_axis_freq != 0 && layout->per_axis_freq != 1))
+    return fail(SOL_ERR_INVALID_ARG, "%s: layout.reserved must be 0, per_axis_freq 0 or 1", fn);
+  const bool quant_v = layout->v_out != nullptr;
+  if (quant_v && !int8)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: v_out needs int8_out (v is only quantised)", fn);
+  if (!qkv || !q_out || !k_out || (int8 && (!layout->q_scale || !layout->k_scale)) ||
+      (quant_v && !layout->v_scale))
     return fail(SOL_ERR_INVALID_ARG, "%s: qkv, q_out, k_out (and scales) must be non-null", fn);
+  if (quant_v && ld_qkv < 3 * D)
+    return fail(SOL_ERR_INVALID_ARG, "%s: quantising v needs ld_qkv >= 3*D", fn);
   if (2 * D * 2 > kMaxRowBytesQk)
     return fail(SOL_ERR_UNSUPPORTED, "%s: 2*D=%lld exceeds %lld elements", fn, (long long)(2 * D),
                 (long long)(kMaxRowBytesQk / 2));
@@ -383,28 +391,36 @@ sol_status sol_qknorm_rope3d_ex(const void *qkv, int64_t ld_qkv, void *q_out, vo
       (gamma_k && !aligned16(gamma_k)) || reinterpret_cast<uintptr_t>(q_out) % vb ||
       reinterpret_cast<uintptr_t>(k_out) % vb || sb % vb || sr % vb || sh % vb ||
       (int8 && ((reinterpret_cast<uintptr_t>(layout->q_scale) & 3u) ||
-                (reinterpret_cast<uintptr_t>(layout->k_scale) & 3u))))
+                (reinterpret_cast<uintptr_t>(layout->k_scale) & 3u))) ||
+      (quant_v && ((reinterpret_cast<uintptr_t>(layout->v_out) % vb) ||
+                   (reinterpret_cast<uintptr_t>(layout->v_scale) & 3u))))
     return fail(SOL_ERR_MISALIGNED, "%s: pointers and strides must be aligned", fn);
   // byte extent of one output: last element + 1
   const int64_t ext = (B - 1) * sb + (L - 1) * sr + (n_heads - 1) * sh + head_dim * oes;
   const Span qs = span_of(q_out, 1, 0, ext), ks = span_of(k_out, 1, 0, ext);
-  const Span in = span_of(qkv, rows, ld_qkv * 2, 2 * D * 2);
-  if (spans_overlap(qs, in) || spans_overlap(ks, in) || spans_overlap(qs, ks))
-    return fail(SOL_ERR_INVALID_ARG, "%s: q_out and k_out must overlap neither qkv nor each other",
-                fn);
+  // the columns read: q and k, and v too when it is quantised
+  const Span in = span_of(qkv, rows, ld_qkv * 2, (quant_v ? 3 : 2) * D * 2);
+  // v's codes: the layout of q_out; an empty span when v is not quantised
+  const Span vs = quant_v ? span_of(layout->v_out, 1, 0, ext) : Span{0, 0};
+  if (spans_overlap(qs, in) || spans_overlap(ks, in) || spans_overlap(qs, ks) ||
+      spans_overlap(vs, in) || spans_overlap(vs, qs) || spans_overlap(vs, ks))
+    return fail(SOL_ERR_INVALID_ARG,
+                "%s: q_out, k_out and v_out must overlap neither qkv nor each other", fn);
   if (int8) {
     const int64_t sc = rows * n_heads * 4;
     const Span a1 = span_of(layout->q_scale, 1, 0, sc), a2 = span_of(layout->k_scale, 1, 0, sc);
-    for (const Span &z : {a1, a2})
-      if (spans_overlap(z, qs) || spans_overlap(z, ks) || spans_overlap(z, in))
+    const Span a3 = quant_v ? span_of(layout->v_scale, 1, 0, sc) : Span{0, 0};
+    for (const Span &z : {a1, a2, a3})
+      if (spans_overlap(z, qs) || spans_overlap(z, ks) || spans_overlap(z, vs) ||
+          spans_overlap(z, in))
         return fail(SOL_ERR_INVALID_ARG, "%s: a scale array overlaps a tensor", fn);
-    if (spans_overlap(a1, a2))
-      return fail(SOL_ERR_INVALID_ARG, "%s: q_scale and k_scale overlap", fn);
+    if (spans_overlap(a1, a2) || spans_overlap(a1, a3) || spans_overlap(a2, a3))
+      return fail(SOL_ERR_INVALID_ARG, "%s: the scale arrays overlap", fn);
   }
   for (const void *g : {gamma_q, gamma_k}) {
     if (!g) continue;
     const Span gs = span_of(g, 1, 0, head_dim * 2);
-    if (spans_overlap(gs, qs) || spans_overlap(gs, ks))
+    if (spans_overlap(gs, qs) || spans_overlap(gs, ks) || spans_overlap(gs, vs))
       return fail(SOL_ERR_INVALID_ARG, "%s: an output overlaps gamma", fn);
   }
 
@@ -436,10 +452,27 @@ sol_status sol_qknorm_rope3d_ex(const void *qkv, int64_t ld_qkv, void *q_out, vo
   a.q_scale = layout->q_scale;
   a.k_scale = layout->k_scale;
   a.n_heads = static_cast<int>(n_heads);
+  a.per_axis = layout->per_axis_freq;
   const bool half = layout->half_split != 0;
   cudaError_t e = int8 ? launch_qknorm_rope3d_ex_int8out(a, half, stream, nullptr)
                        : launch_qknorm_rope3d_ex_bf16out(a, half, stream, nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "sol_qknorm_rope3d_ex launch");
+  if (quant_v) {
+    QuantArgs v{};
+    v.src = static_cast<const unsigned char *>(qkv) + 2 * D * 2;
+    v.ld_src_bytes = ld_qkv * 2;
+    v.out = layout->v_out;
+    v.scale = layout->v_scale;
+    v.out_sb = sb;
+    v.out_sr = sr;
+    v.out_sh = sh;
+    v.rows = rows;
+    v.L = static_cast<int>(L);
+    v.nvec = static_cast<int>(D * 2 / 16);
+    v.n_heads = static_cast<int>(n_heads);
+    e = launch_quantize_heads_int8(v, static_cast<int>(head_dim), stream, nullptr);
+    if (e != cudaSuccess) return cuda_fail(e, "sol_qknorm_rope3d_ex v quantisation launch");
+  }
   return ok();
 }
 

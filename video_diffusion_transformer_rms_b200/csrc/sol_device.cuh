@@ -214,4 +214,22 @@ struct GridCursor {
   }
 };
 
+// ---- INT8 codes ---------------------------------------------------------
+
+// Round-half-even of x*s for |x*s| <= 127 by adding 1.5 * 2^23: the fp32
+// sum has an ulp of 1, so one FMA rounds the exact product to an integer and
+// leaves it, as a two's-complement byte, in the low byte of the bit pattern.
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
+// Low bytes of four words, in order, as one word.
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// 8-byte streaming store (evict-first, like st_stream16).
+__device__ __forceinline__ void st_stream8(void *gmem_dst, uint32_t lo, uint32_t hi) {
+  asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};\n" ::"l"(gmem_dst), "r"(lo), "r"(hi)
+               : "memory");
+}
+
 }  // namespace sol

@@ -108,6 +108,24 @@ struct QkArgs {
   float *q_scale;
   float *k_scale;
   int n_heads;
+  int per_axis;  // 1: each rotary section its own frequency ladder, theta^(-j/s)
+};
+
+// Per-head symmetric INT8 quantisation of rows of bf16 head vectors (the v
+// columns of merged QKV): codes to out + b*out_sb + r*out_sr + h*out_sh
+// (bytes), scales max|x|/127 to scale[(b*L + r)*n_heads + h].
+struct QuantArgs {
+  const void *src;       // row 0's first element
+  int64_t ld_src_bytes;  // row pitch of src
+  void *out;
+  float *scale;
+  int64_t out_sb;
+  int64_t out_sr;
+  int64_t out_sh;
+  int64_t rows;          // B * L
+  int L;
+  int nvec;              // 16-byte vectors per row (D / 8)
+  int n_heads;
 };
 
 // First-Block-Cache change detector.  `partial` is the caller's workspace:
@@ -157,6 +175,9 @@ cudaError_t launch_qknorm_rope3d_ex_bf16out(const QkArgs &a, bool half_split, cu
                                            Geometry *geo);
 cudaError_t launch_qknorm_rope3d_ex_int8out(const QkArgs &a, bool half_split, cudaStream_t stream,
                                            Geometry *geo);
+// head_dim 64, 128 or 256 (8, 16 or 32 lanes per head).
+cudaError_t launch_quantize_heads_int8(const QuantArgs &a, int head_dim, cudaStream_t stream,
+                                       Geometry *geo);
 inline cudaError_t launch_qknorm_rope3d(const QkArgs &a, int dtype, cudaStream_t stream,
                                         Geometry *geo) {
   return dtype == 0 ? launch_qknorm_rope3d_f32(a, stream, geo)
