@@ -306,13 +306,22 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
   cp_async_wait<0>();
 }
 
+// The CTA split each variant takes, measured inside a step at the 5 s clip:
+// the row-reduction rule (pick_split, <= 6 vectors per thread: 128 x 5 at
+// D = 5120, which divides the row exactly) for interleaved INT8 (0.86 against
+// 0.97 ms) and half-split bf16 (0.92 against 0.97 ms); the QK rule
+// (pick_split_qk: 256 x 3, more warps, a sixth of the vector slots empty)
+// for interleaved bf16 and half-split INT8.
+template <bool HALF, bool OUT8>
+constexpr bool kRowSplit = HALF != OUT8;
+
 template <int G, int NT, int VPT, bool HALF, bool OUT8>
 cudaError_t launch_ex(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
-  // INT8: one row per stage halves the ring, so a third CTA (24 warps per
-  // SM) fits beside the register limit: 0.90 against 1.04 ms at the 5 s
-  // clip.  The bf16 variants keep two rows per stage (one barrier per two
-  // rows), which measured as fast or faster for them.
-  constexpr int R = OUT8 ? 1 : (VPT <= 6 ? 2 : 1);
+  // One row per ring stage for INT8 and for half-split bf16 (half the ring,
+  // more CTAs per SM; INT8 0.90 against 1.04 ms at the 5 s clip), two rows
+  // per stage (one barrier per two rows) for interleaved bf16, which measured
+  // as fast or faster for it.
+  constexpr int R = (OUT8 || HALF) ? 1 : (VPT <= 6 ? 2 : 1);
   constexpr int S = 2;
   const void *fn =
       reinterpret_cast<const void *>(&qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8>);
@@ -332,7 +341,7 @@ cudaError_t dispatch_ex(const QkArgs &a, int threads, int vpt, cudaStream_t stre
                         Geometry *geo) {
 #define SOL_CASE(NT, V) \
   if (threads == NT && vpt == V) return launch_ex<G, NT, V, HALF, OUT8>(a, stream, geo);
-  if constexpr (OUT8 && !HALF) {
+  if constexpr (kRowSplit<HALF, OUT8>) {
     SOL_SPLITS(SOL_CASE)
   } else {
     SOL_QK_SPLITS(SOL_CASE)

@@ -10,7 +10,11 @@ cudaError_t launch_qknorm_rope3d_ex_bf16out(const QkArgs &a, bool half_split, cu
   const int G = a.head_dim * 2 / 16;
   if (a.npairs > qk::kMaxPairs) return cudaErrorInvalidValue;
   int threads = 0, vpt = 0;
-  if (!pick_split_qk(a.nvec_q, &threads, &vpt)) return cudaErrorInvalidValue;
+  // the split rule of qk::kRowSplit, which dispatch_ex instantiates
+  const bool row = half_split ? qk::kRowSplit<true, false> : qk::kRowSplit<false, false>;
+  const bool split = row ? pick_split(a.nvec_q, &threads, &vpt)
+                         : pick_split_qk(a.nvec_q, &threads, &vpt);
+  if (!split) return cudaErrorInvalidValue;
   switch (G) {
     case 8:
       return half_split ? qk::dispatch_ex<8, true, false>(a, threads, vpt, stream, geo)
