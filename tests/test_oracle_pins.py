@@ -412,6 +412,31 @@ def test_rope_audio_rows_are_1d_temporal():
     assert np.max(np.abs(q[55, :32] - q[0, :32])) > 1e-3
 
 
+@pytest.mark.parametrize("half", [False, True])
+def test_rope_composition_adds_angles(half):
+    # R(phi1) R(phi2) = R(phi1 + phi2): with eps = 0 and no gamma a head that
+    # is already normalised passes QKNorm unchanged (rms 1), so
+    # rotating audio row i1's output again as audio row i2 equals rotating
+    # the input once as audio row i1 + i2 (positions (i, 0, 0))
+    hd, nh, na = 128, 2, 12
+    x = f32(RNG.standard_normal((1, 3 * nh * hd)))
+
+    def rope_audio(inp, i):
+        rows = np.repeat(inp, na, axis=0)
+        q, k = oracle.qknorm_rope3d_ex(rows, 1, 1, 1, na - 1, nh, hd, (16, 24, 24), 0.0, 1e4,
+                                       half)
+        return q[1 + i], k[1 + i]  # row 0 is the single video row at (0, 0, 0)
+
+    for i1, i2 in ((1, 2), (3, 4), (5, 5)):
+        q1, k1 = rope_audio(x, i1)
+        # fed back as fp32 (the oracle's input type): ~1e-7 relative rounding
+        again = f32(np.concatenate([q1, k1, np.zeros(nh * hd)])[None, :])
+        q12, k12 = rope_audio(again, i2)
+        q_once, k_once = rope_audio(x, i1 + i2)
+        np.testing.assert_allclose(q12, q_once, rtol=0, atol=1e-6)
+        np.testing.assert_allclose(k12, k_once, rtol=0, atol=1e-6)
+
+
 def test_rope_scores_depend_only_on_position_difference():
     # q.k per head after RoPE depends only on (dt, dh, dw) (RoFormer's
     # relative-position property), so equal displacements give equal scores.
