@@ -2,7 +2,7 @@
 for profilers (ncu) that should capture a small, self-contained case.
 
     python -m video_diffusion_transformer_rms_b200.profile_case \
-        [--workload clip5s] [--frames 4] [--launches 1] [--kernel norm|gemm|qk_bhsd|qk_half|qk_int8]
+        [--workload clip5s] [--frames 4] [--launches 1] [--kernel norm|gemm|qk_bhsd|qk_half|qk_int8|next]
 
 The slice keeps the clip's H x W latent grid, D and head layout, takes the
 first `--frames` latent frames (T) and scales the audio rows by the same
@@ -12,14 +12,15 @@ meaningful while the device footprint stays near 1.5 GB.  `--kernel gemm`
 runs the MLP up-projection with fused GELU on the same slice instead
 (A [rows, D], W1 [4D, D], C [rows, 4D]: about 1 GB at 4 frames), and
 `--kernel qk_*` one QKNorm+RoPE epilogue variant ([B, H, L, hd] output,
-half-split pairs, INT8 output).
+half-split pairs, INT8 output), and `--kernel next` the fused residual +
+RMS-AdaLN and the change detector (read-only, then with the cache refresh).
 """
 import argparse
 import dataclasses
 
 import torch
 
-from . import api
+from . import _abi, api
 from .workloads import WORKLOADS, make_inputs
 
 
@@ -29,7 +30,7 @@ def main():
     ap.add_argument("--frames", type=int, default=4)
     ap.add_argument("--launches", type=int, default=1)
     ap.add_argument("--kernel", default="norm",
-                    choices=["norm", "gemm", "qk_bhsd", "qk_half", "qk_int8"])
+                    choices=["norm", "gemm", "qk_bhsd", "qk_half", "qk_int8", "next"])
     args = ap.parse_args()
     full = WORKLOADS[args.workload]
     T = max(1, min(full.T, args.frames))
@@ -46,6 +47,17 @@ def main():
     y = torch.empty_like(x)
     out = torch.empty_like(h)
     qk = torch.empty((w.B, w.L, 2 * D), dtype=qkv.dtype, device=qkv.device)
+    if args.kernel == "next":
+        ws = torch.empty(_abi.sol_residual_change_workspace_bytes(w.B), dtype=torch.uint8,
+                         device=x.device)
+        for _ in range(args.launches):
+            api.gate_residual_rms_adaln(h, br, t["gate"], t["scale"], t["shift"], w.n_video,
+                                        h_out=out, y=y, eps=w.eps)
+            api.residual_change(h, br, workspace=ws)
+            api.residual_change(h, br, prev_out=out, workspace=ws)
+        torch.cuda.synchronize()
+        print(f"{w.name}: {w.rows} rows, D={D}, {args.launches} launch(es) of the next rows")
+        return
     if args.kernel.startswith("qk_"):
         opts = {"qk_bhsd": {"layout": "bhsd"}, "qk_half": {"half_split": True},
                 "qk_int8": {"int8": True}}[args.kernel]
