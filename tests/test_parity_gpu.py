@@ -617,6 +617,25 @@ def test_qknorm_rope3d_ex_quantized_v(name, layout):
     assert torch.equal(qs, qs2) and torch.equal(ks, ks2)
 
 
+@pytest.mark.parametrize("secs", [(64, 0, 0), (0, 32, 32), (20, 0, 44), (16, 24, 24)])
+def test_qknorm_rope3d_ex_per_axis_sections(secs):
+    # per-axis ladders with empty and uneven sections (an empty section holds
+    # no pair, so its size never divides)
+    B, T, H, W, na, nh, hd = 1, 4, 6, 5, 9, 4, 128
+    L = T * H * W + na
+    D = nh * hd
+    qkv = activation(B * L, 3 * D, torch.bfloat16, DEV, 81, outliers=True).view(B, L, 3 * D)
+    gq = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 82)
+    gk = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 83)
+    for half in (False, True):
+        q, k = api.qknorm_rope3d_ex(qkv, T, H, W, na, nh, hd, secs, gq, gk, half_split=half,
+                                    per_axis_freq=True)
+        wq, wk = oracle.qknorm_rope3d_ex(_o(qkv.view(B * L, 3 * D)), T, H, W, na, nh, hd, secs,
+                                         1e-6, 1e4, half, _o(gq), _o(gk), per_axis=True)
+        assert_close(q.reshape(B * L, D), wq, f"per-axis sections {secs} half={half} q")
+        assert_close(k.reshape(B * L, D), wk, f"per-axis sections {secs} half={half} k")
+
+
 def test_qknorm_rope3d_ex_interleaved_matches_default_entry_point():
     # same arithmetic as sol_qknorm_rope3d, only the addressing differs:
     # bit-identical results in both layouts
@@ -634,25 +653,32 @@ def test_qknorm_rope3d_ex_interleaved_matches_default_entry_point():
 
 @pytest.mark.parametrize("hd,secs", [(64, (8, 12, 12)), (256, (32, 48, 48))])
 @pytest.mark.parametrize("half", [False, True])
-def test_qknorm_rope3d_ex_head_dims(hd, secs, half):
+@pytest.mark.parametrize("per_axis", [False, True])
+def test_qknorm_rope3d_ex_head_dims(hd, secs, half, per_axis):
     B, T, H, W, na, nh = 2, 3, 5, 7, 11, 6
     L = T * H * W + na
     D = nh * hd
     qkv = activation(B * L, 3 * D, torch.bfloat16, DEV, 61, outliers=True).view(B, L, 3 * D)
     gq = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 62)
     gk = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 63)
+    wq, wk = oracle.qknorm_rope3d_ex(_o(qkv.view(B * L, 3 * D)), T, H, W, na, nh, hd, secs,
+                                     1e-6, 1e4, half, _o(gq), _o(gk), per_axis=per_axis)
+    tag = f"hd={hd} half={half} per_axis={per_axis}"
     for int8 in (False, True):
         res = api.qknorm_rope3d_ex(qkv, T, H, W, na, nh, hd, secs, gq, gk, layout="bhsd",
-                                   half_split=half, int8=int8)
-        wq, wk = oracle.qknorm_rope3d_ex(_o(qkv.view(B * L, 3 * D)), T, H, W, na, nh, hd, secs,
-                                         1e-6, 1e4, half, _o(gq), _o(gk))
+                                   half_split=half, int8=int8, per_axis_freq=per_axis,
+                                   quantize_v=int8)
         q, k = (_bshd(r, "bhsd").reshape(B * L, D) for r in res[:2])
         if int8:
-            _check_int8(q, res[2], wq, nh, hd, f"hd={hd} q")
-            _check_int8(k, res[3], wk, nh, hd, f"hd={hd} k")
+            _check_int8(q, res[2], wq, nh, hd, tag + " q")
+            _check_int8(k, res[3], wk, nh, hd, tag + " k")
+            # v, quantised as it stands (G = hd/8 lanes per head in its kernel too)
+            want_v = oracle.widen(_o(qkv.view(B * L, 3 * D)[:, 2 * D:].contiguous()))
+            _check_int8(_bshd(res[4], "bhsd").reshape(B * L, D), res[5], want_v, nh, hd,
+                        tag + " v")
         else:
-            assert_close(q, wq, f"hd={hd} half={half} q")
-            assert_close(k, wk, f"hd={hd} half={half} k")
+            assert_close(q, wq, tag + " q")
+            assert_close(k, wk, tag + " k")
 
 
 
