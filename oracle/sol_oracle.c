@@ -28,7 +28,7 @@
  *     t/h/w sections (M-RoPE style), sections 16/24/24 of 64 pairs, theta
  *     10000, audio tokens at positions (t=i,0,0).
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *   eps inside the square root; mean over all D (or head_dim) channels;
  *   order normalise -> gamma -> modulate; modulation (1 + scale) not scale;
  *   per sample b the rows are the N_v = T*H*W video rows (raster order,
