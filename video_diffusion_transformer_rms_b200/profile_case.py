@@ -2,7 +2,7 @@
 for profilers (ncu) that should capture a small, self-contained case.
 
     python -m video_diffusion_transformer_rms_b200.profile_case \
-        [--workload clip5s] [--frames 4] [--launches 1] [--kernel norm|gemm|qk_bhsd|qk_half|qk_int8|next]
+        [--workload clip5s] [--frames 4] [--launches 1] [--kernel norm|gemm|qk_bhsd|qk_half|qk_int8|qk_all|next]
 
 The slice keeps the clip's H x W latent grid, D and head layout, takes the
 first `--frames` latent frames (T) and scales the audio rows by the same
@@ -12,7 +12,8 @@ meaningful while the device footprint stays near 1.5 GB.  `--kernel gemm`
 runs the MLP up-projection with fused GELU on the same slice instead
 (A [rows, D], W1 [4D, D], C [rows, 4D]: about 1 GB at 4 frames), and
 `--kernel qk_*` one QKNorm+RoPE epilogue variant ([B, H, L, hd] output,
-half-split pairs, INT8 output), and `--kernel next` the fused residual +
+half-split pairs, INT8 output; qk_all runs the first two and INT8 with the
+quantised v, one launch each), and `--kernel next` the fused residual +
 RMS-AdaLN and the change detector (read-only, then with the cache refresh).
 """
 import argparse
@@ -30,7 +31,7 @@ def main():
     ap.add_argument("--frames", type=int, default=4)
     ap.add_argument("--launches", type=int, default=1)
     ap.add_argument("--kernel", default="norm",
-                    choices=["norm", "gemm", "qk_bhsd", "qk_half", "qk_int8", "next"])
+                    choices=["norm", "gemm", "qk_bhsd", "qk_half", "qk_int8", "qk_all", "next"])
     args = ap.parse_args()
     full = WORKLOADS[args.workload]
     T = max(1, min(full.T, args.frames))
@@ -59,11 +60,15 @@ def main():
         print(f"{w.name}: {w.rows} rows, D={D}, {args.launches} launch(es) of the next rows")
         return
     if args.kernel.startswith("qk_"):
-        opts = {"qk_bhsd": {"layout": "bhsd"}, "qk_half": {"half_split": True},
-                "qk_int8": {"int8": True}}[args.kernel]
+        variants = {"qk_bhsd": [{"layout": "bhsd"}], "qk_half": [{"half_split": True}],
+                    "qk_int8": [{"int8": True}],
+                    "qk_all": [{"layout": "bhsd"}, {"half_split": True},
+                               {"int8": True, "quantize_v": True}]}[args.kernel]
         for _ in range(args.launches):
-            api.qknorm_rope3d_ex(qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim,
-                                 w.sections, t["gamma_q"], t["gamma_k"], w.eps, w.theta, **opts)
+            for opts in variants:
+                api.qknorm_rope3d_ex(qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim,
+                                     w.sections, t["gamma_q"], t["gamma_k"], w.eps, w.theta,
+                                     **opts)
         torch.cuda.synchronize()
         print(f"{w.name}: {w.rows} rows, D={D}, {args.launches} launch(es) of {args.kernel}")
         return
