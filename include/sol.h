@@ -362,7 +362,9 @@ const char *sol_status_string(sol_status status);
  * next libsol call. */
 const char *sol_last_error(void);
 
-/* ABI version, (major << 16) | minor. */
+/* ABI version, (major << 16) | minor.  2.0: sol_qk_layout gained
+ * per_axis_freq, reserved, v_out and v_scale (a larger struct; callers built
+ * against 1.x must be rebuilt). */
 int sol_version(void);
 
 #ifdef __cplusplus

@@ -39,7 +39,7 @@ def test_status_strings_and_version():
     assert _abi.status_string(_abi.SOL_OK) == "SOL_OK"
     assert _abi.status_string(_abi.SOL_ERR_MISALIGNED) == "SOL_ERR_MISALIGNED"
     assert _abi.status_string(99) == "SOL_ERR_UNKNOWN"
-    assert _abi.sol_version() >> 16 == 1
+    assert _abi.sol_version() >> 16 == 2  # sol_qk_layout grew in 2.0
 
 
 # Fake device addresses: validation must reject these calls on the host.

@@ -107,12 +107,18 @@ int resident_blocks(const void *kernel, int threads, size_t smem) {
   if (it != c.occ.end()) return it->second;
   auto akey = std::make_pair(kernel, dev);
   if (!c.attr_set[akey]) {
+    // allow dynamic shared memory up to the opt-in limit less the kernel's
+    // static shared memory (the attribute counts only the dynamic part)
     int optin = 0;
+    cudaFuncAttributes fa{};
     if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
-        cudaSuccess)
+            cudaSuccess ||
+        cudaFuncGetAttributes(&fa, kernel) != cudaSuccess)
       return 0;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) !=
-        cudaSuccess)
+    const int dyn_max = optin - static_cast<int>(fa.sharedSizeBytes);
+    if (dyn_max <= 0 ||
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max) !=
+            cudaSuccess)
       return 0;
     c.attr_set[akey] = true;
   }
@@ -155,7 +161,7 @@ using namespace sol;
 
 extern "C" {
 
-int sol_version(void) { return (1 << 16) | 0; }
+int sol_version(void) { return (2 << 16) | 0; }
 
 const char *sol_status_string(sol_status s) {
   switch (s) {
