@@ -437,6 +437,27 @@ def test_rope_composition_adds_angles(half):
         np.testing.assert_allclose(k12, k_once, rtol=0, atol=1e-6)
 
 
+def test_rope_video_column_grid_is_1d_temporal():
+    # H = W = 1: video row t sits at (t, 0, 0), exactly where an audio-only
+    # sequence puts audio row t, so the two agree element by element (both
+    # reduce to 1D RoPE on the t section)
+    rows, nh, hd = 7, 2, 128
+    qkv = f32(np.tile(RNG.standard_normal((1, 3 * nh * hd)), (rows, 1)))  # one row repeated
+    for half in (False, True):
+        qv, kv = oracle.qknorm_rope3d_ex(qkv, rows, 1, 1, 0, nh, hd, (16, 24, 24), 1e-6, 1e4,
+                                         half)
+        qa, ka = oracle.qknorm_rope3d_ex(qkv, 0, 0, 0, rows, nh, hd, (16, 24, 24), 1e-6, 1e4,
+                                         half)
+        np.testing.assert_array_equal(qv, qa)
+        np.testing.assert_array_equal(kv, ka)
+        # the same input row: row 3 differs from row 0 only by its rotation,
+        # which touches the t section and nothing else
+        assert np.abs(qv[3] - qv[0]).max() > 1e-3
+        t_cols = np.r_[0:32] if not half else np.r_[0:16, 64:80]
+        other = np.setdiff1d(np.arange(hd), t_cols)
+        np.testing.assert_array_equal(qv[3, other], qv[0, other])
+
+
 def test_rope_scores_depend_only_on_position_difference():
     # q.k per head after RoPE depends only on (dt, dh, dw) (RoFormer's
     # relative-position property), so equal displacements give equal scores.
