@@ -485,8 +485,10 @@ def run_ours(args):
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                     "steps": e2e["steps"],
                     "path": "pinned host inputs -> H2D -> api.rms_adaln / api.qknorm_rope3d / "
-                            "api.gate_residual -> D2H of y, q, k, out; copy-in, kernels and "
-                            "copy-out on three streams ordered by events; CUDA events"},
+                            "api.gate_residual -> D2H of y, q, k, out; of the merged QKV rows "
+                            "only the q and k columns the step reads are copied (one pitched "
+                            "copy); copy-in, kernels and copy-out on three streams ordered by "
+                            "events; CUDA events"},
             "gpu_launches": len(KERNELS) * K,
             "clocks": clock_info,
         }
@@ -567,13 +569,30 @@ def run_e2e(args, w, t, stream, api):
     for n in names:
         host[n].copy_(t[n])
     dev = {n: torch.empty_like(t[n]) for n in names}
+    # merged QKV: the step reads only the q and k columns, so one pitched copy
+    # brings those (2D of every 3D-wide host row) into a packed [rows, 2D]
+    # device buffer, which the API takes as merged rows with ld_qkv = 2D
+    from cuda.bindings import runtime as cudart
+    rows, esize = w.rows, t["qkv"].element_size()
+    dev["qkv"] = torch.empty((rows, 2 * D), dtype=t["qkv"].dtype, device=t["qkv"].device)
+
+    def copy_in(n):
+        if n != "qkv":
+            dev[n].copy_(host[n], non_blocking=True)
+            return
+        err, = cudart.cudaMemcpy2DAsync(dev[n].data_ptr(), 2 * D * esize, host[n].data_ptr(),
+                                        3 * D * esize, 2 * D * esize, rows,
+                                        cudart.cudaMemcpyKind.cudaMemcpyHostToDevice,
+                                        s_in.cuda_stream)
+        if err != cudart.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaMemcpy2DAsync: {err}")
     y = torch.empty((w.B, w.L, D), dtype=t["x"].dtype, device=t["x"].device)
     qk = torch.empty((w.B, w.L, 2 * D), dtype=t["x"].dtype, device=t["x"].device)
     out = torch.empty_like(y)
     results = {"rms_adaln": y, "qknorm_rope3d": qk, "gate_residual": out}
     host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
                 for k, v in results.items()}
-    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    h2d = sum(dev[n].numel() * dev[n].element_size() for n in names)  # bytes copied in
     d2h = sum(v.numel() * v.element_size() for v in host_out.values())
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()  # noqa: E731
@@ -585,7 +604,7 @@ def run_e2e(args, w, t, stream, api):
             api.rms_adaln(dev["x"].view(w.B, w.L, D), dev["scale"], dev["shift"], w.n_video,
                           eps=w.eps, out=y, stream=stream)
         elif k == "qknorm_rope3d":
-            api.qknorm_rope3d(dev["qkv"].view(w.B, w.L, 3 * D), w.T, w.H, w.W, w.n_audio,
+            api.qknorm_rope3d(dev["qkv"].view(w.B, w.L, 2 * D), w.T, w.H, w.W, w.n_audio,
                               w.n_heads, w.head_dim, w.sections, dev["gamma_q"],
                               dev["gamma_k"], w.eps, w.theta, q_out=qk[..., :D],
                               k_out=qk[..., D:], stream=stream)
@@ -599,7 +618,7 @@ def run_e2e(args, w, t, stream, api):
                 s_in.wait_event(read_done[k])
             with torch.cuda.stream(s_in):
                 for n in g:
-                    dev[n].copy_(host[n], non_blocking=True)
+                    copy_in(n)
             arrived = ev()
             arrived.record(s_in)
             stream.wait_event(arrived)
