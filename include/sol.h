@@ -2,7 +2,8 @@
  * sol.h - C ABI of libsol, the fused per-token hot path of a joint
  * video+audio diffusion-transformer block on NVIDIA B200 (sm_100a).
  *
- * Three operations, each one kernel launch:
+ * The three operations of the per-token path, each one kernel launch (the
+ * variants and next steps are declared further down):
  *   sol_rms_adaln      RMSNorm then AdaLN modulation  x^ * (1 + scale) + shift
  *   sol_gate_residual  AdaLN-gated residual add        h + gate * branch
  *   sol_qknorm_rope3d  per-head RMS norm of q and k, then 3D multimodal RoPE
@@ -12,8 +13,8 @@
  * round-trips across the modulation branch; "fused QKNorm + RoPE": no
  * separate read/write passes over Q and K, no separate 3D MM-RoPE indexing);
  * the KOCPC Sol-H3 article repeats them in "Technical Composition".  The
- * gated residual is the "leftover elementwise chain" of the same page's
- * torch.compile row, the adaLN gate of the DiT block.
+ * gated residual is one of the elementwise steps that the same page leaves to
+ * its torch.compile row: the adaLN gate of the DiT block.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -99,8 +100,8 @@ sol_status sol_rms_adaln(const void *x, void *y, const void *scale,
                          sol_dtype dtype, sol_stream_t stream);
 
 /*
- * AdaLN-gated residual add (the adaLN gate of the DiT block; the residual
- * update the Sol pages fold under "leftover elementwise chains").  For every
+ * AdaLN-gated residual add (the adaLN gate of the DiT block; one of the
+ * elementwise steps the Sol pages leave to torch.compile capture).  For every
  * row of sample b with modality m:
  *
  *   out[c] = h[c] + gate[b][m][c] * branch[c]
@@ -116,9 +117,9 @@ sol_status sol_gate_residual(const void *h, const void *branch,
 
 /*
  * Fused AdaLN-gated residual + RMS-AdaLN: the block's "h = h + gate * attn;
- * x = RMS-AdaLN(h)" chain in one pass (the pages' "leftover elementwise
- * chains" of the torch.compile row fused into the "fused RMS-AdaLN" row of
- * the Sol Video Inference Engine MiniMax-H3 fusion table).  For every row of
+ * x = RMS-AdaLN(h)" chain in one pass (an elementwise step of the pages'
+ * torch.compile row fused into the fused RMS-AdaLN row of the Sol Video
+ * Inference Engine MiniMax-H3 fusion table).  For every row of
  * sample b with modality m:
  *
  *   h_out[c] = h[c] + gate[b][m][c] * branch[c]

@@ -19,7 +19,7 @@
  *   - AdaLN branches firing on every denoising step, joint video-plus-audio
  *     single-stream sequence: same H3-OnDevice page, model description; the
  *     ThakiCloud MiniMax-H3 post, section "MiniMax-H3: what the model does,
- *     and how much" ("dense single-stream").
+ *     and how much" (a dense transformer over one joint sequence).
  *   - RMSNorm: y = x / sqrt(mean(x^2) + eps) (Zhang & Sennrich, 2019).
  *   - AdaLN modulation x*(1+scale)+shift and the gated residual h+gate*branch
  *     (adaLN-Zero DiT block, Peebles & Xie, 2023).

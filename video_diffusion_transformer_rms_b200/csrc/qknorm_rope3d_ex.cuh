@@ -5,7 +5,7 @@
 //   - the half-split rotary pair layout, pair i = elements (i, i + hd/2);
 //   - INT8 output: symmetric per-(row, head) codes round(x * 127 / max|x|)
 //     with fp32 scales max|x| / 127, the quantised Q/K that the KOCPC Sol-H3
-//     article's 4x/8x B300 runs send between GPUs ("INT8 QKV ... transfer");
+//     article's 4x/8x B300 runs send between GPUs;
 //   - a per-axis frequency ladder: each of the t/h/w sections a RoPE of its
 //     own, pair j of a section of s pairs at theta^(-j/s).
 // Same structure as qknorm_rope3d.cuh (ring, cursors, per-row angle tables,

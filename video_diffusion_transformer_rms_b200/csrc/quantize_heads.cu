@@ -1,7 +1,7 @@
 // Per-head symmetric INT8 quantisation of bf16 head vectors: the v part of a
 // merged QKV row for the INT8 Q/K/V exchange between GPUs that the KOCPC
-// Sol-H3 article's 4x/8x B300 runs use ("INT8 QKV ... transfer").  For each
-// token row and head h (channels [h*hd, (h+1)*hd) of the row):
+// Sol-H3 article's 4x/8x B300 runs use.  For each token row and head h
+// (channels [h*hd, (h+1)*hd) of the row):
 //   scale = max|x| / 127,  code = round_half_even(x * 127 / max|x|)
 // (scale 0 and all codes 0 for an all-zero head), codes in the same layouts as
 // the QKNorm+RoPE epilogue's INT8 q and k.
