@@ -162,24 +162,31 @@ class ClockSampler:
             self.proc.kill()
         self.file.flush()
         self.file.seek(0)
+        lines = self.file.read().splitlines()
+        os.unlink(self.file.name)
+        return self.summarise(lines, self.uuid, t0, t1)
+
+    @classmethod
+    def summarise(cls, lines, uuid, t0, t1):
+        """Median SM clock, max clock and the throttle reasons active in the
+        samples of this GPU (uuid) taken within [t0 - 1, t1 + 1] (all of its
+        samples if none fall inside)."""
         rows = []
-        for line in self.file.read().splitlines():
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 10:
                 continue
-            uuid = parts[2]
-            if self.uuid and self.uuid not in uuid and uuid not in f"GPU-{self.uuid}":
+            if uuid and uuid not in parts[2] and parts[2] not in f"GPU-{uuid}":
                 continue
             try:
                 ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
                 rows.append((ts, float(parts[3]), float(parts[4]), parts[6:10]))
             except ValueError:
                 continue
-        os.unlink(self.file.name)
         inside = [r for r in rows if t0 - 1 <= r[0] <= t1 + 1] or rows
         if not inside:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "no samples"}
-        reasons = sorted({name for r in inside for name, v in zip(self.REASONS, r[3])
+        reasons = sorted({name for r in inside for name, v in zip(cls.REASONS, r[3])
                           if v.strip().lower() == "active"})
         return {"sm_mhz": float(np.median([r[1] for r in inside])),
                 "sm_max_mhz": float(max(r[2] for r in inside)), "reasons": reasons,
