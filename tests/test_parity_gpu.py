@@ -636,6 +636,25 @@ def test_qknorm_rope3d_ex_per_axis_sections(secs):
         assert_close(k.reshape(B * L, D), wk, f"per-axis sections {secs} half={half} k")
 
 
+def test_qknorm_rope3d_packed_qk_input():
+    # a [B, L, 2D] tensor holding only q and k (ld_qkv = 2D, the form the
+    # end-to-end path copies to the device) gives the same q and k, bit for
+    # bit, as the merged [B, L, 3D] rows
+    w = WORKLOADS["medium"]
+    t = make_inputs(w, DEV, which=("qknorm_rope3d",))
+    qkv = t["qkv"].view(w.B, w.L, 3 * w.D)
+    packed = qkv[..., :2 * w.D].contiguous()
+    args = (w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections, t["gamma_q"],
+            t["gamma_k"], w.eps, w.theta)
+    q0, k0 = api.qknorm_rope3d(qkv, *args)
+    q1, k1 = api.qknorm_rope3d(packed, *args)
+    assert torch.equal(q0, q1) and torch.equal(k0, k1)
+    for kw in ({"layout": "bhsd"}, {"int8": True}):
+        r0 = api.qknorm_rope3d_ex(qkv, *args, **kw)
+        r1 = api.qknorm_rope3d_ex(packed, *args, **kw)
+        assert all(torch.equal(a, b) for a, b in zip(r0, r1))
+
+
 def test_qknorm_rope3d_ex_interleaved_matches_default_entry_point():
     # same arithmetic as sol_qknorm_rope3d, only the addressing differs:
     # bit-identical results in both layouts
