@@ -30,6 +30,18 @@ def _ptr(t: Optional[torch.Tensor]):
     return t.data_ptr()
 
 
+def _expect(t: Optional[torch.Tensor], shape, name: str, like: torch.Tensor):
+    """The library sees only pointers, so every tensor handed to it must be
+    contiguous, of exactly this shape, and on the device of `like`."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous tensor of shape {tuple(shape)}, got "
+                         f"{tuple(t.shape)}{'' if t.is_contiguous() else ' (not contiguous)'}")
+    if t.device != like.device:
+        raise ValueError(f"{name} is on {t.device}, the inputs on {like.device}")
+
+
 def _stream(stream: Optional[torch.cuda.Stream]):
     s = stream if stream is not None else torch.cuda.current_stream()
     return s.cuda_stream
@@ -44,6 +56,9 @@ def rms_adaln(x: torch.Tensor, scale: torch.Tensor, shift: torch.Tensor, n_video
     if x.dim() != 3 or not x.is_contiguous():
         raise ValueError("x must be a contiguous [B, L, D] tensor")
     B, L, D = x.shape
+    for t, shape, name in ((scale, (B, 2, D), "scale"), (shift, (B, 2, D), "shift"),
+                           (gamma, (D,), "gamma"), (out, (B, L, D), "out")):
+        _expect(t, shape, name, x)
     y = torch.empty_like(x) if out is None else out
     _abi.check(_abi.sol_rms_adaln(_ptr(x), _ptr(y), _ptr(scale), _ptr(shift), _ptr(gamma),
                                   B, L, n_video, D, eps, _dtype(x, y, scale, shift, gamma),
@@ -55,9 +70,12 @@ def gate_residual(h: torch.Tensor, branch: torch.Tensor, gate: torch.Tensor, n_v
                   out: Optional[torch.Tensor] = None,
                   stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """out = h + gate[b, m] * branch; h/branch: [B, L, D], gate: [B, 2, D]."""
-    if h.dim() != 3 or not h.is_contiguous() or branch.shape != h.shape:
-        raise ValueError("h and branch must be contiguous [B, L, D] tensors of one shape")
+    if h.dim() != 3 or not h.is_contiguous():
+        raise ValueError("h must be a contiguous [B, L, D] tensor")
     B, L, D = h.shape
+    for t, shape, name in ((branch, (B, L, D), "branch"), (gate, (B, 2, D), "gate"),
+                           (out, (B, L, D), "out")):
+        _expect(t, shape, name, h)
     o = torch.empty_like(h) if out is None else out
     _abi.check(_abi.sol_gate_residual(_ptr(h), _ptr(branch), _ptr(gate), _ptr(o), B, L,
                                       n_video, D, _dtype(h, branch, gate, o), _stream(stream)))
@@ -72,9 +90,14 @@ def gate_residual_rms_adaln(h: torch.Tensor, branch: torch.Tensor, gate: torch.T
                             ) -> Tuple[torch.Tensor, torch.Tensor]:
     """h_out = h + gate[b, m] * branch; y = RMS-AdaLN(h_out) with scale/shift;
     returns (h_out, y).  Pass h_out=h to update the residual stream in place."""
-    if h.dim() != 3 or not h.is_contiguous() or branch.shape != h.shape:
-        raise ValueError("h and branch must be contiguous [B, L, D] tensors of one shape")
+    if h.dim() != 3 or not h.is_contiguous():
+        raise ValueError("h must be a contiguous [B, L, D] tensor")
     B, L, D = h.shape
+    for t, shape, name in ((branch, (B, L, D), "branch"), (gate, (B, 2, D), "gate"),
+                           (scale, (B, 2, D), "scale"), (shift, (B, 2, D), "shift"),
+                           (gamma, (D,), "gamma"), (h_out, (B, L, D), "h_out"),
+                           (y, (B, L, D), "y")):
+        _expect(t, shape, name, h)
     ho = torch.empty_like(h) if h_out is None else h_out
     yo = torch.empty_like(h) if y is None else y
     _abi.check(_abi.sol_gate_residual_rms_adaln(
@@ -94,9 +117,16 @@ def residual_change(cur: torch.Tensor, prev: torch.Tensor,
     sum |prev|, their ratio) per sample and, in the last row, for the batch.
     With prev_out (may be prev itself) the cache is refreshed to cur in the
     same pass.  The workspace is allocated by PyTorch unless given."""
-    if cur.dim() != 3 or not cur.is_contiguous() or prev.shape != cur.shape:
-        raise ValueError("cur and prev must be contiguous [B, L, D] tensors of one shape")
+    if cur.dim() != 3 or not cur.is_contiguous():
+        raise ValueError("cur must be a contiguous [B, L, D] tensor")
     B, L, D = cur.shape
+    for t, shape, name in ((prev, (B, L, D), "prev"), (prev_out, (B, L, D), "prev_out"),
+                           (out, (B + 1, 3), "out")):
+        _expect(t, shape, name, cur)
+    if out is not None and out.dtype != torch.float64:
+        raise TypeError("out must be float64")
+    if workspace is not None:
+        _expect(workspace, (workspace.numel(),), "workspace", cur)
     need = _abi.sol_residual_change_workspace_bytes(B)
     ws = workspace if workspace is not None else torch.empty(
         max(need, 16), dtype=torch.uint8, device=cur.device)
@@ -124,6 +154,8 @@ def qknorm_rope3d(qkv: torch.Tensor, T: int, H: int, W: int, n_audio: int, n_hea
     D = n_heads * head_dim
     if L != T * H * W + n_audio:
         raise ValueError("L must equal T*H*W + n_audio")
+    for t, name in ((gamma_q, "gamma_q"), (gamma_k, "gamma_k")):
+        _expect(t, (head_dim,), name, qkv)
     if q_out is None and k_out is None:
         buf = torch.empty((B, L, 2 * D), dtype=qkv.dtype, device=qkv.device)
         q_out, k_out = buf[..., :D], buf[..., D:]
@@ -131,6 +163,11 @@ def qknorm_rope3d(qkv: torch.Tensor, T: int, H: int, W: int, n_audio: int, n_hea
         raise ValueError("pass both q_out and k_out, or neither")
     if q_out.stride() != k_out.stride() or q_out.stride(2) != 1:
         raise ValueError("q_out and k_out must share a row stride with unit column stride")
+    for t, name in ((q_out, "q_out"), (k_out, "k_out")):
+        if tuple(t.shape) != (B, L, D) or t.stride(0) != L * t.stride(1):
+            raise ValueError(f"{name} must be a [B, L, D] view with packed rows")
+        if t.device != qkv.device:
+            raise ValueError(f"{name} is on {t.device}, qkv on {qkv.device}")
     ld_out = q_out.stride(1)
     st, sh, sw = sections
     _abi.check(_abi.sol_qknorm_rope3d(
@@ -160,6 +197,8 @@ def qknorm_rope3d_ex(qkv: torch.Tensor, T: int, H: int, W: int, n_audio: int, n_
     B, L, _ = qkv.shape
     if L != T * H * W + n_audio:
         raise ValueError("L must equal T*H*W + n_audio")
+    for t, name in ((gamma_q, "gamma_q"), (gamma_k, "gamma_k")):
+        _expect(t, (head_dim,), name, qkv)
     odt = torch.int8 if int8 else qkv.dtype
     if layout == "bshd":
         shape = (B, L, n_heads, head_dim)
@@ -202,6 +241,9 @@ def gemm_gelu(A: torch.Tensor, B: torch.Tensor, bias: Optional[torch.Tensor] = N
         raise ValueError("A and B must be contiguous")
     M, K = A.shape
     N = B.shape[0]
+    _expect(B, (N, K), "B", A)
+    _expect(bias, (N,), "bias", A)
+    _expect(out, (M, N), "out", A)
     C = torch.empty((M, N), dtype=A.dtype, device=A.device) if out is None else out
     need = _abi.sol_gemm_gelu_workspace_bytes(M, N, K)
     ws = torch.empty(need, dtype=torch.uint8, device=A.device) if need else None
