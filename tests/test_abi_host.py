@@ -2,6 +2,7 @@
 every function include/sol.h declares, and rejects bad arguments before any
 CUDA call (fake, never-dereferenced addresses are enough for that)."""
 import ctypes
+import os
 import subprocess
 
 import pytest
@@ -274,3 +275,51 @@ def test_qknorm_rope3d_ex_null_layout():
     assert _abi.sol_qknorm_rope3d_ex(A, 3 * 1024, A + (1 << 30), A + (2 << 30), None, None,
                                      None, 1, 2, 4, 6, 8, 8, 128, 16, 24, 24, 1e-6, 1e4, BF,
                                      None) == _abi.SOL_ERR_INVALID_ARG
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "sol.h"
+
+int main(void) {
+    sol_qk_layout lay;
+    memset(&lay, 0, sizeof lay);
+    lay.stride_b = 1;
+    lay.stride_row = 1;
+    lay.stride_head = 1;
+    lay.reserved = 1; /* must be 0: refused before any CUDA call */
+    if ((sol_version() >> 16) != 2) return 1;
+    if (sol_rms_adaln(NULL, NULL, NULL, NULL, NULL, 1, 4, 4, 8, 1e-6f, SOL_BF16, NULL) !=
+        SOL_ERR_INVALID_ARG) return 2;
+    if (strlen(sol_last_error()) == 0) return 3;
+    if (sol_qknorm_rope3d_ex((const void *)0x1000, 3 * 256, (void *)0x100000,
+                             (void *)0x200000, &lay, NULL, NULL, 1, 2, 4, 6, 8, 2, 128,
+                             16, 24, 24, 1e-6f, 1e4f, SOL_BF16, NULL) != SOL_ERR_INVALID_ARG)
+        return 4;
+    printf("%s | %s\n", sol_status_string(SOL_ERR_INVALID_ARG), sol_last_error());
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_the_library_links_from_c(tmp_path):
+    # the boundary is a C ABI: a C99 client compiles against include/sol.h with
+    # every warning an error, links libsol.so and gets statuses back (no GPU
+    # call is made: both calls fail validation)
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(_abi.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(root, "include"), str(src), "-o", str(exe),
+                    "-L", libdir, "-lsol", f"-Wl,-rpath,{libdir}"], check=True)
+    p = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert p.returncode == 0, (p.returncode, p.stdout, p.stderr)
+    assert "layout.reserved must be 0" in p.stdout
