@@ -258,6 +258,89 @@ sol_status sol_qknorm_rope3d_ex(const void *qkv, int64_t ld_qkv, void *q_out,
                                 sol_dtype dtype, sol_stream_t stream);
 
 /*
+ * Precomputed rotary table for the table-driven QKNorm + 3D RoPE entry
+ * points (the "3D MM-RoPE indexing" of the MiniMax-H3 page's "fused QKNorm +
+ * RoPE" row, done once instead of per row).
+ *
+ * Rotary positions are integers on every axis (t, h, w, and the audio index
+ * on t), so every (cos, sin) a call needs is a function of (position p,
+ * pair i) alone.  Row p of the table holds cos(p * f_i) for the head_dim/2
+ * pairs i, then sin(p * f_i): head_dim floats per row, n_pos rows.  f_i is
+ * theta^(-2i/head_dim), or with per_axis_freq theta^(-j/s) for local pair j
+ * of a section of s pairs (as sol_qk_layout.per_axis_freq).  Angles, sines
+ * and cosines are computed in fp64 and rounded once to fp32.
+ *
+ * The table depends only on these fields: build it once per video shape and
+ * reuse it for every layer and denoising step.  The caller owns `data`.
+ */
+typedef struct sol_rope_table {
+    float *data;        /* device, sol_rope_table_bytes(n_pos, head_dim)
+                           bytes, 16-byte aligned */
+    int64_t n_pos;      /* rows: positions 0 .. n_pos - 1 on every axis */
+    int64_t head_dim;   /* even, 2 .. 256 */
+    int64_t sec_t;      /* rotary pairs on t, h and w; sum = head_dim / 2 */
+    int64_t sec_h;
+    int64_t sec_w;
+    float theta;        /* > 0 */
+    int32_t per_axis_freq; /* 0 or 1, as in sol_qk_layout */
+} sol_rope_table;
+
+/* Bytes of a rotary table: n_pos * head_dim * 4 (0 if n_pos < 0, head_dim
+ * is odd or not in [2, 256], or the size overflows). */
+size_t sol_rope_table_bytes(int64_t n_pos, int64_t head_dim);
+
+/*
+ * Fill tab->data on `stream` (one kernel).  SOL_ERR_INVALID_ARG for a null
+ * table or data, n_pos < 0 or beyond 2^31 - 1, a bad head_dim, sections
+ * that do not sum to head_dim / 2, theta <= 0 or per_axis_freq outside
+ * {0, 1}; SOL_ERR_MISALIGNED if data is not 16-byte aligned.  n_pos = 0 is
+ * a no-op.
+ */
+sol_status sol_rope_table_build(const sol_rope_table *tab, sol_stream_t stream);
+
+/*
+ * sol_qknorm_rope3d with the rotation's (cos, sin) read from a rotary table
+ * built by sol_rope_table_build (on the same stream, or ordered before this
+ * call) instead of being computed per row.  head_dim, the sections, theta
+ * and the frequency rule are the table's; the other arguments and rules are
+ * those of sol_qknorm_rope3d.  The kernel keeps no per-row angle work and
+ * no CTA barrier.
+ *
+ *   tab   host pointer to the descriptor; tab->data is read by the kernel.
+ *         Every position the call meets must be a table row:
+ *         n_pos >= max(T, H, W) when T*H*W > 0, and n_pos >= n_audio
+ *         (SOL_ERR_INVALID_ARG otherwise).  The outputs must not overlap
+ *         the table.
+ * Results differ from sol_qknorm_rope3d's by the rounding of the table
+ * (fp64-exact (cos, sin) rounded once to fp32, against sincosf of the
+ * fp64-reduced angle), i.e. within an fp32 ulp or two before the bf16
+ * rounding of the output.
+ */
+sol_status sol_qknorm_rope3d_tab(const void *qkv, int64_t ld_qkv, void *q_out,
+                                 void *k_out, int64_t ld_out,
+                                 const void *gamma_q, const void *gamma_k,
+                                 const sol_rope_table *tab, int64_t B,
+                                 int64_t T, int64_t H, int64_t W,
+                                 int64_t n_audio, int64_t n_heads, float eps,
+                                 sol_dtype dtype, sol_stream_t stream);
+
+/*
+ * sol_qknorm_rope3d_ex with the rotation read from a rotary table, as
+ * sol_qknorm_rope3d_tab.  layout->per_axis_freq must equal
+ * tab->per_axis_freq (SOL_ERR_INVALID_ARG otherwise); head_dim, sections
+ * and theta are the table's; everything else as sol_qknorm_rope3d_ex.
+ */
+sol_status sol_qknorm_rope3d_ex_tab(const void *qkv, int64_t ld_qkv,
+                                    void *q_out, void *k_out,
+                                    const sol_qk_layout *layout,
+                                    const void *gamma_q, const void *gamma_k,
+                                    const sol_rope_table *tab, int64_t B,
+                                    int64_t T, int64_t H, int64_t W,
+                                    int64_t n_audio, int64_t n_heads,
+                                    float eps, sol_dtype dtype,
+                                    sol_stream_t stream);
+
+/*
  * First-Block-Cache change detector (Sol Video Inference Engine MiniMax-H3
  * page, cross-step caching paragraph: the first block's residual is compared
  * with the previous denoising step's, and the remaining blocks are skipped
@@ -313,7 +396,10 @@ size_t sol_residual_change_workspace_bytes(int64_t B);
  *
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  Every call shares the one array and it keeps
+ * before any stream capture.  The address is kept for the life of the
+ * process: a cudaDeviceReset of that device makes it stale (the library may
+ * be loaded again elsewhere in device memory), so do not call this entry
+ * point on a device after resetting it; use sol_residual_change there.  Every call shares the one array and it keeps
  * the last call's contents; each call rewrites every slot it later reads,
  * so nothing needs clearing, but calls whose kernels overlap on the GPU
  * (different streams, or different host threads on one device) race on it:
@@ -365,7 +451,8 @@ const char *sol_last_error(void);
 
 /* ABI version, (major << 16) | minor.  2.0: sol_qk_layout gained
  * per_axis_freq, reserved, v_out and v_scale (a larger struct; callers built
- * against 1.x must be rebuilt). */
+ * against 1.x must be rebuilt).  2.1: the rotary table (sol_rope_table,
+ * sol_qknorm_rope3d_tab, sol_qknorm_rope3d_ex_tab). */
 int sol_version(void);
 
 #ifdef __cplusplus

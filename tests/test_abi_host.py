@@ -21,7 +21,8 @@ def test_header_declares_the_entry_points():
     for name in ("sol_rms_adaln", "sol_gate_residual", "sol_qknorm_rope3d",
                  "sol_gate_residual_rms_adaln", "sol_residual_change",
                  "sol_residual_change_workspace_bytes", "sol_qknorm_rope3d_ex",
-                 "sol_residual_change_noalloc",
+                 "sol_residual_change_noalloc", "sol_rope_table_bytes",
+                 "sol_rope_table_build", "sol_qknorm_rope3d_tab", "sol_qknorm_rope3d_ex_tab",
                  "sol_status_string", "sol_last_error", "sol_version"):
         assert name in syms
 
@@ -41,6 +42,7 @@ def test_status_strings_and_version():
     assert _abi.status_string(_abi.SOL_ERR_MISALIGNED) == "SOL_ERR_MISALIGNED"
     assert _abi.status_string(99) == "SOL_ERR_UNKNOWN"
     assert _abi.sol_version() >> 16 == 2  # sol_qk_layout grew in 2.0
+    assert _abi.sol_version() & 0xFFFF >= 1  # 2.1: the rotary table entry points
 
 
 # Fake device addresses: validation must reject these calls on the host.
@@ -277,6 +279,98 @@ def test_qknorm_rope3d_ex_null_layout():
                                      None) == _abi.SOL_ERR_INVALID_ARG
 
 
+# a fake table address far from every other fake buffer
+TB = A + (8 << 30)
+
+
+def table(data=TB, n_pos=8, hd=128, secs=(16, 24, 24), theta=1e4, per_axis=0):
+    return _abi.RopeTable(data, n_pos, hd, *secs, theta, per_axis)
+
+
+def test_rope_table_bytes():
+    assert _abi.sol_rope_table_bytes(4680, 128) == 4680 * 128 * 4
+    assert _abi.sol_rope_table_bytes(0, 128) == 0
+    for n, hd in ((-1, 128), (10, 127), (10, 0), (10, 258), (1 << 31, 128)):
+        assert _abi.sol_rope_table_bytes(n, hd) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(data=None), _abi.SOL_ERR_INVALID_ARG),
+    (dict(data=TB + 4), _abi.SOL_ERR_MISALIGNED),
+    (dict(n_pos=-1), _abi.SOL_ERR_INVALID_ARG),
+    (dict(hd=127, secs=(16, 24, 23)), _abi.SOL_ERR_INVALID_ARG),
+    (dict(hd=258, secs=(43, 43, 43)), _abi.SOL_ERR_INVALID_ARG),
+    (dict(secs=(16, 24, 25)), _abi.SOL_ERR_INVALID_ARG),
+    (dict(theta=0.0), _abi.SOL_ERR_INVALID_ARG),
+    (dict(theta=float("nan")), _abi.SOL_ERR_INVALID_ARG),
+    (dict(per_axis=2), _abi.SOL_ERR_INVALID_ARG),
+])
+def test_rope_table_build_rejects(kw, status):
+    assert _abi.sol_rope_table_build(table(**kw), None) == status
+
+
+def test_rope_table_build_null_and_empty():
+    assert _abi.sol_rope_table_build(None, None) == _abi.SOL_ERR_INVALID_ARG
+    assert _abi.sol_rope_table_build(table(n_pos=0), None) == _abi.SOL_OK
+
+
+def qktab(tab=None, qkv=A, ldq=768, qo=A + (1 << 30), ko=A + (2 << 30), ldo=256, B=1, T=2,
+          H=4, W=6, na=8, nh=2, dt=BF):
+    tab = table() if tab is None else tab
+    return _abi.sol_qknorm_rope3d_tab(qkv, ldq, qo, ko, ldo, None, None, tab, B, T, H, W, na,
+                                      nh, 1e-6, dt, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(tab=table(n_pos=7)), _abi.SOL_ERR_INVALID_ARG),     # needs max(T, H, W, na) = 8
+    (dict(tab=table(data=None)), _abi.SOL_ERR_INVALID_ARG),
+    (dict(tab=table(data=TB + 8)), _abi.SOL_ERR_MISALIGNED),
+    (dict(tab=table(secs=(16, 24, 25))), _abi.SOL_ERR_INVALID_ARG),
+    (dict(tab=table(data=A + (1 << 30) + 4096)), _abi.SOL_ERR_INVALID_ARG),  # table under q_out
+    (dict(tab=table(data=A + (2 << 30))), _abi.SOL_ERR_INVALID_ARG),         # ... under k_out
+    (dict(qkv=None), _abi.SOL_ERR_INVALID_ARG),                # the usual checks still apply
+    (dict(ldo=200), _abi.SOL_ERR_INVALID_ARG),
+    (dict(qo=A + 512), _abi.SOL_ERR_INVALID_ARG),
+    (dict(T=1, H=1 << 16, W=1 << 16, na=0), _abi.SOL_ERR_UNSUPPORTED),
+])
+def test_qknorm_rope3d_tab_rejects(kw, status):
+    assert qktab(**kw) == status
+
+
+def test_qknorm_rope3d_tab_positions_needed():
+    # video-only calls need max(T, H, W) rows, audio-only calls n_audio rows
+    assert qktab(tab=table(n_pos=4), T=3, H=5, W=4, na=0) == _abi.SOL_ERR_INVALID_ARG
+    assert qktab(tab=table(n_pos=10), T=0, H=0, W=0, na=11) == _abi.SOL_ERR_INVALID_ARG
+    assert "positions" in _abi.last_error()
+    # zero rows: nothing to check against the table's size
+    assert qktab(tab=table(n_pos=0), B=0) == _abi.SOL_OK
+
+
+def qkextab(tab=None, per_axis=0, int8=0, qs=None, ks=None, **kw):
+    tab = table() if tab is None else tab
+    L = 2 * 4 * 6 + 8
+    nh, hd = 8, 128
+    lay = _abi.QkLayout(L * nh * hd, nh * hd, hd, 0, int8, qs, ks, per_axis, 0, None, None)
+    return _abi.sol_qknorm_rope3d_ex_tab(A, 3 * 1024, A + (1 << 30), A + (2 << 30), lay, None,
+                                         None, tab, 1, 2, 4, 6, 8, nh, 1e-6, BF, None)
+
+
+def test_qknorm_rope3d_ex_tab_rejects():
+    # the layout's frequency rule must be the table's
+    assert qkextab(per_axis=1) == _abi.SOL_ERR_INVALID_ARG
+    assert "per_axis_freq" in _abi.last_error()
+    assert qkextab(tab=table(per_axis=1)) == _abi.SOL_ERR_INVALID_ARG
+    assert qkextab(tab=table(n_pos=7)) == _abi.SOL_ERR_INVALID_ARG
+    # a scale array over the table
+    assert qkextab(int8=1, qs=TB + 256, ks=Q8S) == _abi.SOL_ERR_INVALID_ARG
+    assert _abi.sol_qknorm_rope3d_ex_tab(A, 3 * 1024, A + (1 << 30), A + (2 << 30), None, None,
+                                         None, table(), 1, 2, 4, 6, 8, 8, 1e-6, BF,
+                                         None) == _abi.SOL_ERR_INVALID_ARG
+    assert _abi.sol_qknorm_rope3d_ex_tab(A, 3 * 1024, A + (1 << 30), A + (2 << 30), None, None,
+                                         None, None, 1, 2, 4, 6, 8, 8, 1e-6, BF,
+                                         None) == _abi.SOL_ERR_INVALID_ARG
+
+
 C_CLIENT = r"""
 #include <stdio.h>
 #include <string.h>
@@ -323,3 +417,25 @@ def test_header_is_plain_c_and_the_library_links_from_c(tmp_path):
     p = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert p.returncode == 0, (p.returncode, p.stdout, p.stderr)
     assert "layout.reserved must be 0" in p.stdout
+
+
+def test_cutlass_tree_is_explicit(monkeypatch, tmp_path):
+    # the GEMM + GELU kernel names its CUTLASS tree: SOL_CUTLASS_DIR when set,
+    # else the copy vendored in flashinfer; a missing or old tree fails with
+    # the path in the message
+    from video_diffusion_transformer_rms_b200 import build as b
+    root, ver = b.cutlass_info()
+    assert tuple(int(x) for x in ver.split("."))[:2] >= b.CUTLASS_MIN
+    monkeypatch.setenv("SOL_CUTLASS_DIR", str(tmp_path))
+    with pytest.raises(RuntimeError, match="SOL_CUTLASS_DIR"):
+        b.cutlass_info()
+    inc = tmp_path / "include"
+    (inc / "cute").mkdir(parents=True)
+    (inc / "cutlass").mkdir()
+    (inc / "cutlass" / "version.h").write_text(
+        "#define CUTLASS_MAJOR 4\n#define CUTLASS_MINOR 5\n#define CUTLASS_PATCH 1\n")
+    assert b.cutlass_info() == (str(tmp_path), "4.5.1")
+    (inc / "cutlass" / "version.h").write_text(
+        "#define CUTLASS_MAJOR 3\n#define CUTLASS_MINOR 5\n#define CUTLASS_PATCH 0\n")
+    with pytest.raises(RuntimeError, match="version"):
+        b.cutlass_info()

@@ -387,13 +387,29 @@ def _qk_oracle(qkv2, w_like, gq, gk, ids=None):
                                 gamma_q=gq, gamma_k=gk, row_ids=ids)
 
 
+def _table(use, T, H, W, na, hd, secs=(16, 24, 24), theta=1e4, per_axis=False):
+    """The rotary table of the table-driven entry points (sol_qknorm_rope3d_tab,
+    sol_qknorm_rope3d_ex_tab) covering a call's positions, or None for the
+    on-the-fly ones."""
+    if not use:
+        return None
+    return api.RopeTable.for_grid(T, H, W, na, hd, sections=secs, theta=theta,
+                                  per_axis_freq=per_axis, device=DEV)
+
+
+ROPE = pytest.mark.parametrize("tab", [False, True], ids=["otf", "table"])
+
+
 @pytest.mark.parametrize("name", SMALL + LARGE)
-def test_qknorm_rope3d_workload(name):
+@ROPE
+def test_qknorm_rope3d_workload(name, tab):
     w = WORKLOADS[name]
     t = make_inputs(w, DEV, which=("qknorm_rope3d",))
     qkv = t["qkv"].view(w.B, w.L, 3 * w.D)
     q, k = api.qknorm_rope3d(qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim,
-                             w.sections, t["gamma_q"], t["gamma_k"], w.eps, w.theta)
+                             w.sections, t["gamma_q"], t["gamma_k"], w.eps, w.theta,
+                             table=_table(tab, w.T, w.H, w.W, w.n_audio, w.head_dim, w.sections,
+                                          w.theta))
     torch.cuda.synchronize()
     spec = (w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections, w.eps, w.theta)
     q2, k2 = q.reshape(-1, w.D), k.reshape(-1, w.D)
@@ -431,7 +447,8 @@ QK_CASES = [
 
 
 @pytest.mark.parametrize("B,T,H,W,na,nh,hd,secs,dt,pad", QK_CASES)
-def test_qknorm_rope3d_cases(B, T, H, W, na, nh, hd, secs, dt, pad):
+@ROPE
+def test_qknorm_rope3d_cases(B, T, H, W, na, nh, hd, secs, dt, pad, tab):
     D = nh * hd
     L = T * H * W + na
     C = 3 * D + pad
@@ -439,8 +456,9 @@ def test_qknorm_rope3d_cases(B, T, H, W, na, nh, hd, secs, dt, pad):
     gq = vectors((hd,), 1.0, 0.1, dt, DEV, 32)
     gk = vectors((hd,), 1.0, 0.1, dt, DEV, 33)
     spec = (T, H, W, na, nh, hd, secs, 1e-6, 1e4)
+    table = _table(tab, T, H, W, na, hd, secs)
     for gam in ((gq, gk), (None, None)):
-        q, k = api.qknorm_rope3d(qkv, T, H, W, na, nh, hd, secs, gam[0], gam[1])
+        q, k = api.qknorm_rope3d(qkv, T, H, W, na, nh, hd, secs, gam[0], gam[1], table=table)
         wq, wk = _qk_oracle(_o(qkv.view(B * L, C)), spec,
                             None if gam[0] is None else _o(gq),
                             None if gam[1] is None else _o(gk))
@@ -448,13 +466,16 @@ def test_qknorm_rope3d_cases(B, T, H, W, na, nh, hd, secs, dt, pad):
         assert_close(k.reshape(-1, D), wk, "k")
 
 
-def test_qknorm_rope3d_layouts_and_v_untouched():
+@ROPE
+def test_qknorm_rope3d_layouts_and_v_untouched(tab):
     w = WORKLOADS["medium"]
     D = w.D
     t = make_inputs(w, DEV, which=("qknorm_rope3d",))
     qkv = t["qkv"].view(w.B, w.L, 3 * D)
     args = (w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections, t["gamma_q"],
             t["gamma_k"])
+    table = _table(tab, w.T, w.H, w.W, w.n_audio, w.head_dim)
+    kw = {"table": table}
     spec = (w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections, w.eps, w.theta)
     ids = sample_rows(w.rows, w.L, w.n_video, w.B, 1500, seed=5)
     wq, wk = _qk_oracle(take_rows(qkv.view(-1, 3 * D)[:, :2 * D], ids), spec,
@@ -462,13 +483,13 @@ def test_qknorm_rope3d_layouts_and_v_untouched():
     # separate q and k tensors (ld_out = D)
     qo = torch.empty((w.B, w.L, D), dtype=qkv.dtype, device=DEV)
     ko = torch.empty_like(qo)
-    api.qknorm_rope3d(qkv, *args, q_out=qo, k_out=ko)
+    api.qknorm_rope3d(qkv, *args, q_out=qo, k_out=ko, **kw)
     assert_close(take_rows_gpu(qo.view(-1, D), ids), wq, "q separate")
     assert_close(take_rows_gpu(ko.view(-1, D), ids), wk, "k separate")
     # in place, v columns untouched
     qi = qkv.clone()
     v_before = qi[..., 2 * D:].clone()
-    api.qknorm_rope3d(qi, *args, q_out=qi[..., :D], k_out=qi[..., D:2 * D])
+    api.qknorm_rope3d(qi, *args, q_out=qi[..., :D], k_out=qi[..., D:2 * D], **kw)
     torch.cuda.synchronize()
     assert torch.equal(qi[..., 2 * D:], v_before)
     assert_close(take_rows_gpu(qi.view(-1, 3 * D)[:, :D], ids), wq, "q in place")
@@ -478,18 +499,19 @@ def test_qknorm_rope3d_layouts_and_v_untouched():
     n = w.rows * 2 * D
     buf = torch.full((n + 2 * pad,), 1.5, dtype=qkv.dtype, device=DEV)
     o = buf[pad:pad + n].view(w.B, w.L, 2 * D)
-    api.qknorm_rope3d(qkv, *args, q_out=o[..., :D], k_out=o[..., D:])
+    api.qknorm_rope3d(qkv, *args, q_out=o[..., :D], k_out=o[..., D:], **kw)
     torch.cuda.synchronize()
     assert torch.all(buf[:pad] == 1.5) and torch.all(buf[-pad:] == 1.5)
     assert_close(take_rows_gpu(o.view(-1, 2 * D)[:, :D], ids), wq, "q guarded")
 
 
-def test_qknorm_rope3d_large_positions_are_accurate():
+@ROPE
+def test_qknorm_rope3d_large_positions_are_accurate(tab):
     # audio positions up to 4679 (15 s clip): angles reach thousands of radians
     B, T, H, W, na, nh, hd = 1, 0, 0, 0, 4680, 4, 128
     L = na
     qkv = activation(L, 3 * nh * hd, torch.bfloat16, DEV, 77, outliers=False).view(1, L, -1)
-    q, k = api.qknorm_rope3d(qkv, T, H, W, na, nh, hd)
+    q, k = api.qknorm_rope3d(qkv, T, H, W, na, nh, hd, table=_table(tab, T, H, W, na, hd))
     ids = np.arange(L - 300, L)
     wq, wk = oracle.qknorm_rope3d(take_rows(qkv.view(L, -1), ids), T, H, W, na, nh, hd,
                                   (16, 24, 24), 1e-6, 1e4, row_ids=ids)
@@ -527,13 +549,15 @@ def _check_int8(codes, scales, want, n_heads, hd, what):
 @pytest.mark.parametrize("half", [False, True])
 @pytest.mark.parametrize("layout", ["bshd", "bhsd"])
 @pytest.mark.parametrize("int8", [False, True])
-def test_qknorm_rope3d_ex_workload(name, half, layout, int8):
+@ROPE
+def test_qknorm_rope3d_ex_workload(name, half, layout, int8, tab):
     w = WORKLOADS[name]
     t = make_inputs(w, DEV, which=("qknorm_rope3d",))
     qkv = t["qkv"].view(w.B, w.L, 3 * w.D)
     res = api.qknorm_rope3d_ex(qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim,
                                w.sections, t["gamma_q"], t["gamma_k"], w.eps, w.theta,
-                               layout=layout, half_split=half, int8=int8)
+                               layout=layout, half_split=half, int8=int8,
+                               table=_table(tab, w.T, w.H, w.W, w.n_audio, w.head_dim))
     torch.cuda.synchronize()
     q, k = (_bshd(r, layout).reshape(w.rows, w.D) for r in res[:2])
     ids = None if name == "medium" else _ids(w, 512)
@@ -544,7 +568,7 @@ def test_qknorm_rope3d_ex_workload(name, half, layout, int8):
                                      _o(t["gamma_k"]), row_ids=ids)
     if ids is not None:
         q, k = take_rows_gpu(q, ids), take_rows_gpu(k, ids)
-    tag = f"ex[{name} half={half} {layout} int8={int8}]"
+    tag = f"ex[{name} half={half} {layout} int8={int8} table={tab}]"
     if int8:
         qs, ks = (r.reshape(w.rows, w.n_heads) for r in res[2:])
         if ids is not None:
@@ -559,14 +583,17 @@ def test_qknorm_rope3d_ex_workload(name, half, layout, int8):
 @pytest.mark.parametrize("name", ("medium", "clip5s"))
 @pytest.mark.parametrize("half", [False, True])
 @pytest.mark.parametrize("int8", [False, True])
-def test_qknorm_rope3d_ex_per_axis_freq(name, half, int8):
+@ROPE
+def test_qknorm_rope3d_ex_per_axis_freq(name, half, int8, tab):
     # each rotary section with a frequency ladder of its own, theta^(-j/s)
     w = WORKLOADS[name]
     t = make_inputs(w, DEV, which=("qknorm_rope3d",))
     qkv = t["qkv"].view(w.B, w.L, 3 * w.D)
     res = api.qknorm_rope3d_ex(qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim,
                                w.sections, t["gamma_q"], t["gamma_k"], w.eps, w.theta,
-                               layout="bhsd", half_split=half, int8=int8, per_axis_freq=True)
+                               layout="bhsd", half_split=half, int8=int8, per_axis_freq=True,
+                               table=_table(tab, w.T, w.H, w.W, w.n_audio, w.head_dim,
+                                            per_axis=True))
     torch.cuda.synchronize()
     q, k = (_bshd(r, "bhsd").reshape(w.rows, w.D) for r in res[:2])
     ids = None if name == "medium" else _ids(w, 384)
@@ -577,7 +604,7 @@ def test_qknorm_rope3d_ex_per_axis_freq(name, half, int8):
                                      _o(t["gamma_k"]), row_ids=ids, per_axis=True)
     if ids is not None:
         q, k = take_rows_gpu(q, ids), take_rows_gpu(k, ids)
-    tag = f"per-axis[{name} half={half} int8={int8}]"
+    tag = f"per-axis[{name} half={half} int8={int8} table={tab}]"
     if int8:
         qs, ks = (r.reshape(w.rows, w.n_heads) for r in res[2:4])
         if ids is not None:
@@ -617,8 +644,10 @@ def test_qknorm_rope3d_ex_quantized_v(name, layout):
     assert torch.equal(qs, qs2) and torch.equal(ks, ks2)
 
 
-@pytest.mark.parametrize("secs", [(64, 0, 0), (0, 32, 32), (20, 0, 44), (16, 24, 24)])
-def test_qknorm_rope3d_ex_per_axis_sections(secs):
+@pytest.mark.parametrize("secs", [(64, 0, 0), (0, 32, 32), (20, 0, 44), (16, 24, 24),
+                                  (18, 22, 24)])
+@ROPE
+def test_qknorm_rope3d_ex_per_axis_sections(secs, tab):
     # per-axis ladders with empty and uneven sections (an empty section holds
     # no pair, so its size never divides)
     B, T, H, W, na, nh, hd = 1, 4, 6, 5, 9, 4, 128
@@ -627,9 +656,10 @@ def test_qknorm_rope3d_ex_per_axis_sections(secs):
     qkv = activation(B * L, 3 * D, torch.bfloat16, DEV, 81, outliers=True).view(B, L, 3 * D)
     gq = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 82)
     gk = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 83)
+    table = _table(tab, T, H, W, na, hd, secs, per_axis=True)
     for half in (False, True):
         q, k = api.qknorm_rope3d_ex(qkv, T, H, W, na, nh, hd, secs, gq, gk, half_split=half,
-                                    per_axis_freq=True)
+                                    per_axis_freq=True, table=table)
         wq, wk = oracle.qknorm_rope3d_ex(_o(qkv.view(B * L, 3 * D)), T, H, W, na, nh, hd, secs,
                                          1e-6, 1e4, half, _o(gq), _o(gk), per_axis=True)
         assert_close(q.reshape(B * L, D), wq, f"per-axis sections {secs} half={half} q")
@@ -655,17 +685,19 @@ def test_qknorm_rope3d_packed_qk_input():
         assert all(torch.equal(a, b) for a, b in zip(r0, r1))
 
 
-def test_qknorm_rope3d_ex_interleaved_matches_default_entry_point():
-    # same arithmetic as sol_qknorm_rope3d, only the addressing differs:
-    # bit-identical results in both layouts
+@ROPE
+def test_qknorm_rope3d_ex_interleaved_matches_default_entry_point(tab):
+    # same arithmetic as sol_qknorm_rope3d (sol_qknorm_rope3d_tab), only the
+    # addressing differs: bit-identical results in both layouts
     w = WORKLOADS["medium"]
     t = make_inputs(w, DEV, which=("qknorm_rope3d",))
     qkv = t["qkv"].view(w.B, w.L, 3 * w.D)
     args = (w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections, t["gamma_q"],
             t["gamma_k"], w.eps, w.theta)
-    q0, k0 = api.qknorm_rope3d(qkv, *args)
+    table = _table(tab, w.T, w.H, w.W, w.n_audio, w.head_dim)
+    q0, k0 = api.qknorm_rope3d(qkv, *args, table=table)
     for layout in ("bshd", "bhsd"):
-        q1, k1 = api.qknorm_rope3d_ex(qkv, *args, layout=layout)
+        q1, k1 = api.qknorm_rope3d_ex(qkv, *args, layout=layout, table=table)
         assert torch.equal(_bshd(q1, layout).reshape(q0.shape), q0)
         assert torch.equal(_bshd(k1, layout).reshape(k0.shape), k0)
 
@@ -673,7 +705,8 @@ def test_qknorm_rope3d_ex_interleaved_matches_default_entry_point():
 @pytest.mark.parametrize("hd,secs", [(64, (8, 12, 12)), (256, (32, 48, 48))])
 @pytest.mark.parametrize("half", [False, True])
 @pytest.mark.parametrize("per_axis", [False, True])
-def test_qknorm_rope3d_ex_head_dims(hd, secs, half, per_axis):
+@ROPE
+def test_qknorm_rope3d_ex_head_dims(hd, secs, half, per_axis, tab):
     B, T, H, W, na, nh = 2, 3, 5, 7, 11, 6
     L = T * H * W + na
     D = nh * hd
@@ -682,11 +715,12 @@ def test_qknorm_rope3d_ex_head_dims(hd, secs, half, per_axis):
     gk = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 63)
     wq, wk = oracle.qknorm_rope3d_ex(_o(qkv.view(B * L, 3 * D)), T, H, W, na, nh, hd, secs,
                                      1e-6, 1e4, half, _o(gq), _o(gk), per_axis=per_axis)
-    tag = f"hd={hd} half={half} per_axis={per_axis}"
+    tag = f"hd={hd} half={half} per_axis={per_axis} table={tab}"
+    table = _table(tab, T, H, W, na, hd, secs, per_axis=per_axis)
     for int8 in (False, True):
         res = api.qknorm_rope3d_ex(qkv, T, H, W, na, nh, hd, secs, gq, gk, layout="bhsd",
                                    half_split=half, int8=int8, per_axis_freq=per_axis,
-                                   quantize_v=int8)
+                                   quantize_v=int8, table=table)
         q, k = (_bshd(r, "bhsd").reshape(B * L, D) for r in res[:2])
         if int8:
             _check_int8(q, res[2], wq, nh, hd, tag + " q")
@@ -744,7 +778,8 @@ def test_gemm_gelu_clip_mlp_shape_sampled():
 
 
 @pytest.mark.parametrize("half", [False, True])
-def test_qknorm_rope3d_ex_int8_edge_heads(half):
+@ROPE
+def test_qknorm_rope3d_ex_int8_edge_heads(half, tab):
     # per row: a normal head, an all-zero head, a head of tiny normal values
     # (x * 2^-110, so max|u| < 2^-96 and the kernel rescales before dividing),
     # and a head with one 1e4 outlier; q, k and v get different heads
@@ -761,7 +796,8 @@ def test_qknorm_rope3d_ex_int8_edge_heads(half):
     gq = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 72)
     gk = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 73)
     res = api.qknorm_rope3d_ex(qkv, T, H, W, na, nh, hd, (16, 24, 24), gq, gk, layout="bshd",
-                               half_split=half, int8=True, quantize_v=True)
+                               half_split=half, int8=True, quantize_v=True,
+                               table=_table(tab, T, H, W, na, hd))
     torch.cuda.synchronize()
     wq, wk = oracle.qknorm_rope3d_ex(_o(qkv.view(L, 3 * D)), T, H, W, na, nh, hd, (16, 24, 24),
                                      1e-6, 1e4, half, _o(gq), _o(gk))
@@ -777,3 +813,79 @@ def test_qknorm_rope3d_ex_int8_edge_heads(half):
     assert torch.all(ks.view(L, nh)[:, 2] == 0) and torch.all(k.view(L, nh, hd)[:, 2] == 0)
     # the tiny heads use the full code range
     assert int(q.view(L, nh, hd)[:, 2].abs().amax()) == 127
+
+
+# ----------------------------------------------------------------------------
+# Rotary table (sol_rope_table_build) and the table-driven entry points
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("hd,secs,per_axis", [(128, (16, 24, 24), False),
+                                              (128, (16, 24, 24), True),
+                                              (64, (8, 12, 12), True), (16, (2, 3, 3), False)])
+def test_rope_table_entries(hd, secs, per_axis):
+    # row p: cos(p f_i) for every pair i, then sin(p f_i); each entry the fp64
+    # value rounded once to fp32 (within half an fp32 ulp, plus the fp64
+    # sincos error)
+    n_pos = 4680
+    tab = api.RopeTable(n_pos, hd, secs, 1e4, per_axis, device=DEV)
+    got = tab.data.view(n_pos, hd).double().cpu().numpy()
+    npairs = hd // 2
+    i = np.arange(npairs)
+    if per_axis:
+        start = np.concatenate([np.full(s, sum(secs[:a])) for a, s in enumerate(secs)])
+        size = np.concatenate([np.full(s, s) for s in secs])
+        f = 1e4 ** (-(i - start) / size)
+    else:
+        f = 1e4 ** (-2.0 * i / hd)
+    ang = np.arange(n_pos, dtype=np.float64)[:, None] * f[None, :]
+    want = np.concatenate([np.cos(ang), np.sin(ang)], axis=1)
+    err = np.abs(got - want)
+    assert err.max() <= 2.0 ** -24 * 1.01 + 1e-15, err.max()
+
+
+def test_rope_table_zero_positions_and_reuse():
+    # n_pos = 0 is a no-op build; a table is reused across calls and samples
+    tab0 = api.RopeTable(0, 128, device=DEV)
+    assert tab0.n_pos == 0
+    w = WORKLOADS["medium"]
+    t = make_inputs(w, DEV, which=("qknorm_rope3d",))
+    qkv = t["qkv"].view(w.B, w.L, 3 * w.D)
+    table = _table(True, w.T, w.H, w.W, w.n_audio, w.head_dim)
+    args = (w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections, t["gamma_q"],
+            t["gamma_k"], w.eps, w.theta)
+    q0, k0 = api.qknorm_rope3d(qkv, *args, table=table)
+    q1, k1 = api.qknorm_rope3d(qkv, *args, table=table)
+    assert torch.equal(q0, q1) and torch.equal(k0, k1)
+    # the table path differs from the on-the-fly one only by the rounding of
+    # (cos, sin): at most a bf16 ulp or two of the output, on few elements
+    q2, _ = api.qknorm_rope3d(qkv, *args)
+    d = (q2.float() - q0.float()).abs()
+    assert float(d.max()) <= 2.0 ** -6 * float(q0.float().abs().max())
+    assert float((d > 0).float().mean()) < 0.05
+
+
+def test_rope_table_too_small_or_overlapping_is_rejected():
+    # the host refuses a table with too few positions, or an output over the
+    # table, before launching anything
+    T, H, W, na, nh, hd = 2, 3, 4, 5, 2, 128
+    L = T * H * W + na
+    D = nh * hd
+    qkv = activation(L, 3 * D, torch.bfloat16, DEV, 91, outliers=False).view(1, L, 3 * D)
+    small = api.RopeTable(4, hd, device=DEV)   # needs max(T, H, W, na) = 5
+    with pytest.raises(_abi.SolError, match="positions"):
+        api.qknorm_rope3d(qkv, T, H, W, na, nh, hd, table=small)
+    ok = api.RopeTable(5, hd, device=DEV)
+    api.qknorm_rope3d(qkv, T, H, W, na, nh, hd, table=ok)
+    # an output that overlaps the table
+    big = api.RopeTable(2 * L * D // hd + 8, hd, device=DEV)
+    before = big.data.clone()
+    out = big.data.view(torch.bfloat16)[:L * 2 * D].view(1, L, 2 * D)
+    with pytest.raises(_abi.SolError, match="table"):
+        api.qknorm_rope3d(qkv, T, H, W, na, nh, hd, table=big, q_out=out[..., :D],
+                          k_out=out[..., D:])
+    torch.cuda.synchronize()
+    assert torch.equal(big.data, before)
+    # per-axis flag of the layout and the table must agree
+    pa = api.RopeTable(5, hd, per_axis_freq=True, device=DEV)
+    with pytest.raises(ValueError):
+        api.qknorm_rope3d_ex(qkv, T, H, W, na, nh, hd, table=pa)

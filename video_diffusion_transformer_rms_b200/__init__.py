@@ -11,7 +11,8 @@ path.
 """
 from ._abi import (SOL_BF16, SOL_F32, SolError, sol_gate_residual,  # noqa: F401
                    sol_gate_residual_rms_adaln, sol_last_error, sol_qknorm_rope3d,
-                   sol_qknorm_rope3d_ex,
+                   sol_qknorm_rope3d_ex, sol_qknorm_rope3d_ex_tab, sol_qknorm_rope3d_tab,
+                   sol_rope_table_build, sol_rope_table_bytes,
                    sol_residual_change, sol_residual_change_workspace_bytes,
                    sol_rms_adaln, sol_status_string, sol_version)
 

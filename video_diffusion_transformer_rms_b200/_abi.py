@@ -34,6 +34,15 @@ class QkLayout(ctypes.Structure):
                 ("v_scale", ctypes.c_void_p)]
 
 
+class RopeTable(ctypes.Structure):
+    """sol_rope_table of include/sol.h: a rotary table's device buffer and the
+    fields it was (or will be) built from."""
+    _fields_ = [("data", ctypes.c_void_p), ("n_pos", ctypes.c_int64),
+                ("head_dim", ctypes.c_int64), ("sec_t", ctypes.c_int64),
+                ("sec_h", ctypes.c_int64), ("sec_w", ctypes.c_int64),
+                ("theta", ctypes.c_float), ("per_axis_freq", ctypes.c_int32)]
+
+
 _lock = threading.Lock()
 _lib = None
 
@@ -82,6 +91,17 @@ def lib() -> ctypes.CDLL:
         L.sol_qknorm_rope3d.argtypes = [p, i64, p, p, i64, p, p, i64, i64, i64, i64, i64,
                                         i64, i64, i64, i64, i64, f, f, i, p]
         L.sol_qknorm_rope3d.restype = i
+        L.sol_rope_table_bytes.argtypes = [i64, i64]
+        L.sol_rope_table_bytes.restype = ctypes.c_size_t
+        L.sol_rope_table_build.argtypes = [ctypes.POINTER(RopeTable), p]
+        L.sol_rope_table_build.restype = i
+        L.sol_qknorm_rope3d_tab.argtypes = [p, i64, p, p, i64, p, p, ctypes.POINTER(RopeTable),
+                                            i64, i64, i64, i64, i64, i64, f, i, p]
+        L.sol_qknorm_rope3d_tab.restype = i
+        L.sol_qknorm_rope3d_ex_tab.argtypes = [p, i64, p, p, ctypes.POINTER(QkLayout), p, p,
+                                               ctypes.POINTER(RopeTable), i64, i64, i64, i64,
+                                               i64, i64, f, i, p]
+        L.sol_qknorm_rope3d_ex_tab.restype = i
         L.sol_status_string.argtypes = [i]
         L.sol_status_string.restype = ctypes.c_char_p
         L.sol_last_error.argtypes = []
@@ -158,6 +178,33 @@ def sol_qknorm_rope3d_ex(qkv, ld_qkv, q_out, k_out, layout, gamma_q, gamma_k, B,
     return lib().sol_qknorm_rope3d_ex(qkv, ld_qkv, q_out, k_out, ref, gamma_q, gamma_k, B, T,
                                       H, W, n_audio, n_heads, head_dim, sec_t, sec_h, sec_w,
                                       eps, theta, dtype, stream)
+
+
+def _ref(x):
+    return ctypes.byref(x) if x is not None else None
+
+
+def sol_rope_table_bytes(n_pos, head_dim) -> int:
+    return lib().sol_rope_table_bytes(n_pos, head_dim)
+
+
+def sol_rope_table_build(tab, stream) -> int:
+    """tab: a RopeTable (or None, which the library rejects)."""
+    return lib().sol_rope_table_build(_ref(tab), stream)
+
+
+def sol_qknorm_rope3d_tab(qkv, ld_qkv, q_out, k_out, ld_out, gamma_q, gamma_k, tab, B, T, H, W,
+                          n_audio, n_heads, eps, dtype, stream) -> int:
+    return lib().sol_qknorm_rope3d_tab(qkv, ld_qkv, q_out, k_out, ld_out, gamma_q, gamma_k,
+                                       _ref(tab), B, T, H, W, n_audio, n_heads, eps, dtype,
+                                       stream)
+
+
+def sol_qknorm_rope3d_ex_tab(qkv, ld_qkv, q_out, k_out, layout, gamma_q, gamma_k, tab, B, T, H,
+                             W, n_audio, n_heads, eps, dtype, stream) -> int:
+    return lib().sol_qknorm_rope3d_ex_tab(qkv, ld_qkv, q_out, k_out, _ref(layout), gamma_q,
+                                          gamma_k, _ref(tab), B, T, H, W, n_audio, n_heads, eps,
+                                          dtype, stream)
 
 
 def sol_gemm_gelu(A, B, bias, C, M, N, K, workspace, workspace_bytes, stream) -> int:

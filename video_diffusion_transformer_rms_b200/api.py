@@ -138,16 +138,55 @@ def residual_change(cur: torch.Tensor, prev: torch.Tensor,
     return o
 
 
+class RopeTable:
+    """A rotary table on the device (sol_rope_table): row p holds cos(p*f_i)
+    for every rotary pair i, then sin(p*f_i), fp32, for positions
+    0 .. n_pos-1.  Build it once per video shape; pass it as `table=` to
+    qknorm_rope3d / qknorm_rope3d_ex."""
+
+    def __init__(self, n_pos: int, head_dim: int, sections: Sequence[int] = (16, 24, 24),
+                 theta: float = 10000.0, per_axis_freq: bool = False, device=None,
+                 stream: Optional[torch.cuda.Stream] = None):
+        nbytes = _abi.sol_rope_table_bytes(n_pos, head_dim)
+        if nbytes == 0 and n_pos != 0:
+            raise ValueError("n_pos must be >= 0 and head_dim even in [2, 256]")
+        self.data = torch.empty(max(nbytes // 4, 4), dtype=torch.float32, device=device)
+        self.n_pos, self.head_dim = n_pos, head_dim
+        self.sections = tuple(int(x) for x in sections)
+        self.theta, self.per_axis_freq = float(theta), bool(per_axis_freq)
+        st, sh, sw = self.sections
+        self.desc = _abi.RopeTable(self.data.data_ptr(), n_pos, head_dim, st, sh, sw, theta,
+                                   int(self.per_axis_freq))
+        _abi.check(_abi.sol_rope_table_build(self.desc, _stream(stream)))
+
+    @classmethod
+    def for_grid(cls, T: int, H: int, W: int, n_audio: int, head_dim: int, **kw):
+        """A table covering every position of a T x H x W video grid plus
+        n_audio audio tokens."""
+        n = max(n_audio, max(T, H, W) if T * H * W > 0 else 0)
+        return cls(n, head_dim, **kw)
+
+    def check(self, head_dim: int, sections: Sequence[int], theta: float,
+              per_axis_freq: bool = False):
+        if (head_dim != self.head_dim or tuple(sections) != self.sections
+                or float(theta) != self.theta or bool(per_axis_freq) != self.per_axis_freq):
+            raise ValueError("the rotary table was built for other head_dim, sections, theta "
+                             "or frequency rule")
+
+
 def qknorm_rope3d(qkv: torch.Tensor, T: int, H: int, W: int, n_audio: int, n_heads: int,
                   head_dim: int, sections: Sequence[int] = (16, 24, 24),
                   gamma_q: Optional[torch.Tensor] = None,
                   gamma_k: Optional[torch.Tensor] = None, eps: float = 1e-6,
                   theta: float = 10000.0, q_out: Optional[torch.Tensor] = None,
                   k_out: Optional[torch.Tensor] = None,
-                  stream: Optional[torch.cuda.Stream] = None
+                  stream: Optional[torch.cuda.Stream] = None,
+                  table: Optional[RopeTable] = None
                   ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Per-head QKNorm + 3D RoPE of q and k in a merged qkv [B, L, >=2D]
-    (row stride qkv.stride(1)); returns (q, k) as [B, L, D] views."""
+    (row stride qkv.stride(1)); returns (q, k) as [B, L, D] views.  With
+    `table` the (cos, sin) come from that rotary table (sol_qknorm_rope3d_tab)
+    instead of being computed per row."""
     if qkv.dim() != 3 or qkv.stride(2) != 1 or qkv.stride(0) != qkv.shape[1] * qkv.stride(1):
         raise ValueError("qkv must be [B, L, C] with unit column stride and packed rows")
     B, L, _ = qkv.shape
@@ -170,10 +209,19 @@ def qknorm_rope3d(qkv: torch.Tensor, T: int, H: int, W: int, n_audio: int, n_hea
             raise ValueError(f"{name} is on {t.device}, qkv on {qkv.device}")
     ld_out = q_out.stride(1)
     st, sh, sw = sections
-    _abi.check(_abi.sol_qknorm_rope3d(
-        _ptr(qkv), qkv.stride(1), _ptr(q_out), _ptr(k_out), ld_out, _ptr(gamma_q),
-        _ptr(gamma_k), B, T, H, W, n_audio, n_heads, head_dim, st, sh, sw, eps, theta,
-        _dtype(qkv, q_out, k_out, gamma_q, gamma_k), _stream(stream)))
+    dt = _dtype(qkv, q_out, k_out, gamma_q, gamma_k)
+    if table is not None:
+        table.check(head_dim, sections, theta)
+        if table.data.device != qkv.device:
+            raise ValueError(f"the rotary table is on {table.data.device}, qkv on {qkv.device}")
+        _abi.check(_abi.sol_qknorm_rope3d_tab(
+            _ptr(qkv), qkv.stride(1), _ptr(q_out), _ptr(k_out), ld_out, _ptr(gamma_q),
+            _ptr(gamma_k), table.desc, B, T, H, W, n_audio, n_heads, eps, dt, _stream(stream)))
+    else:
+        _abi.check(_abi.sol_qknorm_rope3d(
+            _ptr(qkv), qkv.stride(1), _ptr(q_out), _ptr(k_out), ld_out, _ptr(gamma_q),
+            _ptr(gamma_k), B, T, H, W, n_audio, n_heads, head_dim, st, sh, sw, eps, theta, dt,
+            _stream(stream)))
     return q_out, k_out
 
 
@@ -183,13 +231,16 @@ def qknorm_rope3d_ex(qkv: torch.Tensor, T: int, H: int, W: int, n_audio: int, n_
                      gamma_k: Optional[torch.Tensor] = None, eps: float = 1e-6,
                      theta: float = 10000.0, layout: str = "bshd", half_split: bool = False,
                      int8: bool = False, per_axis_freq: bool = False, quantize_v: bool = False,
-                     stream: Optional[torch.cuda.Stream] = None):
+                     stream: Optional[torch.cuda.Stream] = None,
+                     table: Optional[RopeTable] = None):
     """QKNorm + 3D RoPE epilogue variants (bf16 input).  layout "bshd" gives
     q, k as [B, L, H, hd]; "bhsd" as attention's [B, H, L, hd].  half_split
     pairs element i with i + hd/2; per_axis_freq gives each rotary section a
     frequency ladder of its own.  int8 returns (q, k, q_scale, k_scale): int8
     codes in the chosen layout and scales fp32 [B, L, H]; with quantize_v
-    also (v, v_scale), v quantised as it stands; else (q, k) in bf16."""
+    also (v, v_scale), v quantised as it stands; else (q, k) in bf16.  With
+    `table` the (cos, sin) come from that rotary table
+    (sol_qknorm_rope3d_ex_tab)."""
     if qkv.dim() != 3 or qkv.stride(2) != 1 or qkv.stride(0) != qkv.shape[1] * qkv.stride(1):
         raise ValueError("qkv must be [B, L, C] with unit column stride and packed rows")
     if quantize_v and not int8:
@@ -221,10 +272,18 @@ def qknorm_rope3d_ex(qkv: torch.Tensor, T: int, H: int, W: int, n_audio: int, n_
                         int(bool(int8)), _ptr(qs), _ptr(ks), int(bool(per_axis_freq)), 0,
                         _ptr(v), _ptr(vs))
     st, sh, sw = sections
-    _abi.check(_abi.sol_qknorm_rope3d_ex(
-        _ptr(qkv), qkv.stride(1), _ptr(q), _ptr(k), lay, _ptr(gamma_q), _ptr(gamma_k), B, T, H,
-        W, n_audio, n_heads, head_dim, st, sh, sw, eps, theta,
-        _dtype(qkv, gamma_q, gamma_k), _stream(stream)))
+    dt = _dtype(qkv, gamma_q, gamma_k)
+    if table is not None:
+        table.check(head_dim, sections, theta, per_axis_freq)
+        if table.data.device != qkv.device:
+            raise ValueError(f"the rotary table is on {table.data.device}, qkv on {qkv.device}")
+        _abi.check(_abi.sol_qknorm_rope3d_ex_tab(
+            _ptr(qkv), qkv.stride(1), _ptr(q), _ptr(k), lay, _ptr(gamma_q), _ptr(gamma_k),
+            table.desc, B, T, H, W, n_audio, n_heads, eps, dt, _stream(stream)))
+    else:
+        _abi.check(_abi.sol_qknorm_rope3d_ex(
+            _ptr(qkv), qkv.stride(1), _ptr(q), _ptr(k), lay, _ptr(gamma_q), _ptr(gamma_k), B, T,
+            H, W, n_audio, n_heads, head_dim, st, sh, sw, eps, theta, dt, _stream(stream)))
     if quantize_v:
         return q, k, qs, ks, v, vs
     return (q, k, qs, ks) if int8 else (q, k)

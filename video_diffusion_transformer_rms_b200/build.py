@@ -22,7 +22,7 @@ LIB = os.path.join(PKG, "libsol.so")
 
 SOURCES = ["sol_abi.cu", "rms_adaln.cu", "gate_residual.cu", "qknorm_rope3d_bf16.cu",
            "qknorm_rope3d_f32.cu", "qknorm_rope3d_ex_bf16.cu", "qknorm_rope3d_ex_int8.cu",
-           "residual_change.cu", "quantize_heads.cu", "gemm_gelu.cu"]
+           "residual_change.cu", "quantize_heads.cu", "rope_table.cu", "gemm_gelu.cu"]
 # sources built against the CUTLASS / CuTe headers (the sm100 GEMM templates)
 CUTLASS_SOURCES = {"gemm_gelu.cu"}
 HEADERS = ["sol_device.cuh", "sol_launch.h", "qknorm_rope3d.cuh", "qknorm_rope3d_ex.cuh"]
@@ -39,15 +39,55 @@ def _nvcc():
     raise RuntimeError("nvcc not found: the CUDA toolkit is required to build libsol")
 
 
+# The GEMM + GELU kernel is assembled from CUTLASS's sm100 collective
+# templates (CTA-pair tcgen05 MMA, TMA, TMEM); it was built and measured with
+# CUTLASS 4.5.0.  Older trees lack parts of the sm100 builders it uses.
+CUTLASS_MIN = (4, 0)
+
+
+def _cutlass_version(root):
+    """(major, minor, patch) from include/cutlass/version.h, or None."""
+    import re
+    try:
+        with open(os.path.join(root, "include", "cutlass", "version.h")) as fh:
+            text = fh.read()
+    except OSError:
+        return None
+    v = [re.search(rf"#define CUTLASS_{k}\s+(\d+)", text) for k in ("MAJOR", "MINOR", "PATCH")]
+    return tuple(int(m.group(1)) for m in v) if all(v) else None
+
+
 def _cutlass_root():
-    """The CUTLASS tree vendored with flashinfer (headers only; no import)."""
-    import importlib.util
-    spec = importlib.util.find_spec("flashinfer")
-    for base in (spec.submodule_search_locations if spec else []) or []:
-        root = os.path.join(base, "data", "cutlass")
+    """The CUTLASS / CuTe header tree the GEMM + GELU kernel is built against:
+    $SOL_CUTLASS_DIR if set (a CUTLASS checkout: include/cute and
+    include/cutlass), else the tree vendored inside the installed flashinfer
+    package (flashinfer/data/cutlass; headers only, flashinfer is not
+    imported).  Fails with the path it looked at."""
+    env = os.environ.get("SOL_CUTLASS_DIR")
+    if env:
+        candidates, where = [env], f"SOL_CUTLASS_DIR={env}"
+    else:
+        import importlib.util
+        spec = importlib.util.find_spec("flashinfer")
+        bases = (spec.submodule_search_locations if spec else None) or []
+        candidates = [os.path.join(b, "data", "cutlass") for b in bases]
+        where = ("flashinfer/data/cutlass (" + ", ".join(candidates) + ")" if candidates
+                 else "flashinfer/data/cutlass (flashinfer is not installed)")
+    for root in candidates:
         if os.path.isdir(os.path.join(root, "include", "cute")):
+            ver = _cutlass_version(root)
+            if ver is None or ver[:2] < CUTLASS_MIN:
+                raise RuntimeError(f"CUTLASS at {root} is version {ver}; gemm_gelu.cu needs "
+                                   f">= {CUTLASS_MIN[0]}.{CUTLASS_MIN[1]} (set SOL_CUTLASS_DIR)")
             return root
-    raise RuntimeError("CUTLASS headers not found (expected flashinfer/data/cutlass)")
+    raise RuntimeError(f"CUTLASS headers not found at {where}: gemm_gelu.cu needs a CUTLASS "
+                       f">= {CUTLASS_MIN[0]}.{CUTLASS_MIN[1]} tree; set SOL_CUTLASS_DIR to one")
+
+
+def cutlass_info():
+    """(root, 'major.minor.patch') of the CUTLASS tree the build uses."""
+    root = _cutlass_root()
+    return root, ".".join(map(str, _cutlass_version(root)))
 
 
 def _digest():
@@ -58,6 +98,8 @@ def _digest():
     with open(os.path.join(INCLUDE, "sol.h"), "rb") as fh:
         h.update(fh.read())
     h.update(" ".join(ARCH + FLAGS).encode())
+    root, ver = cutlass_info()
+    h.update(f"cutlass {ver} {root}".encode())
     return h.hexdigest()
 
 

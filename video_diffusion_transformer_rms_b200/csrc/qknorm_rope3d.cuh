@@ -20,6 +20,15 @@
 // the thousands) into a double-buffered shared table, one barrier per R rows.  Pairs are processed
 // two at a time with packed fp32x2 arithmetic (even and odd elements of two
 // adjacent rotary pairs side by side), gamma folded into the rotation.
+//
+// Table-driven form (TAB): the caller builds a rotary table once per
+// (positions, theta, head_dim, sections) -- row p holds cos(p*f_i) for every
+// pair i, then sin(p*f_i), each computed in fp64 and rounded once to fp32 --
+// and every thread reads the (cos, sin) of its own pairs at the row's
+// position on their axis straight from it (read-only path; the table is a few
+// hundred KB to a few MB and stays in L1/L2).  That removes the per-row fp64
+// angle work, sincosf, the shared angle tables and the CTA barrier: no thread
+// of the CTA waits for another, and the ring can run deeper.
 #pragma once
 #include "sol_device.cuh"
 #include "sol_launch.h"
@@ -38,18 +47,122 @@ __host__ __device__ constexpr size_t header_bytes() {
   return kMaxPairs * 8 + 2 * (2 * R * kMaxPairs * 4);
 }
 
-template <typename T, int G, int NT, int VPT, int R, int S>
+// Rotary axis of pair p: 0 = t, 1 = h, 2 = w.
+__device__ __forceinline__ int pair_axis(int p, int sec_t, int sec_th) {
+  return p < sec_t ? 0 : (p < sec_th ? 1 : 2);
+}
+
+// The NPR consecutive pairs p0 .. p0+NPR-1 that one thread rotates, read from
+// the rotary table of QkArgs::rope_tab (row stride 2*npairs floats: cos of
+// every pair, then sin).  `axes` holds each pair's axis (2 bits per pair);
+// `uni` says all of them share one axis, so their entries are adjacent in one
+// table row and come in 16-byte loads.
+template <int NPR>
+struct TabPairs {
+  int axes;
+  bool uni;
+  __device__ __forceinline__ void init(int p0, int sec_t, int sec_th) {
+    axes = 0;
+    const int a0 = pair_axis(p0, sec_t, sec_th);
+    uni = true;
+#pragma unroll
+    for (int i = 0; i < NPR; ++i) {
+      const int ax = pair_axis(p0 + i, sec_t, sec_th);
+      axes |= ax << (2 * i);
+      uni &= ax == a0;
+    }
+  }
+  // c[i], s[i]: cos and sin of pair p0 + i at position (t, h, w)
+  __device__ __forceinline__ void read(const float *tab, int npairs, int p0, int t, int h, int w,
+                                       float (&c)[NPR], float (&s)[NPR]) const {
+    const int64_t ld = 2 * static_cast<int64_t>(npairs);
+    if (uni) {
+      const int ax = axes & 3;
+      const int at = ax == 0 ? t : (ax == 1 ? h : w);
+      const float *row = tab + at * ld + p0;
+      if constexpr (NPR % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < NPR; i += 4) {
+          const float4 cv = __ldg(reinterpret_cast<const float4 *>(row + i));
+          const float4 sv = __ldg(reinterpret_cast<const float4 *>(row + npairs + i));
+          c[i] = cv.x, c[i + 1] = cv.y, c[i + 2] = cv.z, c[i + 3] = cv.w;
+          s[i] = sv.x, s[i + 1] = sv.y, s[i + 2] = sv.z, s[i + 3] = sv.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < NPR; i += 2) {
+          const float2 cv = __ldg(reinterpret_cast<const float2 *>(row + i));
+          const float2 sv = __ldg(reinterpret_cast<const float2 *>(row + npairs + i));
+          c[i] = cv.x, c[i + 1] = cv.y;
+          s[i] = sv.x, s[i + 1] = sv.y;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < NPR; ++i) {
+        const int ax = (axes >> (2 * i)) & 3;
+        const int at = ax == 0 ? t : (ax == 1 ? h : w);
+        const float *row = tab + at * ld + p0 + i;
+        c[i] = __ldg(row);
+        s[i] = __ldg(row + npairs);
+      }
+    }
+  }
+};
+
+// On-the-fly form: the (cos, sin) of the rotary angles of R consecutive rows,
+// the first at the cursors (rows past the CTA's share are computed but never
+// read), into cos_out/sin_out[R][kMaxPairs].  The angle pos * freq is formed
+// and reduced modulo 2*pi in fp64, then sincosf runs on the reduced fp32
+// angle.  The CTA's NT threads share the R * npairs entries.
+template <int R, int NT>
+__device__ __forceinline__ void angle_tables(const QkArgs &a, const double *freq, TokenCursor tok,
+                                             GridCursor pos, float *cos_out, float *sin_out) {
+  int pt[R], ph[R], pw[R];
+#pragma unroll
+  for (int q = 0; q < R; ++q) {
+    pt[q] = pos.t;
+    ph[q] = pos.h;
+    pw[q] = pos.w;
+    tok.next(a.L);
+    pos.next(tok.r, a.n_video, a.H, a.W);
+  }
+  for (int idx = threadIdx.x; idx < R * a.npairs; idx += NT) {
+    int q = 0, p = idx;
+#pragma unroll
+    for (int qq = 1; qq < R; ++qq)
+      if (p >= a.npairs) {
+        p -= a.npairs;
+        q = qq;
+      }
+    int at = pw[0];
+#pragma unroll
+    for (int qq = 0; qq < R; ++qq)
+      if (q == qq) at = p < a.sec_t ? pt[qq] : (p < a.sec_th ? ph[qq] : pw[qq]);
+    const double ang = static_cast<double>(at) * freq[p];
+    const double turns = rint(ang * kInv2Pi);
+    const float red = static_cast<float>(fma(-turns, k2Pi, ang));
+    float sv, cv;
+    sincosf(red, &sv, &cv);
+    cos_out[q * kMaxPairs + p] = cv;
+    sin_out[q * kMaxPairs + p] = sv;
+  }
+}
+
+template <typename T, int G, int NT, int VPT, int R, int S, bool TAB, int K = 0, bool BAR = false>
 __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
+  static_assert(K % R == 0, "a ring stage's rows must lie in one chunk");
   using IO = Io<T>;
   constexpr int E = IO::E;
   constexpr int PPV = E / 2;  // rotary pairs per 16-byte vector
   constexpr int Q = PPV / 2;  // float2 lanes of (pair 2m, pair 2m+1) per vector
-  constexpr int TAB = 2 * R * kMaxPairs;
+  constexpr int NTAB = 2 * R * kMaxPairs;
+  constexpr size_t HDR = TAB ? 0 : header_bytes<R>();
   extern __shared__ __align__(16) unsigned char smem[];
   double *freq = reinterpret_cast<double *>(smem);
-  float *cosb = reinterpret_cast<float *>(smem + kMaxPairs * 8);         // [2][R][kMaxPairs]
-  float *sinb = cosb + TAB;                                              // [2][R][kMaxPairs]
-  uint4 *ring = reinterpret_cast<uint4 *>(smem + header_bytes<R>());     // [S][R][2][VPT][NT]
+  float *cosb = reinterpret_cast<float *>(smem + kMaxPairs * 8);  // [2][R][kMaxPairs]
+  float *sinb = cosb + NTAB;                                      // [2][R][kMaxPairs]
+  uint4 *ring = reinterpret_cast<uint4 *>(smem + HDR);            // [S][R][2][VPT][NT]
 
   const int tid = threadIdx.x;
   const int gl = tid % G;   // lane within the head
@@ -76,16 +189,18 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
       for (int m = 0; m < Q; ++m) gev[part][m] = god[part][m] = splat2(1.f);
     }
   }
-  for (int p = tid; p < a.npairs; p += NT)
-    freq[p] = pow(static_cast<double>(a.theta), -2.0 * p / a.head_dim);
+  TabPairs<PPV> tp;
+  if constexpr (TAB) {
+    tp.init(p0, a.sec_t, a.sec_th);
+  } else {
+    for (int p = tid; p < a.npairs; p += NT)
+      freq[p] = pow(static_cast<double>(a.theta), -2.0 * p / a.head_dim);
+  }
 
-  int64_t begin;
-  int count;
-  cta_rows(a.rows, blockIdx.x, gridDim.x, begin, count);
+  RowOrder<K> ro;
+  ro.init(a.rows);
+  const int count = ro.count;
   const int iters = (count + R - 1) / R;
-  const unsigned char *src_c = qkv + begin * a.ld_qkv_bytes;
-  unsigned char *qo_c = qo + begin * a.ld_out_bytes;
-  unsigned char *ko_c = ko + begin * a.ld_out_bytes;
   auto slot = [&](int s, int q, int part, int k) -> uint4 * {
     return &ring[(((s * R + q) * 2 + part) * VPT + k) * NT + tid];
   };
@@ -94,7 +209,7 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
     for (int q = 0; q < R; ++q) {
       const int j = it * R + q;
       if (j < count) {
-        const unsigned char *src = src_c + j * a.ld_qkv_bytes;
+        const unsigned char *src = qkv + ro.row(j) * a.ld_qkv_bytes;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
           const uint4 *ps = reinterpret_cast<const uint4 *>(src + part * part_bytes) + tid;
@@ -109,55 +224,25 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
 
 #pragma unroll
   for (int s = 0; s < S - 1; ++s) issue(s, s);
-  __syncthreads();  // freq[] visible
+  if constexpr (!TAB) __syncthreads();  // freq[] visible
 
   TokenCursor tok;
-  tok.init(begin, a.L);
   GridCursor pos;
-  pos.init(tok.r, a.n_video, a.HW, a.W);
   int cons = 0;
   int buf = 0;
   for (int it = 0; it < iters; ++it) {
     issue(it + S - 1, cons == 0 ? S - 1 : cons - 1);
+    if (ro.run_start(it * R)) {  // this stage's rows start a new run
+      tok.init(ro.row(it * R), a.L);
+      pos.init(tok.r, a.n_video, a.HW, a.W);
+    }
 
-    // positions of this iteration's rows (rows past `end` are never read)
-    int pt[R], ph[R], pw[R];
-    {
-      TokenCursor t2 = tok;
-      GridCursor g2 = pos;
-#pragma unroll
-      for (int q = 0; q < R; ++q) {
-        pt[q] = g2.t;
-        ph[q] = g2.h;
-        pw[q] = g2.w;
-        t2.next(a.L);
-        g2.next(t2.r, a.n_video, a.H, a.W);
-      }
-    }
-    // (cos, sin) of every row's rotary angles, angle reduced modulo 2*pi in fp64
-    for (int idx = tid; idx < R * a.npairs; idx += NT) {
-      int q = 0, p = idx;
-#pragma unroll
-      for (int qq = 1; qq < R; ++qq)
-        if (p >= a.npairs) {
-          p -= a.npairs;
-          q = qq;
-        }
-      int at = pw[0];
-#pragma unroll
-      for (int qq = 0; qq < R; ++qq)
-        if (q == qq) at = p < a.sec_t ? pt[qq] : (p < a.sec_th ? ph[qq] : pw[qq]);
-      const double ang = static_cast<double>(at) * freq[p];
-      const double turns = rint(ang * kInv2Pi);
-      const float red = static_cast<float>(fma(-turns, k2Pi, ang));
-      float sv, cv;
-      sincosf(red, &sv, &cv);
-      cosb[(buf * R + q) * kMaxPairs + p] = cv;
-      sinb[(buf * R + q) * kMaxPairs + p] = sv;
-    }
+    if constexpr (!TAB)
+      angle_tables<R, NT>(a, freq, tok, pos, cosb + buf * R * kMaxPairs,
+                          sinb + buf * R * kMaxPairs);
 
     cp_async_wait<S - 1>();
-    __syncthreads();  // angle tables of these rows visible
+    if constexpr (!TAB || BAR) __syncthreads();  // angle tables of these rows visible
 
 #pragma unroll
     for (int q = 0; q < R; ++q) {
@@ -165,10 +250,22 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
       if (j < count) {
         // cs[m] = (cos of pair p0+2m, cos of pair p0+2m+1); likewise sn
         float2 cs[Q], sn[Q];
+        if constexpr (TAB) {
+          float c[PPV], s[PPV];
+          tp.read(a.rope_tab, a.npairs, p0, pos.t, pos.h, pos.w, c, s);
 #pragma unroll
-        for (int m = 0; m < Q; ++m) {
-          cs[m] = *reinterpret_cast<const float2 *>(&cosb[(buf * R + q) * kMaxPairs + p0 + 2 * m]);
-          sn[m] = *reinterpret_cast<const float2 *>(&sinb[(buf * R + q) * kMaxPairs + p0 + 2 * m]);
+          for (int m = 0; m < Q; ++m) {
+            cs[m] = make_float2(c[2 * m], c[2 * m + 1]);
+            sn[m] = make_float2(s[2 * m], s[2 * m + 1]);
+          }
+        } else {
+#pragma unroll
+          for (int m = 0; m < Q; ++m) {
+            cs[m] =
+                *reinterpret_cast<const float2 *>(&cosb[(buf * R + q) * kMaxPairs + p0 + 2 * m]);
+            sn[m] =
+                *reinterpret_cast<const float2 *>(&sinb[(buf * R + q) * kMaxPairs + p0 + 2 * m]);
+          }
         }
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
@@ -183,7 +280,7 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
             c1[m] = mul2(god[part][m], cs[m]);
           }
           uint4 *dst =
-              reinterpret_cast<uint4 *>((part == 0 ? qo_c : ko_c) + j * a.ld_out_bytes) + tid;
+              reinterpret_cast<uint4 *>((part == 0 ? qo : ko) + ro.row(j) * a.ld_out_bytes) + tid;
 #pragma unroll
           for (int k = 0; k < VPT; ++k) {
             // every lane joins the shuffles; ok[] only guards memory accesses
@@ -219,24 +316,48 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
   cp_async_wait<0>();
 }
 
-template <typename T, int G, int NT, int VPT>
-cudaError_t launch(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
-  constexpr int R = VPT <= 6 ? 2 : 1;  // keeps the ring within shared memory
-  constexpr int S = 2;
-  const void *fn = reinterpret_cast<const void *>(&qknorm_rope3d_kernel<T, G, NT, VPT, R, S>);
-  const size_t smem = header_bytes<R>() + static_cast<size_t>(S) * R * 2 * VPT * NT * 16;
+// One launch of a fixed configuration: a wave of as many CTAs as fit.
+template <typename T, int G, int NT, int VPT, int R, int S, bool TAB, int K = 0, bool BAR = false>
+cudaError_t launch_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
+  const void *fn =
+      reinterpret_cast<const void *>(&qknorm_rope3d_kernel<T, G, NT, VPT, R, S, TAB, K, BAR>);
+  const size_t smem =
+      (TAB ? 0 : header_bytes<R>()) + static_cast<size_t>(S) * R * 2 * VPT * NT * 16;
   const int per_sm = resident_blocks(fn, NT, smem);
   if (per_sm <= 0) return cudaErrorInvalidConfiguration;
   int64_t grid = static_cast<int64_t>(per_sm) * device_sms();
   if (grid > a.rows) grid = a.rows;
   if (geo) *geo = Geometry{NT, VPT, S, smem, static_cast<int>(grid)};
-  qknorm_rope3d_kernel<T, G, NT, VPT, R, S>
+  qknorm_rope3d_kernel<T, G, NT, VPT, R, S, TAB, K, BAR>
       <<<static_cast<unsigned>(grid), NT, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
+template <typename T, int G, int NT, int VPT>
+cudaError_t launch(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
+  constexpr int R = VPT <= 6 ? 2 : 1;  // keeps the ring within shared memory
+  return launch_cfg<T, G, NT, VPT, R, 2, false>(a, stream, geo);
+}
+
+// Table-driven kernels: with no barrier and no angle tables the ring runs
+// one row per stage, three stages deep (two rows in flight per CTA).
+constexpr int kTabRows = 1;
+constexpr int kTabStages = 3;
+
+template <typename T, int G>
+cudaError_t dispatch_tab(const QkArgs &a, int threads, int vpt, cudaStream_t stream,
+                         Geometry *geo) {
+#define SOL_CASE(NT, V)          \
+  if (threads == NT && vpt == V) \
+    return launch_cfg<T, G, NT, V, kTabRows, kTabStages, true>(a, stream, geo);
+  SOL_QK_SPLITS(SOL_CASE)
+#undef SOL_CASE
+  return cudaErrorInvalidValue;
+}
+
 template <typename T, int G>
 cudaError_t dispatch(const QkArgs &a, int threads, int vpt, cudaStream_t stream, Geometry *geo) {
+  if (a.rope_tab) return dispatch_tab<T, G>(a, threads, vpt, stream, geo);
 #define SOL_CASE(NT, V) \
   if (threads == NT && vpt == V) return launch<T, G, NT, V>(a, stream, geo);
   SOL_QK_SPLITS(SOL_CASE)

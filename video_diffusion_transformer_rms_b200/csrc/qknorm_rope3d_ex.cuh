@@ -8,8 +8,8 @@
 //     article's 4x/8x B300 runs send between GPUs;
 //   - a per-axis frequency ladder: each of the t/h/w sections a RoPE of its
 //     own, pair j of a section of s pairs at theta^(-j/s).
-// Same structure as qknorm_rope3d.cuh (ring, cursors, per-row angle tables,
-// G lanes per head).  With the half-split layout a thread's partner elements
+// Same structure as qknorm_rope3d.cuh (ring, cursors, per-row angle tables or
+// the precomputed rotary table (TAB), G lanes per head).  With the half-split layout a thread's partner elements
 // (i + hd/2, or i - hd/2) sit in lane gl ^ G/2 of the same head: one 16-byte
 // shuffle per vector brings them over, and each thread writes only its own
 // elements.  With INT8 output the head's max |x| is a G-lane shuffle max,
@@ -22,19 +22,23 @@
 namespace sol {
 namespace qk {
 
-template <int G, int NT, int VPT, int R, int S, bool HALF, bool OUT8>
+template <int G, int NT, int VPT, int R, int S, bool HALF, bool OUT8, bool TAB, int K = 0,
+          bool BAR = false>
 __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
+  static_assert(K % R == 0, "a ring stage's rows must lie in one chunk");
   using IO = Io<__nv_bfloat16>;
   constexpr int E = IO::E;    // 8 elements per 16-byte vector
   constexpr int P = E / 2;    // natural pairs (2e, 2e+1)
   constexpr int Q = P / 2;    // float2 lanes of two rotary pairs (interleaved layout)
   constexpr int VB = OUT8 ? 8 : 16;  // output bytes per vector
-  constexpr int TAB = 2 * R * kMaxPairs;
+  constexpr int NPR = HALF ? E : P;  // rotary pairs of one thread's vector
+  constexpr int NTAB = 2 * R * kMaxPairs;
+  constexpr size_t HDR = TAB ? 0 : header_bytes<R>();
   extern __shared__ __align__(16) unsigned char smem[];
   double *freq = reinterpret_cast<double *>(smem);
   float *cosb = reinterpret_cast<float *>(smem + kMaxPairs * 8);
-  float *sinb = cosb + TAB;
-  uint4 *ring = reinterpret_cast<uint4 *>(smem + header_bytes<R>());
+  float *sinb = cosb + NTAB;
+  uint4 *ring = reinterpret_cast<uint4 *>(smem + HDR);
 
   const int tid = threadIdx.x;
   const int gl = tid % G;
@@ -74,22 +78,27 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
   // frequency of each rotary pair: one ladder over all pairs, or with
   // per_axis one per section (local pair j of a section of s pairs at
   // theta^(-j/s))
-  for (int p = tid; p < a.npairs; p += NT) {
-    double e = -2.0 * p / a.head_dim;
-    if (a.per_axis) {
-      const int start = p < a.sec_t ? 0 : (p < a.sec_th ? a.sec_t : a.sec_th);
-      const int size = p < a.sec_t ? a.sec_t : (p < a.sec_th ? a.sec_th - a.sec_t
-                                                             : a.npairs - a.sec_th);
-      e = -static_cast<double>(p - start) / size;
+  TabPairs<NPR> tp;
+  if constexpr (TAB) {
+    tp.init(p0, a.sec_t, a.sec_th);
+  } else {
+    for (int p = tid; p < a.npairs; p += NT) {
+      double e = -2.0 * p / a.head_dim;
+      if (a.per_axis) {
+        const int start = p < a.sec_t ? 0 : (p < a.sec_th ? a.sec_t : a.sec_th);
+        const int size = p < a.sec_t ? a.sec_t : (p < a.sec_th ? a.sec_th - a.sec_t
+                                                               : a.npairs - a.sec_th);
+        e = -static_cast<double>(p - start) / size;
+      }
+      freq[p] = pow(static_cast<double>(a.theta), e);
     }
-    freq[p] = pow(static_cast<double>(a.theta), e);
   }
 
-  int64_t begin;
-  int count;
-  cta_rows(a.rows, blockIdx.x, gridDim.x, begin, count);
+  RowOrder<K> ro;
+  ro.init(a.rows);
+  const int count = ro.count;
   const int iters = (count + R - 1) / R;
-  const unsigned char *src_c = static_cast<const unsigned char *>(a.qkv) + begin * a.ld_qkv_bytes;
+  const unsigned char *qkv = static_cast<const unsigned char *>(a.qkv);
   auto slot = [&](int s, int q, int part, int k) -> uint4 * {
     return &ring[(((s * R + q) * 2 + part) * VPT + k) * NT + tid];
   };
@@ -98,7 +107,7 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
     for (int q = 0; q < R; ++q) {
       const int j = it * R + q;
       if (j < count) {
-        const unsigned char *src = src_c + j * a.ld_qkv_bytes;
+        const unsigned char *src = qkv + ro.row(j) * a.ld_qkv_bytes;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
           const uint4 *ps = reinterpret_cast<const uint4 *>(src + part * part_bytes) + tid;
@@ -113,59 +122,40 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
 
 #pragma unroll
   for (int s = 0; s < S - 1; ++s) issue(s, s);
-  __syncthreads();
+  if constexpr (!TAB) __syncthreads();
 
   TokenCursor tok;
-  tok.init(begin, a.L);
   GridCursor pos;
-  pos.init(tok.r, a.n_video, a.HW, a.W);
   int cons = 0;
   int buf = 0;
   for (int it = 0; it < iters; ++it) {
     issue(it + S - 1, cons == 0 ? S - 1 : cons - 1);
-    int pt[R], ph[R], pw[R];
-    {
-      TokenCursor t2 = tok;
-      GridCursor g2 = pos;
-#pragma unroll
-      for (int q = 0; q < R; ++q) {
-        pt[q] = g2.t;
-        ph[q] = g2.h;
-        pw[q] = g2.w;
-        t2.next(a.L);
-        g2.next(t2.r, a.n_video, a.H, a.W);
-      }
+    if (ro.run_start(it * R)) {  // this stage's rows start a new run
+      tok.init(ro.row(it * R), a.L);
+      pos.init(tok.r, a.n_video, a.HW, a.W);
     }
-    for (int idx = tid; idx < R * a.npairs; idx += NT) {
-      int q = 0, p = idx;
-#pragma unroll
-      for (int qq = 1; qq < R; ++qq)
-        if (p >= a.npairs) {
-          p -= a.npairs;
-          q = qq;
-        }
-      int at = pw[0];
-#pragma unroll
-      for (int qq = 0; qq < R; ++qq)
-        if (q == qq) at = p < a.sec_t ? pt[qq] : (p < a.sec_th ? ph[qq] : pw[qq]);
-      const double ang = static_cast<double>(at) * freq[p];
-      const double turns = rint(ang * kInv2Pi);
-      const float red = static_cast<float>(fma(-turns, k2Pi, ang));
-      float sv, cv;
-      sincosf(red, &sv, &cv);
-      cosb[(buf * R + q) * kMaxPairs + p] = cv;
-      sinb[(buf * R + q) * kMaxPairs + p] = sv;
-    }
+    if constexpr (!TAB)
+      angle_tables<R, NT>(a, freq, tok, pos, cosb + buf * R * kMaxPairs,
+                          sinb + buf * R * kMaxPairs);
 
     cp_async_wait<S - 1>();
-    __syncthreads();
+    if constexpr (!TAB || BAR) __syncthreads();
 
 #pragma unroll
     for (int q = 0; q < R; ++q) {
       const int j = it * R + q;
       if (j < count) {
-        const float *ct = &cosb[(buf * R + q) * kMaxPairs + p0];
-        const float *st = &sinb[(buf * R + q) * kMaxPairs + p0];
+        // cos and sin of this thread's NPR pairs p0 .. p0 + NPR - 1
+        float ct[NPR], st[NPR];
+        if constexpr (TAB) {
+          tp.read(a.rope_tab, a.npairs, p0, pos.t, pos.h, pos.w, ct, st);
+        } else {
+#pragma unroll
+          for (int i = 0; i < NPR; ++i) {
+            ct[i] = cosb[(buf * R + q) * kMaxPairs + p0 + i];
+            st[i] = sinb[(buf * R + q) * kMaxPairs + p0 + i];
+          }
+        }
         const int64_t row_off = static_cast<int64_t>(tok.b) * a.out_sb +
                                 static_cast<int64_t>(tok.r) * a.out_sr;
 #pragma unroll
@@ -177,16 +167,16 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
             const float sgn = gl >= G / 2 ? 1.f : -1.f;
 #pragma unroll
             for (int m = 0; m < P; ++m) {
-              const float2 cc = *reinterpret_cast<const float2 *>(ct + 2 * m);
-              const float2 ss = *reinterpret_cast<const float2 *>(st + 2 * m);
+              const float2 cc = make_float2(ct[2 * m], ct[2 * m + 1]);
+              const float2 ss = make_float2(st[2 * m], st[2 * m + 1]);
               ca[m] = mul2(gown[part][m], cc);
               sb[m] = mul2(gpar[part][m], make_float2(sgn * ss.x, sgn * ss.y));
             }
           } else {
 #pragma unroll
             for (int m = 0; m < Q; ++m) {
-              const float2 cs = *reinterpret_cast<const float2 *>(ct + 2 * m);
-              const float2 sn = *reinterpret_cast<const float2 *>(st + 2 * m);
+              const float2 cs = make_float2(ct[2 * m], ct[2 * m + 1]);
+              const float2 sn = make_float2(st[2 * m], st[2 * m + 1]);
               c0[m] = mul2(gev[part][m], cs);
               s0[m] = mul2(gev[part][m], sn);
               ns1[m] = mul2(god[part][m], make_float2(-sn.x, -sn.y));
@@ -196,7 +186,7 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
           unsigned char *obase = static_cast<unsigned char *>(part == 0 ? a.q_out : a.k_out) +
                                  row_off;
           float *scale_row = OUT8 ? (part == 0 ? a.q_scale : a.k_scale) +
-                                        (begin + j) * static_cast<int64_t>(a.n_heads)
+                                        ro.row(j) * static_cast<int64_t>(a.n_heads)
                                   : nullptr;
 #pragma unroll
           for (int k = 0; k < VPT; ++k) {
@@ -319,25 +309,34 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
 template <bool HALF, bool OUT8>
 constexpr bool kRowSplit = HALF != OUT8;
 
-template <int G, int NT, int VPT, bool HALF, bool OUT8>
-cudaError_t launch_ex(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
-  // One row per ring stage for INT8 and for half-split bf16 (half the ring,
-  // more CTAs per SM; INT8 0.90 against 1.04 ms at the 5 s clip), two rows
-  // per stage (one barrier per two rows) for interleaved bf16, which measured
-  // as fast or faster for it.
-  constexpr int R = (OUT8 || HALF) ? 1 : (VPT <= 6 ? 2 : 1);
-  constexpr int S = 2;
-  const void *fn =
-      reinterpret_cast<const void *>(&qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8>);
-  const size_t smem = header_bytes<R>() + static_cast<size_t>(S) * R * 2 * VPT * NT * 16;
+// One launch of a fixed configuration: a wave of as many CTAs as fit.
+template <int G, int NT, int VPT, int R, int S, bool HALF, bool OUT8, bool TAB, int K = 0,
+          bool BAR = false>
+cudaError_t launch_ex_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
+  const void *fn = reinterpret_cast<const void *>(
+      &qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8, TAB, K, BAR>);
+  const size_t smem =
+      (TAB ? 0 : header_bytes<R>()) + static_cast<size_t>(S) * R * 2 * VPT * NT * 16;
   const int per_sm = resident_blocks(fn, NT, smem);
   if (per_sm <= 0) return cudaErrorInvalidConfiguration;
   int64_t grid = static_cast<int64_t>(per_sm) * device_sms();
   if (grid > a.rows) grid = a.rows;
   if (geo) *geo = Geometry{NT, VPT, S, smem, static_cast<int>(grid)};
-  qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8>
+  qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8, TAB, K, BAR>
       <<<static_cast<unsigned>(grid), NT, smem, stream>>>(a);
   return cudaGetLastError();
+}
+
+template <int G, int NT, int VPT, bool HALF, bool OUT8>
+cudaError_t launch_ex(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
+  if (a.rope_tab)
+    return launch_ex_cfg<G, NT, VPT, kTabRows, kTabStages, HALF, OUT8, true>(a, stream, geo);
+  // One row per ring stage for INT8 and for half-split bf16 (half the ring,
+  // more CTAs per SM; INT8 0.90 against 1.04 ms at the 5 s clip), two rows
+  // per stage (one barrier per two rows) for interleaved bf16, which measured
+  // as fast or faster for it.
+  constexpr int R = (OUT8 || HALF) ? 1 : (VPT <= 6 ? 2 : 1);
+  return launch_ex_cfg<G, NT, VPT, R, 2, HALF, OUT8, false>(a, stream, geo);
 }
 
 template <int G, bool HALF, bool OUT8>

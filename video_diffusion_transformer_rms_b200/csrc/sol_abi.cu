@@ -1,7 +1,9 @@
 // C ABI of libsol (declared in include/sol.h): host-side argument checks,
 // then one kernel launch on the caller's stream.  Nothing is allocated and
 // nothing is synchronised.
+#include <algorithm>
 #include <cstdarg>
+#include <initializer_list>
 #include <cstdio>
 #include <map>
 #include <mutex>
@@ -157,11 +159,302 @@ bool pick_split_qk(int64_t nvec, int *threads, int *vpt) {
 
 }  // namespace sol
 
+namespace sol {
+namespace {
+
+// Argument checks of sol_qknorm_rope3d (and of its table-driven form, which
+// passes the table's head_dim, sections and theta).  On SOL_OK either
+// `empty` is set (zero rows: nothing to launch) or `a` is filled.
+sol_status check_qk(const char *fn, const void *qkv, int64_t ld_qkv, void *q_out, void *k_out,
+                    int64_t ld_out, const void *gamma_q, const void *gamma_k, int64_t B,
+                    int64_t T, int64_t H, int64_t W, int64_t n_audio, int64_t n_heads,
+                    int64_t head_dim, int64_t sec_t, int64_t sec_h, int64_t sec_w, float eps,
+                    float theta, sol_dtype dtype, QkArgs &a, bool &empty) {
+  empty = false;
+  if (dtype != SOL_F32 && dtype != SOL_BF16)
+    return fail(SOL_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
+  if (B < 0 || T < 0 || H < 0 || W < 0 || n_audio < 0)
+    return fail(SOL_ERR_INVALID_ARG, "%s: B, T, H, W, n_audio must be >= 0", fn);
+  if (n_heads <= 0 || head_dim <= 0 || head_dim % 2 != 0)
+    return fail(SOL_ERR_INVALID_ARG, "%s: need n_heads > 0 and an even head_dim > 0 (%lld, %lld)",
+                fn, (long long)n_heads, (long long)head_dim);
+  if (sec_t < 0 || sec_h < 0 || sec_w < 0 || sec_t + sec_h + sec_w != head_dim / 2)
+    return fail(SOL_ERR_INVALID_ARG, "%s: sections %lld+%lld+%lld must sum to head_dim/2 = %lld",
+                fn, (long long)sec_t, (long long)sec_h, (long long)sec_w,
+                (long long)(head_dim / 2));
+  if (!(eps >= 0.f) || !(theta > 0.f))
+    return fail(SOL_ERR_INVALID_ARG, "%s: need eps >= 0 and theta > 0", fn);
+  if (T > kMaxRows || H > kMaxRows || W > kMaxRows || n_audio > kMaxRows || B > kMaxRows ||
+      H * W > kMaxRows || T * H * W > kMaxRows || T * H * W + n_audio > kMaxRows ||
+      B * (T * H * W + n_audio) > kMaxRows)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: B*L and H*W must be below 2^31", fn);
+  const int64_t n_video = T * H * W;
+  const int64_t L = n_video + n_audio;
+  const int64_t rows = B * L;
+  const int64_t D = n_heads * head_dim;
+  if (ld_qkv < 2 * D || ld_out < D)
+    return fail(SOL_ERR_INVALID_ARG, "%s: need ld_qkv >= 2*D and ld_out >= D", fn);
+  if (rows == 0) {
+    empty = true;
+    return ok();
+  }
+  if (!qkv || !q_out || !k_out)
+    return fail(SOL_ERR_INVALID_ARG, "%s: qkv, q_out and k_out must be non-null", fn);
+  const int es = esize_of(dtype);
+  const int64_t hd_bytes = head_dim * es;
+  const int64_t G = hd_bytes / 16;
+  if (hd_bytes % 16 != 0 || G < 2 || G > 32 || (G & (G - 1)) != 0)
+    return fail(SOL_ERR_UNSUPPORTED,
+                "%s: head_dim*%d bytes must be 16*G with G a power of two in "
+                "[2, 32] (head_dim=%lld)",
+                fn, es, (long long)head_dim);
+  const int64_t ldq_b = ld_qkv * es, ldo_b = ld_out * es, D_b = D * es;
+  if (!aligned16(qkv) || !aligned16(q_out) || !aligned16(k_out) || ldq_b % 16 || ldo_b % 16 ||
+      (gamma_q && !aligned16(gamma_q)) || (gamma_k && !aligned16(gamma_k)))
+    return fail(SOL_ERR_MISALIGNED, "%s: pointers and row strides must be 16-byte aligned", fn);
+  if (2 * D_b > kMaxRowBytesQk)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: 2*D=%lld exceeds %lld elements", fn,
+                (long long)(2 * D), (long long)(kMaxRowBytesQk / es));
+  const bool in_place = q_out == qkv && ld_out == ld_qkv &&
+                        static_cast<const unsigned char *>(k_out) ==
+                            static_cast<const unsigned char *>(qkv) + D_b;
+  if (!in_place) {
+    if (!strided_disjoint(qkv, 2 * D_b, q_out, D_b, rows, ldq_b, ldo_b) ||
+        !strided_disjoint(qkv, 2 * D_b, k_out, D_b, rows, ldq_b, ldo_b) ||
+        !strided_disjoint(q_out, D_b, k_out, D_b, rows, ldo_b, ldo_b))
+      return fail(SOL_ERR_INVALID_ARG,
+                  "%s: outputs must be exactly in place (q_out=qkv, "
+                  "k_out=qkv+D, ld_out=ld_qkv) or overlap neither qkv nor each other",
+                  fn);
+  }
+  for (const void *g : {gamma_q, gamma_k}) {
+    if (!g) continue;
+    Span gs = span_of(g, 1, 0, hd_bytes);
+    if (spans_overlap(gs, span_of(q_out, rows, ldo_b, D_b)) ||
+        spans_overlap(gs, span_of(k_out, rows, ldo_b, D_b)))
+      return fail(SOL_ERR_INVALID_ARG, "%s: an output overlaps gamma", fn);
+  }
+
+  a = QkArgs{};
+  a.qkv = qkv;
+  a.q_out = q_out;
+  a.k_out = k_out;
+  a.gamma_q = gamma_q;
+  a.gamma_k = gamma_k;
+  a.ld_qkv_bytes = ldq_b;
+  a.ld_out_bytes = ldo_b;
+  a.rows = rows;
+  a.L = static_cast<int>(L);
+  a.n_video = static_cast<int>(n_video);
+  a.HW = static_cast<int>(H * W);
+  a.H = static_cast<int>(H);
+  a.W = static_cast<int>(W);
+  a.nvec_q = static_cast<int>(D_b / 16);
+  a.npairs = static_cast<int>(head_dim / 2);
+  a.sec_t = static_cast<int>(sec_t);
+  a.sec_th = static_cast<int>(sec_t + sec_h);
+  a.head_dim = static_cast<int>(head_dim);
+  a.eps = eps;
+  a.inv_hd = static_cast<float>(1.0 / static_cast<double>(head_dim));
+  a.theta = theta;
+  return ok();
+}
+
+// The descriptor of a rotary table: fields in range, data aligned.
+sol_status check_table(const char *fn, const sol_rope_table *tab) {
+  if (!tab) return fail(SOL_ERR_INVALID_ARG, "%s: the table descriptor must be non-null", fn);
+  if (tab->n_pos < 0 || tab->n_pos > kMaxRows)
+    return fail(SOL_ERR_INVALID_ARG, "%s: table n_pos must be in [0, 2^31)", fn);
+  if (tab->head_dim < 2 || tab->head_dim % 2 != 0 || tab->head_dim > 2 * kMaxRotaryPairs)
+    return fail(SOL_ERR_INVALID_ARG, "%s: table head_dim must be even and in [2, %lld]", fn,
+                (long long)(2 * kMaxRotaryPairs));
+  if (tab->sec_t < 0 || tab->sec_h < 0 || tab->sec_w < 0 ||
+      tab->sec_t + tab->sec_h + tab->sec_w != tab->head_dim / 2)
+    return fail(SOL_ERR_INVALID_ARG, "%s: table sections must sum to head_dim/2", fn);
+  if (!(tab->theta > 0.f) || (tab->per_axis_freq != 0 && tab->per_axis_freq != 1))
+    return fail(SOL_ERR_INVALID_ARG, "%s: table theta must be > 0 and per_axis_freq 0 or 1", fn);
+  if (!tab->data) return fail(SOL_ERR_INVALID_ARG, "%s: table data must be non-null", fn);
+  if (!aligned16(tab->data))
+    return fail(SOL_ERR_MISALIGNED, "%s: table data must be 16-byte aligned", fn);
+  return ok();
+}
+
+// A call's use of a table: every position it meets is a row, and no output
+// span overlaps the table.
+sol_status check_table_use(const char *fn, const sol_rope_table *tab, int64_t T, int64_t H,
+                           int64_t W, int64_t n_audio, std::initializer_list<Span> outs) {
+  int64_t need = n_audio;
+  if (T * H * W > 0) need = std::max(need, std::max(T, std::max(H, W)));
+  if (tab->n_pos < need)
+    return fail(SOL_ERR_INVALID_ARG,
+                "%s: the table has %lld positions, the call needs %lld (max of T, H, W, n_audio)",
+                fn, (long long)tab->n_pos, (long long)need);
+  const Span ts = span_of(tab->data, 1, 0, static_cast<int64_t>(tab->n_pos) * tab->head_dim * 4);
+  for (const Span &o : outs)
+    if (tab->n_pos > 0 && spans_overlap(o, ts))
+      return fail(SOL_ERR_INVALID_ARG, "%s: an output overlaps the rotary table", fn);
+  return ok();
+}
+
+// sol_qknorm_rope3d_ex and its table-driven form (tab non-null: head_dim,
+// sections and theta are the table's, and the rotation reads it).
+sol_status qk_ex(const char *fn, const void *qkv, int64_t ld_qkv, void *q_out, void *k_out,
+                 const sol_qk_layout *layout, const void *gamma_q, const void *gamma_k,
+                 const sol_rope_table *tab, int64_t B, int64_t T, int64_t H, int64_t W,
+                 int64_t n_audio, int64_t n_heads, int64_t head_dim, int64_t sec_t,
+                 int64_t sec_h, int64_t sec_w, float eps, float theta, sol_dtype dtype,
+                 sol_stream_t stream) {
+  if (!layout) return fail(SOL_ERR_INVALID_ARG, "%s: layout must be non-null", fn);
+  if (dtype != SOL_BF16)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: bf16 input only", fn);
+  if (B < 0 || T < 0 || H < 0 || W < 0 || n_audio < 0 || n_heads <= 0)
+    return fail(SOL_ERR_INVALID_ARG, "%s: B, T, H, W, n_audio must be >= 0, n_heads > 0", fn);
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: head_dim must be 64, 128 or 256 (got %lld)", fn,
+                (long long)head_dim);
+  if (sec_t < 0 || sec_h < 0 || sec_w < 0 || sec_t + sec_h + sec_w != head_dim / 2)
+    return fail(SOL_ERR_INVALID_ARG, "%s: sections must sum to head_dim/2", fn);
+  if (!(eps >= 0.f) || !(theta > 0.f))
+    return fail(SOL_ERR_INVALID_ARG, "%s: need eps >= 0 and theta > 0", fn);
+  if (layout->stride_b < 0 || layout->stride_row < 0 || layout->stride_head < 0)
+    return fail(SOL_ERR_INVALID_ARG, "%s: strides must be >= 0", fn);
+  if (T > kMaxRows || H > kMaxRows || W > kMaxRows || n_audio > kMaxRows || B > kMaxRows ||
+      H * W > kMaxRows || T * H * W > kMaxRows || T * H * W + n_audio > kMaxRows ||
+      B * (T * H * W + n_audio) > kMaxRows)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: B*L and H*W must be below 2^31", fn);
+  const int64_t n_video = T * H * W;
+  const int64_t L = n_video + n_audio;
+  const int64_t rows = B * L;
+  const int64_t D = n_heads * head_dim;
+  if (ld_qkv < 2 * D) return fail(SOL_ERR_INVALID_ARG, "%s: need ld_qkv >= 2*D", fn);
+  if (rows == 0) return ok();
+  const bool int8 = layout->int8_out != 0;
+  if (layout->reserved != 0 || (layout->per_axis_freq != 0 && layout->per_axis_freq != 1))
+    return fail(SOL_ERR_INVALID_ARG, "%s: layout.reserved must be 0, per_axis_freq 0 or 1", fn);
+  const bool quant_v = layout->v_out != nullptr;
+  if (quant_v && !int8)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: v_out needs int8_out (v is only quantised)", fn);
+  if (!qkv || !q_out || !k_out || (int8 && (!layout->q_scale || !layout->k_scale)) ||
+      (quant_v && !layout->v_scale))
+    return fail(SOL_ERR_INVALID_ARG, "%s: qkv, q_out, k_out (and scales) must be non-null", fn);
+  if (quant_v && ld_qkv < 3 * D)
+    return fail(SOL_ERR_INVALID_ARG, "%s: quantising v needs ld_qkv >= 3*D", fn);
+  if (2 * D * 2 > kMaxRowBytesQk)
+    return fail(SOL_ERR_UNSUPPORTED, "%s: 2*D=%lld exceeds %lld elements", fn, (long long)(2 * D),
+                (long long)(kMaxRowBytesQk / 2));
+  const int oes = int8 ? 1 : 2;     // output element size
+  const int vb = int8 ? 8 : 16;     // output bytes per thread vector
+  const int64_t sb = layout->stride_b * oes, sr = layout->stride_row * oes,
+                sh = layout->stride_head * oes;
+  if (!aligned16(qkv) || (ld_qkv * 2) % 16 || (gamma_q && !aligned16(gamma_q)) ||
+      (gamma_k && !aligned16(gamma_k)) || reinterpret_cast<uintptr_t>(q_out) % vb ||
+      reinterpret_cast<uintptr_t>(k_out) % vb || sb % vb || sr % vb || sh % vb ||
+      (int8 && ((reinterpret_cast<uintptr_t>(layout->q_scale) & 3u) ||
+                (reinterpret_cast<uintptr_t>(layout->k_scale) & 3u))) ||
+      (quant_v && ((reinterpret_cast<uintptr_t>(layout->v_out) % vb) ||
+                   (reinterpret_cast<uintptr_t>(layout->v_scale) & 3u))))
+    return fail(SOL_ERR_MISALIGNED, "%s: pointers and strides must be aligned", fn);
+  // byte extent of one output: last element + 1
+  const int64_t ext = (B - 1) * sb + (L - 1) * sr + (n_heads - 1) * sh + head_dim * oes;
+  const Span qs = span_of(q_out, 1, 0, ext), ks = span_of(k_out, 1, 0, ext);
+  // the columns read: q and k, and v too when it is quantised
+  const Span in = span_of(qkv, rows, ld_qkv * 2, (quant_v ? 3 : 2) * D * 2);
+  // v's codes: the layout of q_out; an empty span when v is not quantised
+  const Span vs = quant_v ? span_of(layout->v_out, 1, 0, ext) : Span{0, 0};
+  if (spans_overlap(qs, in) || spans_overlap(ks, in) || spans_overlap(qs, ks) ||
+      spans_overlap(vs, in) || spans_overlap(vs, qs) || spans_overlap(vs, ks))
+    return fail(SOL_ERR_INVALID_ARG,
+                "%s: q_out, k_out and v_out must overlap neither qkv nor each other", fn);
+  if (int8) {
+    const int64_t sc = rows * n_heads * 4;
+    const Span a1 = span_of(layout->q_scale, 1, 0, sc), a2 = span_of(layout->k_scale, 1, 0, sc);
+    const Span a3 = quant_v ? span_of(layout->v_scale, 1, 0, sc) : Span{0, 0};
+    for (const Span &z : {a1, a2, a3})
+      if (spans_overlap(z, qs) || spans_overlap(z, ks) || spans_overlap(z, vs) ||
+          spans_overlap(z, in))
+        return fail(SOL_ERR_INVALID_ARG, "%s: a scale array overlaps a tensor", fn);
+    if (spans_overlap(a1, a2) || spans_overlap(a1, a3) || spans_overlap(a2, a3))
+      return fail(SOL_ERR_INVALID_ARG, "%s: the scale arrays overlap", fn);
+  }
+  for (const void *g : {gamma_q, gamma_k}) {
+    if (!g) continue;
+    const Span gs = span_of(g, 1, 0, head_dim * 2);
+    if (spans_overlap(gs, qs) || spans_overlap(gs, ks) || spans_overlap(gs, vs))
+      return fail(SOL_ERR_INVALID_ARG, "%s: an output overlaps gamma", fn);
+  }
+
+  if (tab) {
+    const int64_t sc = int8 ? rows * n_heads * 4 : 0;
+    const Span z{0, 0};
+    const sol_status st = check_table_use(
+        fn, tab, T, H, W, n_audio,
+        {qs, ks, vs, int8 ? span_of(layout->q_scale, 1, 0, sc) : z,
+         int8 ? span_of(layout->k_scale, 1, 0, sc) : z,
+         quant_v ? span_of(layout->v_scale, 1, 0, sc) : z});
+    if (st != SOL_OK) return st;
+  }
+
+  QkArgs a{};
+  a.qkv = qkv;
+  a.q_out = q_out;
+  a.k_out = k_out;
+  a.gamma_q = gamma_q;
+  a.gamma_k = gamma_k;
+  a.ld_qkv_bytes = ld_qkv * 2;
+  a.ld_out_bytes = 0;
+  a.rows = rows;
+  a.L = static_cast<int>(L);
+  a.n_video = static_cast<int>(n_video);
+  a.HW = static_cast<int>(H * W);
+  a.H = static_cast<int>(H);
+  a.W = static_cast<int>(W);
+  a.nvec_q = static_cast<int>(D * 2 / 16);
+  a.npairs = static_cast<int>(head_dim / 2);
+  a.sec_t = static_cast<int>(sec_t);
+  a.sec_th = static_cast<int>(sec_t + sec_h);
+  a.head_dim = static_cast<int>(head_dim);
+  a.eps = eps;
+  a.inv_hd = static_cast<float>(1.0 / static_cast<double>(head_dim));
+  a.theta = theta;
+  a.out_sb = sb;
+  a.out_sr = sr;
+  a.out_sh = sh;
+  a.q_scale = layout->q_scale;
+  a.k_scale = layout->k_scale;
+  a.n_heads = static_cast<int>(n_heads);
+  a.per_axis = layout->per_axis_freq;
+  a.rope_tab = tab ? tab->data : nullptr;
+  const bool half = layout->half_split != 0;
+  cudaError_t e = int8 ? launch_qknorm_rope3d_ex_int8out(a, half, stream, nullptr)
+                       : launch_qknorm_rope3d_ex_bf16out(a, half, stream, nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  if (quant_v) {
+    QuantArgs v{};
+    v.src = static_cast<const unsigned char *>(qkv) + 2 * D * 2;
+    v.ld_src_bytes = ld_qkv * 2;
+    v.out = layout->v_out;
+    v.scale = layout->v_scale;
+    v.out_sb = sb;
+    v.out_sr = sr;
+    v.out_sh = sh;
+    v.rows = rows;
+    v.L = static_cast<int>(L);
+    v.nvec = static_cast<int>(D * 2 / 16);
+    v.n_heads = static_cast<int>(n_heads);
+    e = launch_quantize_heads_int8(v, static_cast<int>(head_dim), stream, nullptr);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+  }
+  return ok();
+}
+
+}  // namespace
+}  // namespace sol
+
 using namespace sol;
 
 extern "C" {
 
-int sol_version(void) { return (2 << 16) | 0; }
+int sol_version(void) { return (2 << 16) | 1; }
 
 const char *sol_status_string(sol_status s) {
   switch (s) {
@@ -350,136 +643,27 @@ sol_status sol_qknorm_rope3d_ex(const void *qkv, int64_t ld_qkv, void *q_out, vo
                                 int64_t n_audio, int64_t n_heads, int64_t head_dim, int64_t sec_t,
                                 int64_t sec_h, int64_t sec_w, float eps, float theta,
                                 sol_dtype dtype, sol_stream_t stream) {
-  const char *fn = "sol_qknorm_rope3d_ex";
-  if (!layout) return fail(SOL_ERR_INVALID_ARG, "%s: layout must be non-null", fn);
-  if (dtype != SOL_BF16)
-    return fail(SOL_ERR_UNSUPPORTED, "%s: bf16 input only", fn);
-  if (B < 0 || T < 0 || H < 0 || W < 0 || n_audio < 0 || n_heads <= 0)
-    return fail(SOL_ERR_INVALID_ARG, "%s: B, T, H, W, n_audio must be >= 0, n_heads > 0", fn);
-  if (head_dim != 64 && head_dim != 128 && head_dim != 256)
-    return fail(SOL_ERR_UNSUPPORTED, "%s: head_dim must be 64, 128 or 256 (got %lld)", fn,
-                (long long)head_dim);
-  if (sec_t < 0 || sec_h < 0 || sec_w < 0 || sec_t + sec_h + sec_w != head_dim / 2)
-    return fail(SOL_ERR_INVALID_ARG, "%s: sections must sum to head_dim/2", fn);
-  if (!(eps >= 0.f) || !(theta > 0.f))
-    return fail(SOL_ERR_INVALID_ARG, "%s: need eps >= 0 and theta > 0", fn);
-  if (layout->stride_b < 0 || layout->stride_row < 0 || layout->stride_head < 0)
-    return fail(SOL_ERR_INVALID_ARG, "%s: strides must be >= 0", fn);
-  if (T > kMaxRows || H > kMaxRows || W > kMaxRows || n_audio > kMaxRows || B > kMaxRows ||
-      H * W > kMaxRows || T * H * W > kMaxRows || T * H * W + n_audio > kMaxRows ||
-      B * (T * H * W + n_audio) > kMaxRows)
-    return fail(SOL_ERR_UNSUPPORTED, "%s: B*L and H*W must be below 2^31", fn);
-  const int64_t n_video = T * H * W;
-  const int64_t L = n_video + n_audio;
-  const int64_t rows = B * L;
-  const int64_t D = n_heads * head_dim;
-  if (ld_qkv < 2 * D) return fail(SOL_ERR_INVALID_ARG, "%s: need ld_qkv >= 2*D", fn);
-  if (rows == 0) return ok();
-  const bool int8 = layout->int8_out != 0;
-  if (layout->reserved != 0 || (layout->per_axis_freq != 0 && layout->per_axis_freq != 1))
-    return fail(SOL_ERR_INVALID_ARG, "%s: layout.reserved must be 0, per_axis_freq 0 or 1", fn);
-  const bool quant_v = layout->v_out != nullptr;
-  if (quant_v && !int8)
-    return fail(SOL_ERR_UNSUPPORTED, "%s: v_out needs int8_out (v is only quantised)", fn);
-  if (!qkv || !q_out || !k_out || (int8 && (!layout->q_scale || !layout->k_scale)) ||
-      (quant_v && !layout->v_scale))
-    return fail(SOL_ERR_INVALID_ARG, "%s: qkv, q_out, k_out (and scales) must be non-null", fn);
-  if (quant_v && ld_qkv < 3 * D)
-    return fail(SOL_ERR_INVALID_ARG, "%s: quantising v needs ld_qkv >= 3*D", fn);
-  if (2 * D * 2 > kMaxRowBytesQk)
-    return fail(SOL_ERR_UNSUPPORTED, "%s: 2*D=%lld exceeds %lld elements", fn, (long long)(2 * D),
-                (long long)(kMaxRowBytesQk / 2));
-  const int oes = int8 ? 1 : 2;     // output element size
-  const int vb = int8 ? 8 : 16;     // output bytes per thread vector
-  const int64_t sb = layout->stride_b * oes, sr = layout->stride_row * oes,
-                sh = layout->stride_head * oes;
-  if (!aligned16(qkv) || (ld_qkv * 2) % 16 || (gamma_q && !aligned16(gamma_q)) ||
-      (gamma_k && !aligned16(gamma_k)) || reinterpret_cast<uintptr_t>(q_out) % vb ||
-      reinterpret_cast<uintptr_t>(k_out) % vb || sb % vb || sr % vb || sh % vb ||
-      (int8 && ((reinterpret_cast<uintptr_t>(layout->q_scale) & 3u) ||
-                (reinterpret_cast<uintptr_t>(layout->k_scale) & 3u))) ||
-      (quant_v && ((reinterpret_cast<uintptr_t>(layout->v_out) % vb) ||
-                   (reinterpret_cast<uintptr_t>(layout->v_scale) & 3u))))
-    return fail(SOL_ERR_MISALIGNED, "%s: pointers and strides must be aligned", fn);
-  // byte extent of one output: last element + 1
-  const int64_t ext = (B - 1) * sb + (L - 1) * sr + (n_heads - 1) * sh + head_dim * oes;
-  const Span qs = span_of(q_out, 1, 0, ext), ks = span_of(k_out, 1, 0, ext);
-  // the columns read: q and k, and v too when it is quantised
-  const Span in = span_of(qkv, rows, ld_qkv * 2, (quant_v ? 3 : 2) * D * 2);
-  // v's codes: the layout of q_out; an empty span when v is not quantised
-  const Span vs = quant_v ? span_of(layout->v_out, 1, 0, ext) : Span{0, 0};
-  if (spans_overlap(qs, in) || spans_overlap(ks, in) || spans_overlap(qs, ks) ||
-      spans_overlap(vs, in) || spans_overlap(vs, qs) || spans_overlap(vs, ks))
-    return fail(SOL_ERR_INVALID_ARG,
-                "%s: q_out, k_out and v_out must overlap neither qkv nor each other", fn);
-  if (int8) {
-    const int64_t sc = rows * n_heads * 4;
-    const Span a1 = span_of(layout->q_scale, 1, 0, sc), a2 = span_of(layout->k_scale, 1, 0, sc);
-    const Span a3 = quant_v ? span_of(layout->v_scale, 1, 0, sc) : Span{0, 0};
-    for (const Span &z : {a1, a2, a3})
-      if (spans_overlap(z, qs) || spans_overlap(z, ks) || spans_overlap(z, vs) ||
-          spans_overlap(z, in))
-        return fail(SOL_ERR_INVALID_ARG, "%s: a scale array overlaps a tensor", fn);
-    if (spans_overlap(a1, a2) || spans_overlap(a1, a3) || spans_overlap(a2, a3))
-      return fail(SOL_ERR_INVALID_ARG, "%s: the scale arrays overlap", fn);
-  }
-  for (const void *g : {gamma_q, gamma_k}) {
-    if (!g) continue;
-    const Span gs = span_of(g, 1, 0, head_dim * 2);
-    if (spans_overlap(gs, qs) || spans_overlap(gs, ks) || spans_overlap(gs, vs))
-      return fail(SOL_ERR_INVALID_ARG, "%s: an output overlaps gamma", fn);
-  }
+  return qk_ex("sol_qknorm_rope3d_ex", qkv, ld_qkv, q_out, k_out, layout, gamma_q, gamma_k,
+               nullptr, B, T, H, W, n_audio, n_heads, head_dim, sec_t, sec_h, sec_w, eps, theta,
+               dtype, stream);
+}
 
-  QkArgs a{};
-  a.qkv = qkv;
-  a.q_out = q_out;
-  a.k_out = k_out;
-  a.gamma_q = gamma_q;
-  a.gamma_k = gamma_k;
-  a.ld_qkv_bytes = ld_qkv * 2;
-  a.ld_out_bytes = 0;
-  a.rows = rows;
-  a.L = static_cast<int>(L);
-  a.n_video = static_cast<int>(n_video);
-  a.HW = static_cast<int>(H * W);
-  a.H = static_cast<int>(H);
-  a.W = static_cast<int>(W);
-  a.nvec_q = static_cast<int>(D * 2 / 16);
-  a.npairs = static_cast<int>(head_dim / 2);
-  a.sec_t = static_cast<int>(sec_t);
-  a.sec_th = static_cast<int>(sec_t + sec_h);
-  a.head_dim = static_cast<int>(head_dim);
-  a.eps = eps;
-  a.inv_hd = static_cast<float>(1.0 / static_cast<double>(head_dim));
-  a.theta = theta;
-  a.out_sb = sb;
-  a.out_sr = sr;
-  a.out_sh = sh;
-  a.q_scale = layout->q_scale;
-  a.k_scale = layout->k_scale;
-  a.n_heads = static_cast<int>(n_heads);
-  a.per_axis = layout->per_axis_freq;
-  const bool half = layout->half_split != 0;
-  cudaError_t e = int8 ? launch_qknorm_rope3d_ex_int8out(a, half, stream, nullptr)
-                       : launch_qknorm_rope3d_ex_bf16out(a, half, stream, nullptr);
-  if (e != cudaSuccess) return cuda_fail(e, "sol_qknorm_rope3d_ex launch");
-  if (quant_v) {
-    QuantArgs v{};
-    v.src = static_cast<const unsigned char *>(qkv) + 2 * D * 2;
-    v.ld_src_bytes = ld_qkv * 2;
-    v.out = layout->v_out;
-    v.scale = layout->v_scale;
-    v.out_sb = sb;
-    v.out_sr = sr;
-    v.out_sh = sh;
-    v.rows = rows;
-    v.L = static_cast<int>(L);
-    v.nvec = static_cast<int>(D * 2 / 16);
-    v.n_heads = static_cast<int>(n_heads);
-    e = launch_quantize_heads_int8(v, static_cast<int>(head_dim), stream, nullptr);
-    if (e != cudaSuccess) return cuda_fail(e, "sol_qknorm_rope3d_ex v quantisation launch");
-  }
-  return ok();
+sol_status sol_qknorm_rope3d_ex_tab(const void *qkv, int64_t ld_qkv, void *q_out, void *k_out,
+                                    const sol_qk_layout *layout, const void *gamma_q,
+                                    const void *gamma_k, const sol_rope_table *tab, int64_t B,
+                                    int64_t T, int64_t H, int64_t W, int64_t n_audio,
+                                    int64_t n_heads, float eps, sol_dtype dtype,
+                                    sol_stream_t stream) {
+  const char *fn = "sol_qknorm_rope3d_ex_tab";
+  sol_status st = check_table(fn, tab);
+  if (st != SOL_OK) return st;
+  if (layout && layout->per_axis_freq != tab->per_axis_freq)
+    return fail(SOL_ERR_INVALID_ARG,
+                "%s: layout.per_axis_freq (%d) differs from the table's (%d)", fn,
+                (int)layout->per_axis_freq, (int)tab->per_axis_freq);
+  return qk_ex(fn, qkv, ld_qkv, q_out, k_out, layout, gamma_q, gamma_k, tab, B, T, H, W,
+               n_audio, n_heads, tab->head_dim, tab->sec_t, tab->sec_h, tab->sec_w, eps,
+               tab->theta, dtype, stream);
 }
 
 size_t sol_gemm_gelu_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -646,92 +830,62 @@ sol_status sol_qknorm_rope3d(const void *qkv, int64_t ld_qkv, void *q_out, void 
                              int64_t T, int64_t H, int64_t W, int64_t n_audio, int64_t n_heads,
                              int64_t head_dim, int64_t sec_t, int64_t sec_h, int64_t sec_w,
                              float eps, float theta, sol_dtype dtype, sol_stream_t stream) {
-  if (dtype != SOL_F32 && dtype != SOL_BF16)
-    return fail(SOL_ERR_INVALID_ARG, "sol_qknorm_rope3d: unknown dtype %d", (int)dtype);
-  if (B < 0 || T < 0 || H < 0 || W < 0 || n_audio < 0)
-    return fail(SOL_ERR_INVALID_ARG, "sol_qknorm_rope3d: B, T, H, W, n_audio must be >= 0");
-  if (n_heads <= 0 || head_dim <= 0 || head_dim % 2 != 0)
-    return fail(SOL_ERR_INVALID_ARG,
-                "sol_qknorm_rope3d: need n_heads > 0 and an even head_dim > 0 (%lld, %lld)",
-                (long long)n_heads, (long long)head_dim);
-  if (sec_t < 0 || sec_h < 0 || sec_w < 0 || sec_t + sec_h + sec_w != head_dim / 2)
-    return fail(SOL_ERR_INVALID_ARG,
-                "sol_qknorm_rope3d: sections %lld+%lld+%lld must sum to head_dim/2 = %lld",
-                (long long)sec_t, (long long)sec_h, (long long)sec_w, (long long)(head_dim / 2));
-  if (!(eps >= 0.f) || !(theta > 0.f))
-    return fail(SOL_ERR_INVALID_ARG, "sol_qknorm_rope3d: need eps >= 0 and theta > 0");
-  if (T > kMaxRows || H > kMaxRows || W > kMaxRows || n_audio > kMaxRows || B > kMaxRows ||
-      H * W > kMaxRows || T * H * W > kMaxRows || T * H * W + n_audio > kMaxRows ||
-      B * (T * H * W + n_audio) > kMaxRows)
-    return fail(SOL_ERR_UNSUPPORTED, "sol_qknorm_rope3d: B*L and H*W must be below 2^31");
-  const int64_t n_video = T * H * W;
-  const int64_t L = n_video + n_audio;
-  const int64_t rows = B * L;
-  const int64_t D = n_heads * head_dim;
-  if (ld_qkv < 2 * D || ld_out < D)
-    return fail(SOL_ERR_INVALID_ARG, "sol_qknorm_rope3d: need ld_qkv >= 2*D and ld_out >= D");
-  if (rows == 0) return ok();
-  if (!qkv || !q_out || !k_out)
-    return fail(SOL_ERR_INVALID_ARG, "sol_qknorm_rope3d: qkv, q_out and k_out must be non-null");
-  const int es = esize_of(dtype);
-  const int64_t hd_bytes = head_dim * es;
-  const int64_t G = hd_bytes / 16;
-  if (hd_bytes % 16 != 0 || G < 2 || G > 32 || (G & (G - 1)) != 0)
-    return fail(SOL_ERR_UNSUPPORTED,
-                "sol_qknorm_rope3d: head_dim*%d bytes must be 16*G with G a power of two in "
-                "[2, 32] (head_dim=%lld)",
-                es, (long long)head_dim);
-  const int64_t ldq_b = ld_qkv * es, ldo_b = ld_out * es, D_b = D * es;
-  if (!aligned16(qkv) || !aligned16(q_out) || !aligned16(k_out) || ldq_b % 16 || ldo_b % 16 ||
-      (gamma_q && !aligned16(gamma_q)) || (gamma_k && !aligned16(gamma_k)))
-    return fail(SOL_ERR_MISALIGNED,
-                "sol_qknorm_rope3d: pointers and row strides must be 16-byte aligned");
-  if (2 * D_b > kMaxRowBytesQk)
-    return fail(SOL_ERR_UNSUPPORTED, "sol_qknorm_rope3d: 2*D=%lld exceeds %lld elements",
-                (long long)(2 * D), (long long)(kMaxRowBytesQk / es));
-  const bool in_place = q_out == qkv && ld_out == ld_qkv &&
-                        static_cast<const unsigned char *>(k_out) ==
-                            static_cast<const unsigned char *>(qkv) + D_b;
-  if (!in_place) {
-    if (!strided_disjoint(qkv, 2 * D_b, q_out, D_b, rows, ldq_b, ldo_b) ||
-        !strided_disjoint(qkv, 2 * D_b, k_out, D_b, rows, ldq_b, ldo_b) ||
-        !strided_disjoint(q_out, D_b, k_out, D_b, rows, ldo_b, ldo_b))
-      return fail(SOL_ERR_INVALID_ARG,
-                  "sol_qknorm_rope3d: outputs must be exactly in place (q_out=qkv, "
-                  "k_out=qkv+D, ld_out=ld_qkv) or overlap neither qkv nor each other");
-  }
-  for (const void *g : {gamma_q, gamma_k}) {
-    if (!g) continue;
-    Span gs = span_of(g, 1, 0, hd_bytes);
-    if (spans_overlap(gs, span_of(q_out, rows, ldo_b, D_b)) ||
-        spans_overlap(gs, span_of(k_out, rows, ldo_b, D_b)))
-      return fail(SOL_ERR_INVALID_ARG, "sol_qknorm_rope3d: an output overlaps gamma");
-  }
-
+  const char *fn = "sol_qknorm_rope3d";
   QkArgs a{};
-  a.qkv = qkv;
-  a.q_out = q_out;
-  a.k_out = k_out;
-  a.gamma_q = gamma_q;
-  a.gamma_k = gamma_k;
-  a.ld_qkv_bytes = ldq_b;
-  a.ld_out_bytes = ldo_b;
-  a.rows = rows;
-  a.L = static_cast<int>(L);
-  a.n_video = static_cast<int>(n_video);
-  a.HW = static_cast<int>(H * W);
-  a.H = static_cast<int>(H);
-  a.W = static_cast<int>(W);
-  a.nvec_q = static_cast<int>(D_b / 16);
-  a.npairs = static_cast<int>(head_dim / 2);
-  a.sec_t = static_cast<int>(sec_t);
-  a.sec_th = static_cast<int>(sec_t + sec_h);
-  a.head_dim = static_cast<int>(head_dim);
-  a.eps = eps;
-  a.inv_hd = static_cast<float>(1.0 / static_cast<double>(head_dim));
-  a.theta = theta;
+  bool empty = false;
+  sol_status st = check_qk(fn, qkv, ld_qkv, q_out, k_out, ld_out, gamma_q, gamma_k, B, T, H, W,
+                           n_audio, n_heads, head_dim, sec_t, sec_h, sec_w, eps, theta, dtype, a,
+                           empty);
+  if (st != SOL_OK || empty) return st;
   cudaError_t e = launch_qknorm_rope3d(a, dtype == SOL_F32 ? 0 : 1, stream, nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "sol_qknorm_rope3d launch");
+  return ok();
+}
+
+size_t sol_rope_table_bytes(int64_t n_pos, int64_t head_dim) {
+  if (n_pos < 0 || n_pos > kMaxRows || head_dim < 2 || head_dim > 2 * kMaxRotaryPairs ||
+      head_dim % 2 != 0)
+    return 0;
+  return static_cast<size_t>(n_pos) * static_cast<size_t>(head_dim) * 4u;
+}
+
+sol_status sol_rope_table_build(const sol_rope_table *tab, sol_stream_t stream) {
+  const char *fn = "sol_rope_table_build";
+  sol_status st = check_table(fn, tab);
+  if (st != SOL_OK) return st;
+  if (tab->n_pos == 0) return ok();
+  cudaError_t e = launch_rope_table(tab->data, static_cast<int>(tab->n_pos),
+                                    static_cast<int>(tab->head_dim / 2),
+                                    static_cast<int>(tab->head_dim), static_cast<int>(tab->sec_t),
+                                    static_cast<int>(tab->sec_t + tab->sec_h), tab->theta,
+                                    tab->per_axis_freq, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_rope_table_build launch");
+  return ok();
+}
+
+sol_status sol_qknorm_rope3d_tab(const void *qkv, int64_t ld_qkv, void *q_out, void *k_out,
+                                 int64_t ld_out, const void *gamma_q, const void *gamma_k,
+                                 const sol_rope_table *tab, int64_t B, int64_t T, int64_t H,
+                                 int64_t W, int64_t n_audio, int64_t n_heads, float eps,
+                                 sol_dtype dtype, sol_stream_t stream) {
+  const char *fn = "sol_qknorm_rope3d_tab";
+  sol_status st = check_table(fn, tab);
+  if (st != SOL_OK) return st;
+  QkArgs a{};
+  bool empty = false;
+  st = check_qk(fn, qkv, ld_qkv, q_out, k_out, ld_out, gamma_q, gamma_k, B, T, H, W, n_audio,
+                n_heads, tab->head_dim, tab->sec_t, tab->sec_h, tab->sec_w, eps, tab->theta,
+                dtype, a, empty);
+  if (st != SOL_OK || empty) return st;
+  const int es = esize_of(dtype);
+  const int64_t D_b = n_heads * tab->head_dim * es;
+  st = check_table_use(fn, tab, T, H, W, n_audio,
+                       {span_of(q_out, a.rows, a.ld_out_bytes, D_b),
+                        span_of(k_out, a.rows, a.ld_out_bytes, D_b)});
+  if (st != SOL_OK) return st;
+  a.rope_tab = tab->data;
+  cudaError_t e = launch_qknorm_rope3d(a, dtype == SOL_F32 ? 0 : 1, stream, nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_qknorm_rope3d_tab launch");
   return ok();
 }
 

@@ -161,6 +161,45 @@ __device__ __forceinline__ void cta_rows(int64_t rows, int64_t cta, int64_t ctas
   count = static_cast<int>(rows * (cta + 1) / ctas - begin);
 }
 
+// The rows one CTA streams, in order.  K == 0: the CTA's contiguous share
+// (cta_rows).  K > 0: chunks of K consecutive rows dealt round-robin, chunk
+// c to CTA c mod gridDim.x, so that at any moment the grid works through one
+// contiguous window of about K * gridDim.x rows instead of gridDim.x
+// far-apart streams.  Rows within a chunk (or a share) are consecutive.
+template <int K>
+struct RowOrder {
+  int64_t begin;  // K == 0: first row of the share
+  int count;      // rows of this CTA
+  __device__ __forceinline__ void init(int64_t rows) {
+    if constexpr (K == 0) {
+      cta_rows(rows, blockIdx.x, gridDim.x, begin, count);
+    } else {
+      const int64_t chunks = (rows + K - 1) / K, c = blockIdx.x, g = gridDim.x;
+      const int64_t mine = c < chunks ? (chunks - 1 - c) / g + 1 : 0;
+      int64_t n = mine * K;
+      if (mine > 0 && c + (mine - 1) * g == chunks - 1) n -= chunks * K - rows;  // last chunk
+      begin = 0;
+      count = static_cast<int>(n);
+    }
+  }
+  // global index of the CTA's j-th row
+  __device__ __forceinline__ int64_t row(int j) const {
+    if constexpr (K == 0) {
+      return begin + j;
+    } else {
+      return (static_cast<int64_t>(j / K) * gridDim.x + blockIdx.x) * K + j % K;
+    }
+  }
+  // row j is the first of a run of consecutive rows (row cursors restart)
+  __device__ __forceinline__ bool run_start(int j) const {
+    if constexpr (K == 0) {
+      return j == 0;
+    } else {
+      return j % K == 0;
+    }
+  }
+};
+
 // (sample b, row r in the sample) of a global row, advanced one row at a
 // time: one division per CTA instead of one per row.  L < 2^31.
 struct TokenCursor {

@@ -109,6 +109,9 @@ struct QkArgs {
   float *k_scale;
   int n_heads;
   int per_axis;  // 1: each rotary section its own frequency ladder, theta^(-j/s)
+  // table-driven kernels only: rotary table, row p = cos(p*f_i) for every pair
+  // i, then sin(p*f_i) (2*npairs floats per row), rows 0 .. n_pos-1
+  const float *rope_tab;
 };
 
 // Per-head symmetric INT8 quantisation of rows of bf16 head vectors (the v
@@ -184,7 +187,13 @@ inline cudaError_t launch_qknorm_rope3d(const QkArgs &a, int dtype, cudaStream_t
                     : launch_qknorm_rope3d_bf16(a, stream, geo);
 }
 
+// Rotary table (row p: cos(p*f_i) for every pair i, then sin(p*f_i)) for the
+// table-driven QKNorm + RoPE kernels, computed in fp64, rounded to fp32.
+cudaError_t launch_rope_table(float *tab, int n_pos, int npairs, int head_dim, int sec_t,
+                              int sec_th, double theta, int per_axis, cudaStream_t stream);
+
 // Limits the launchers accept (checked by the ABI before calling them).
+constexpr int64_t kMaxRotaryPairs = 128;     // head_dim <= 256
 constexpr int kMaxThreads = 256;
 constexpr int64_t kMaxRows = 0x7fffffff;  // B*L, L, H*W: 32-bit row bookkeeping
 constexpr int kMaxVpt = 8;
