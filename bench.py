@@ -18,10 +18,8 @@ of these operations) on the host cores, one process per core, one bounded
 sample of clip rows per process per step; under torchrun only rank 0 runs it.
 """
 import argparse
-import hashlib
 import json
 import os
-import re
 import subprocess
 import sys
 import tempfile
@@ -34,7 +32,7 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from video_diffusion_transformer_rms_b200 import dist  # noqa: E402
+from video_diffusion_transformer_rms_b200 import dist, traffic  # noqa: E402
 from video_diffusion_transformer_rms_b200.workloads import (WORKLOADS, activation,  # noqa: E402
                                                             make_inputs, to_oracle_array,
                                                             vectors)
@@ -42,12 +40,17 @@ from video_diffusion_transformer_rms_b200.workloads import (WORKLOADS, activatio
 METRIC = "tokens/s and achieved HBM GB/s (% of B200 peak) per fused kernel, 1 GPU"
 WORKLOAD = "clip5s"
 KERNELS = ("rms_adaln", "qknorm_rope3d", "gate_residual")
-_COMMON_SOURCES = ["sol_device.cuh", "sol_launch.h", "sol_abi.cu"]
-KERNEL_SOURCES = {
-    "rms_adaln": ["rms_adaln.cu"] + _COMMON_SOURCES,
-    "gate_residual": ["gate_residual.cu"] + _COMMON_SOURCES,
-    "qknorm_rope3d": ["qknorm_rope3d.cuh", "qknorm_rope3d_bf16.cu"] + _COMMON_SOURCES,
-}
+# Where the step's QKNorm + RoPE gets its (cos, sin): False = per row, on the
+# fly (sol_qknorm_rope3d); True = a rotary table built once per clip shape
+# (sol_qknorm_rope3d_tab).  The other one is timed beside the step.
+QK_TABLE = False
+# the traffic record (profiles/traffic.json) of the kernel each step name runs
+TRAFFIC_NAME = {"rms_adaln": "rms_adaln", "gate_residual": "gate_residual",
+                "qknorm_rope3d": "qknorm_rope3d_tab" if QK_TABLE else "qknorm_rope3d"}
+# every config of the task, each step kernel timed on its own (clip5s is the
+# headline step above)
+PER_CONFIG = ("medium", "clip5s", "clip15s", "cfg5s", "cfg5s_d3072")
+L2_FLUSH_BYTES = 256 << 20   # written between reps where the inputs fit in L2
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -79,7 +82,8 @@ def workload_config(w, n_gpus):
         "global_tokens_per_step": w.rows * n_gpus,
         "D": w.D,
         "io_dtype": w.dtype,
-        "step": "rms_adaln + qknorm_rope3d + gate_residual, one launch each",
+        "step": "rms_adaln + qknorm_rope3d" + ("_tab" if QK_TABLE else "") +
+                " + gate_residual, one launch each",
         "l2": "no flush: every input is larger than the 126 MB L2 (1.3-3.9 GB per tensor)",
         "parallelism": f"{n_gpus} independent shards (one clip per GPU), no data-path collective",
         "inputs": "seeded synthetic N(0,1) activations with 1% outlier channels x20",
@@ -99,27 +103,10 @@ def load_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_sha(kernel):
-    h = hashlib.sha256()
-    for f in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, "video_diffusion_transformer_rms_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
-    return h.hexdigest()
-
-
 def traffic_record(kernel, workload):
-    """DRAM bytes per launch from the committed ncu summary, or None if there
-    is none or the kernel source changed since it was taken."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
-    try:
-        text = open(path).read()
-    except OSError:
-        return None
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    s = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
-    if not m or not s or s.group(1) != kernel_source_sha(kernel):
-        return None
-    return float(m.group(1))
+    """DRAM bytes per full-size launch from profiles/traffic.json, or None if
+    there is no record or the kernel's sources changed since it was taken."""
+    return traffic.lookup(TRAFFIC_NAME.get(kernel, kernel), workload, ROOT)
 
 
 class ClockSampler:
@@ -326,11 +313,24 @@ def run_ours(args):
         return _abi.sol_rms_adaln(p["x"], y.data_ptr(), p["scale"], p["shift"], None, w.B, w.L,
                                   w.n_video, D, w.eps, dt, s)
 
-    def k_qk():
+    # rotary table of the clip's positions, built once per shape (like a
+    # model's RoPE cache) before any timed step; its build is timed apart
+    table = api.RopeTable.for_grid(w.T, w.H, w.W, w.n_audio, w.head_dim, sections=w.sections,
+                                   theta=w.theta, device=dev)
+    tab_ms = time_launches(lambda: _abi.sol_rope_table_build(table.desc, s), stream, 20)
+
+    def k_qk_otf():
         return _abi.sol_qknorm_rope3d(p["qkv"], 3 * D, qk.data_ptr(), qk.data_ptr() + D * 2,
                                       ld_out, p["gamma_q"], p["gamma_k"], w.B, w.T, w.H, w.W,
                                       w.n_audio, w.n_heads, w.head_dim, st, sh_, sw, w.eps,
                                       w.theta, dt, s)
+
+    def k_qk_tab():
+        return _abi.sol_qknorm_rope3d_tab(p["qkv"], 3 * D, qk.data_ptr(), qk.data_ptr() + D * 2,
+                                          ld_out, p["gamma_q"], p["gamma_k"], table.desc, w.B,
+                                          w.T, w.H, w.W, w.n_audio, w.n_heads, w.eps, dt, s)
+
+    k_qk = k_qk_tab if QK_TABLE else k_qk_otf
 
     def k_gate():
         return _abi.sol_gate_residual(p["h"], p["branch"], p["gate"], out.data_ptr(), w.B, w.L,
@@ -396,12 +396,20 @@ def run_ours(args):
                                vs8.data_ptr())
 
     def k_qk_ex(lay, q_ptr, k_ptr):
+        if QK_TABLE:
+            return lambda: _abi.sol_qknorm_rope3d_ex_tab(
+                p["qkv"], 3 * D, q_ptr, k_ptr, lay, p["gamma_q"], p["gamma_k"], table.desc, w.B,
+                w.T, w.H, w.W, w.n_audio, w.n_heads, w.eps, dt, s)
         return lambda: _abi.sol_qknorm_rope3d_ex(
             p["qkv"], 3 * D, q_ptr, k_ptr, lay, p["gamma_q"], p["gamma_k"], w.B, w.T, w.H, w.W,
             w.n_audio, w.n_heads, hd, st, sh_, sw, w.eps, w.theta, dt, s)
 
     row = D * w.esize  # bytes of one D-wide bf16 row
     extra = {
+        # the other source of (cos, sin) for the step's QKNorm + RoPE: per row,
+        # on the fly (fp64 angle reduction, sincosf, a CTA barrier per stage)
+        ("qknorm_rope3d_table" if not QK_TABLE else "qknorm_rope3d_otf"):
+            (4 * row, k_qk_otf if QK_TABLE else k_qk_tab),
         # h_out = h + gate*branch and y = RMS-AdaLN(h_out) in one pass: 4 D-wide rows
         "gate_residual_rms_adaln": (4 * row, lambda: _abi.sol_gate_residual_rms_adaln(
             p["h"], p["branch"], p["gate"], out.data_ptr(), y.data_ptr(), p["scale"],
@@ -431,18 +439,7 @@ def run_ours(args):
     }
     next_rows = {}
     for name, (bytes_per_row, fn) in extra.items():
-        for _ in range(5):
-            _abi.check(fn())
-        n_it = 200
-        ea = torch.cuda.Event(enable_timing=True)
-        eb = torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        ea.record(stream)
-        for _ in range(n_it):
-            _abi.check(fn())
-        eb.record(stream)
-        torch.cuda.synchronize()
-        ms = dist.max_over_ranks(ea.elapsed_time(eb) / n_it)
+        ms = dist.max_over_ranks(time_launches(fn, stream, 200))
         nbytes = bytes_per_row * w.rows
         next_rows[name] = {"ms": round(ms, 4), "tokens_per_s": round(w.rows / (ms / 1e3)),
                            "bytes_per_token": bytes_per_row,
@@ -450,11 +447,14 @@ def run_ours(args):
     del ws, q8, s8, v8, vs8
     next_rows["gemm_gelu"] = time_gemm_gelu(w, D, dev, stream)
 
+    # ---- every config: each step kernel on its own --------------------------
+    peak, peak_kind = load_peak()
+    configs = {c: time_config(WORKLOADS[c], dev, stream, peak) for c in PER_CONFIG}
+
     # ---- end to end through the public API, host buffers ------------------
-    e2e = run_e2e(args, w, t, stream, api)
+    e2e = run_e2e(args, w, t, stream, api, table if QK_TABLE else None)
     e2e_value, _, _ = dist.job_throughput(w.rows * e2e["steps"], e2e["seconds"])
 
-    peak, peak_kind = load_peak()
     bpr = w.bytes_per_row()
     kernels = {}
     for name in KERNELS:
@@ -487,11 +487,19 @@ def run_ours(args):
             "data": "synthetic (seeded; no dataset or weights involved)",
             "config": workload_config(w, world),
             "roofline": roofline, "kernels": kernels, "next_rows": next_rows,
+            "configs": configs,
+            "rope_table": {"n_pos": table.n_pos, "bytes": table.n_pos * w.head_dim * 4,
+                           "build_ms": round(tab_ms, 4),
+                           "note": "built once per clip shape before the timed steps (a "
+                                   "RoPE cache); the step's QKNorm + RoPE reads it"
+                           if QK_TABLE else "not used by the step"},
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                     "steps": e2e["steps"],
-                    "path": "pinned host inputs -> H2D -> api.rms_adaln / api.qknorm_rope3d / "
+                    "path": "pinned host inputs -> H2D -> api.rms_adaln / api.qknorm_rope3d"
+                            + (" (rotary table built once, outside the steps)" if QK_TABLE
+                               else "") + " / "
                             "api.gate_residual -> D2H of y, q, k, out; of the merged QKV rows "
                             "only the q and k columns the step reads are copied (one pitched "
                             "copy); copy-in, kernels and copy-out on three streams ordered by "
@@ -502,6 +510,88 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     dist.barrier()
     dist.shutdown()
+
+
+def time_launches(fn, stream, n, warmup=5):
+    """Mean ms of n back-to-back launches of fn on `stream` (CUDA events)."""
+    from video_diffusion_transformer_rms_b200 import _abi
+    for _ in range(warmup):
+        _abi.check(fn())
+    ea = torch.cuda.Event(enable_timing=True)
+    eb = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    ea.record(stream)
+    for _ in range(n):
+        _abi.check(fn())
+    eb.record(stream)
+    torch.cuda.synchronize()
+    return ea.elapsed_time(eb) / n
+
+
+def time_config(w, dev, stream, peak, reps=20, warmup=3):
+    """The step's three kernels on one config, each timed on its own: CUDA
+    events around every launch, median over `reps`.  Where an activation is
+    under 1 GB (the medium case, whose tensors are L2-sized), the reps are
+    separated by an L2 flush: 256 MB written, then another 256 MB read, so the
+    timed launch starts with no lines of its inputs and no dirty lines in L2.
+    The larger configs stream several GB per launch and need no flush."""
+    from video_diffusion_transformer_rms_b200 import _abi, api
+    t = make_inputs(w, dev)
+    D = w.D
+    p = {k: v.data_ptr() for k, v in t.items()}
+    y = torch.empty_like(t["x"])
+    out = torch.empty_like(t["h"])
+    qk = torch.empty((w.rows, 2 * D), dtype=t["qkv"].dtype, device=dev)
+    table = api.RopeTable.for_grid(w.T, w.H, w.W, w.n_audio, w.head_dim, sections=w.sections,
+                                   theta=w.theta, device=dev)
+    dt = _abi.SOL_BF16 if w.dtype == "bf16" else _abi.SOL_F32
+    s = stream.cuda_stream
+    st, sh, sw = w.sections
+    fns = {
+        "rms_adaln": lambda: _abi.sol_rms_adaln(p["x"], y.data_ptr(), p["scale"], p["shift"],
+                                                None, w.B, w.L, w.n_video, D, w.eps, dt, s),
+        "qknorm_rope3d": (lambda: _abi.sol_qknorm_rope3d_tab(
+            p["qkv"], 3 * D, qk.data_ptr(), qk.data_ptr() + 2 * D, 2 * D, p["gamma_q"],
+            p["gamma_k"], table.desc, w.B, w.T, w.H, w.W, w.n_audio, w.n_heads, w.eps, dt, s))
+        if QK_TABLE else (lambda: _abi.sol_qknorm_rope3d(
+            p["qkv"], 3 * D, qk.data_ptr(), qk.data_ptr() + 2 * D, 2 * D, p["gamma_q"],
+            p["gamma_k"], w.B, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, st, sh, sw,
+            w.eps, w.theta, dt, s)),
+        "gate_residual": lambda: _abi.sol_gate_residual(p["h"], p["branch"], p["gate"],
+                                                        out.data_ptr(), w.B, w.L, w.n_video, D,
+                                                        dt, s),
+    }
+    flush = w.rows * D * w.esize < (1 << 30)
+    if flush:
+        fw = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        fr = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    bpr = w.bytes_per_row()
+    res = {"tokens": w.rows, "B": w.B, "D": D, "l2_flush": bool(flush), "reps": reps,
+           "kernels": {}}
+    for name, fn in fns.items():
+        for _ in range(warmup):
+            _abi.check(fn())
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        for a, b in evs:
+            if flush:
+                fw.fill_(1.0)
+                fr.sum()
+            a.record(stream)
+            _abi.check(fn())
+            b.record(stream)
+        torch.cuda.synchronize()
+        ms = float(np.median([a.elapsed_time(b) for a, b in evs]))
+        ms = dist.max_over_ranks(ms)
+        gbs = bpr[name] * w.rows / (ms / 1e3) / 1e9
+        res["kernels"][name] = {"ms": round(ms, 4), "tokens_per_s": round(w.rows / (ms / 1e3)),
+                                "GB_per_s": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
+                                "frac_of_8TBs_nominal": round(gbs / NOMINAL_HBM_GBS, 4)}
+    del t, y, out, qk, table
+    if flush:
+        del fw, fr
+    torch.cuda.empty_cache()
+    return res
 
 
 def load_tensor_peaks():
@@ -556,7 +646,7 @@ def time_gemm_gelu(w, D, dev, stream):
             "tokens_per_s": round(M / (ms / 1e3))}
 
 
-def run_e2e(args, w, t, stream, api):
+def run_e2e(args, w, t, stream, api, table=None):
     """Same step through the public tensor API, inputs copied every step
     from pinned host memory and every output copied back.
 
@@ -614,7 +704,7 @@ def run_e2e(args, w, t, stream, api):
             api.qknorm_rope3d(dev["qkv"].view(w.B, w.L, 2 * D), w.T, w.H, w.W, w.n_audio,
                               w.n_heads, w.head_dim, w.sections, dev["gamma_q"],
                               dev["gamma_k"], w.eps, w.theta, q_out=qk[..., :D],
-                              k_out=qk[..., D:], stream=stream)
+                              k_out=qk[..., D:], stream=stream, table=table)
         else:
             api.gate_residual(dev["h"].view(w.B, w.L, D), dev["branch"].view(w.B, w.L, D),
                               dev["gate"], w.n_video, out=out, stream=stream)

@@ -1,6 +1,7 @@
 """bench.py host logic on CPU: the clock-sample summary that decides whether a
 run was throttled, and the ncu traffic record that is used only while the
 kernel sources still match the hash recorded with it."""
+import json
 import os
 import shutil
 import time
@@ -8,6 +9,7 @@ import time
 import pytest
 
 import bench
+from video_diffusion_transformer_rms_b200 import traffic
 
 
 def _line(ts, uuid, sm, smax, reasons=("Not Active",) * 4):
@@ -41,18 +43,45 @@ def test_clock_summary_reports_hardware_slowdown_and_empty_input():
 
 
 def test_traffic_record_only_while_the_sources_match(tmp_path, monkeypatch):
-    # a copy of the tree's kernel sources and one summary under a temporary root
+    # a copy of the tree's kernel sources and one record under a temporary root
     csrc = os.path.join(bench.ROOT, "video_diffusion_transformer_rms_b200", "csrc")
     dst = tmp_path / "video_diffusion_transformer_rms_b200" / "csrc"
     shutil.copytree(csrc, dst)
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    sha = bench.kernel_source_sha("rms_adaln")
-    (tmp_path / "profiles" / "rms_adaln_clip5s.md").write_text(
-        f"traffic_bytes_per_launch: 2.5e+09\nsource_sha256: {sha}\n")
+    rec = {"rms_adaln": {"workload": "clip5s", "traffic_bytes_per_launch": 2.5e9,
+                         "source_sha256": traffic.source_sha("rms_adaln", str(tmp_path))}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
     assert bench.traffic_record("rms_adaln", "clip5s") == pytest.approx(2.5e9)
+    assert bench.traffic_record("rms_adaln", "clip15s") is None  # another workload
     # any change to a source the kernel is built from voids the record
     with open(dst / "rms_adaln.cu", "a") as f:
         f.write("\n// edited\n")
     assert bench.traffic_record("rms_adaln", "clip5s") is None
-    assert bench.traffic_record("gate_residual", "clip5s") is None  # no summary at all
+    assert bench.traffic_record("gate_residual", "clip5s") is None  # no record at all
+
+
+NCU_CSV = """==PROF== Connected to process 1234
+"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"
+"0","1","python","h","void sol::qk::qknorm_rope3d_kernel<...>(sol::QkArgs)","1","7","(256, 1, 1)","(296, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","Mbyte","668.10"
+"0","1","python","h","void sol::qk::qknorm_rope3d_kernel<...>(sol::QkArgs)","1","7","(256, 1, 1)","(296, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","Mbyte","660.00"
+"1","1","python","h","void sol::qk::qknorm_rope3d_kernel<...>(sol::QkArgs)","1","7","(256, 1, 1)","(296, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","Gbyte","0.6719"
+"1","1","python","h","void sol::qk::qknorm_rope3d_kernel<...>(sol::QkArgs)","1","7","(256, 1, 1)","(296, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","664000000"
+"""
+
+
+def test_traffic_record_from_an_ncu_csv(tmp_path):
+    # per-launch DRAM bytes from ncu's CSV (units converted, launches
+    # averaged), scaled from the captured slice to the full workload
+    path = tmp_path / "dram.csv"
+    path.write_text(NCU_CSV)
+    launches = traffic.parse_ncu_csv(str(path))
+    assert len(launches) == 2
+    assert launches[0][1:] == pytest.approx((668.10e6, 660.0e6))
+    assert launches[1][1:] == pytest.approx((671.9e6, 664.0e6))
+    rec = traffic.make_record(launches, "qknorm_rope3d_tab", "clip5s", 32768, 4 * 32768, "cmd")
+    assert rec["traffic_bytes_per_launch"] == pytest.approx(4 * (670.0e6 + 662.0e6))
+    assert rec["launches"] == 2 and rec["captured_rows"] == 32768
+    assert rec["source_sha256"] == traffic.source_sha("qknorm_rope3d_tab")
+    with pytest.raises(ValueError):
+        traffic.make_record([], "rms_adaln", "clip5s", 1, 1, "cmd")

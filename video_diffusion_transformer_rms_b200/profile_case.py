@@ -2,7 +2,8 @@
 for profilers (ncu) that should capture a small, self-contained case.
 
     python -m video_diffusion_transformer_rms_b200.profile_case \
-        [--workload clip5s] [--frames 4] [--launches 1] [--kernel norm|gemm|qk_bhsd|qk_half|qk_int8|qk_all|next]
+        [--workload clip5s] [--frames 4] [--launches 1]
+        [--kernel norm|rms|gate|qk|qk_tab|gemm|qk_bhsd|qk_half|qk_int8|qk_all|next] [--table]
 
 The slice keeps the clip's H x W latent grid, D and head layout, takes the
 first `--frames` latent frames (T) and scales the audio rows by the same
@@ -15,6 +16,11 @@ runs the MLP up-projection with fused GELU on the same slice instead
 half-split pairs, INT8 output; qk_all runs the first two and INT8 with the
 quantised v, one launch each), and `--kernel next` the fused residual +
 RMS-AdaLN and the change detector (read-only, then with the cache refresh).
+`--kernel norm` runs the step's three kernels; `rms`, `gate`, `qk` (per-row
+cos/sin) and `qk_tab` (rotary table) one of them alone, for captures that
+must hold a single kernel.  `--table` makes the qk_* variants read a rotary
+table too.  The slice prints its row count (the scale factor to the full
+workload's traffic).
 """
 import argparse
 import dataclasses
@@ -31,7 +37,10 @@ def main():
     ap.add_argument("--frames", type=int, default=4)
     ap.add_argument("--launches", type=int, default=1)
     ap.add_argument("--kernel", default="norm",
-                    choices=["norm", "gemm", "qk_bhsd", "qk_half", "qk_int8", "qk_all", "next"])
+                    choices=["norm", "rms", "gate", "qk", "qk_tab", "gemm", "qk_bhsd", "qk_half",
+                             "qk_int8", "qk_all", "next"])
+    ap.add_argument("--table", action="store_true",
+                    help="QKNorm+RoPE variants read a precomputed rotary table")
     args = ap.parse_args()
     full = WORKLOADS[args.workload]
     T = max(1, min(full.T, args.frames))
@@ -48,6 +57,24 @@ def main():
     y = torch.empty_like(x)
     out = torch.empty_like(h)
     qk = torch.empty((w.B, w.L, 2 * D), dtype=qkv.dtype, device=qkv.device)
+    table = None
+    if args.table or args.kernel == "qk_tab":
+        table = api.RopeTable.for_grid(w.T, w.H, w.W, w.n_audio, w.head_dim, sections=w.sections,
+                                       theta=w.theta, device=qkv.device)
+    if args.kernel in ("rms", "gate", "qk", "qk_tab"):
+        for _ in range(args.launches):
+            if args.kernel == "rms":
+                api.rms_adaln(x, t["scale"], t["shift"], w.n_video, eps=w.eps, out=y)
+            elif args.kernel == "gate":
+                api.gate_residual(h, br, t["gate"], w.n_video, out=out)
+            else:
+                api.qknorm_rope3d(qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim,
+                                  w.sections, t["gamma_q"], t["gamma_k"], w.eps, w.theta,
+                                  q_out=qk[..., :D], k_out=qk[..., D:],
+                                  table=table if args.kernel == "qk_tab" else None)
+        torch.cuda.synchronize()
+        print(f"{w.name}: {w.rows} rows, D={D}, {args.launches} launch(es) of {args.kernel}")
+        return
     if args.kernel == "next":
         ws = torch.empty(_abi.sol_residual_change_workspace_bytes(w.B), dtype=torch.uint8,
                          device=x.device)
@@ -66,9 +93,11 @@ def main():
                                {"int8": True, "quantize_v": True}]}[args.kernel]
         for _ in range(args.launches):
             for opts in variants:
+                if table is not None and opts.get("per_axis_freq"):
+                    raise SystemExit("per-axis variants need a per-axis table")
                 api.qknorm_rope3d_ex(qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim,
                                      w.sections, t["gamma_q"], t["gamma_k"], w.eps, w.theta,
-                                     **opts)
+                                     table=table, **opts)
         torch.cuda.synchronize()
         print(f"{w.name}: {w.rows} rows, D={D}, {args.launches} launch(es) of {args.kernel}")
         return
@@ -76,7 +105,7 @@ def main():
         api.rms_adaln(x, t["scale"], t["shift"], w.n_video, eps=w.eps, out=y)
         api.qknorm_rope3d(qkv, w.T, w.H, w.W, w.n_audio, w.n_heads, w.head_dim, w.sections,
                           t["gamma_q"], t["gamma_k"], w.eps, w.theta, q_out=qk[..., :D],
-                          k_out=qk[..., D:])
+                          k_out=qk[..., D:], table=table)
         api.gate_residual(h, br, t["gate"], w.n_video, out=out)
     torch.cuda.synchronize()
     print(f"{w.name}: {w.rows} rows, D={D}, {args.launches} launch(es) of each kernel")
