@@ -43,7 +43,7 @@ KERNELS = ("rms_adaln", "qknorm_rope3d", "gate_residual")
 # Where the step's QKNorm + RoPE gets its (cos, sin): False = per row, on the
 # fly (sol_qknorm_rope3d); True = a rotary table built once per clip shape
 # (sol_qknorm_rope3d_tab).  The other one is timed beside the step.
-QK_TABLE = False
+QK_TABLE = True
 # the traffic record (profiles/traffic.json) of the kernel each step name runs
 TRAFFIC_NAME = {"rms_adaln": "rms_adaln", "gate_residual": "gate_residual",
                 "qknorm_rope3d": "qknorm_rope3d_tab" if QK_TABLE else "qknorm_rope3d"}

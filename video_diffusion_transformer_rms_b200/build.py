@@ -21,8 +21,10 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsol.so")
 
 SOURCES = ["sol_abi.cu", "rms_adaln.cu", "gate_residual.cu", "qknorm_rope3d_bf16.cu",
-           "qknorm_rope3d_f32.cu", "qknorm_rope3d_ex_bf16.cu", "qknorm_rope3d_ex_int8.cu",
-           "residual_change.cu", "quantize_heads.cu", "rope_table.cu", "gemm_gelu.cu"]
+           "qknorm_rope3d_f32.cu", "qknorm_rope3d_tab_bf16.cu", "qknorm_rope3d_tab_f32.cu",
+           "qknorm_rope3d_ex_bf16.cu", "qknorm_rope3d_ex_int8.cu", "qknorm_rope3d_ex_tab_bf16.cu",
+           "qknorm_rope3d_ex_tab_int8.cu", "residual_change.cu", "quantize_heads.cu",
+           "rope_table.cu", "gemm_gelu.cu"]
 # sources built against the CUTLASS / CuTe headers (the sm100 GEMM templates)
 CUTLASS_SOURCES = {"gemm_gelu.cu"}
 HEADERS = ["sol_device.cuh", "sol_launch.h", "qknorm_rope3d.cuh", "qknorm_rope3d_ex.cuh"]

@@ -333,36 +333,67 @@ cudaError_t launch_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
   return cudaGetLastError();
 }
 
+// Row order and ring of the two forms, measured at the 5 s clip on a B200
+// at 1,965 MHz, 20-step runs after idling:
+//  - Rows go to the CTAs in chunks dealt round-robin, so the whole grid
+//    works through one contiguous window of the tensors; a contiguous share
+//    per CTA (296 far-apart streams) ran in a slower DRAM mode, 0.91-0.92 ms
+//    against 0.79-0.83 ms.
+//  - On the fly: two rows per stage, two stages (the angle tables already
+//    put one CTA barrier on every stage), chunks of 8 rows.
+//  - Table-driven: one row per stage, three stages, chunks of 4 rows, and a
+//    CTA barrier per stage although nothing is shared: it keeps the CTA's
+//    warps on the same row, so each row is requested as one burst (0.84
+//    against 0.90 ms without it at 256 x 3; 0.80 ms at 320 x 2).
+constexpr int kOtfChunk = 8;
+constexpr int kTabRows = 1;
+constexpr int kTabStages = 3;
+constexpr int kTabChunk = 4;
+
 template <typename T, int G, int NT, int VPT>
 cudaError_t launch(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
   constexpr int R = VPT <= 6 ? 2 : 1;  // keeps the ring within shared memory
-  return launch_cfg<T, G, NT, VPT, R, 2, false>(a, stream, geo);
+  return launch_cfg<T, G, NT, VPT, R, 2, false, kOtfChunk, false>(a, stream, geo);
 }
 
-// Table-driven kernels: with no barrier and no angle tables the ring runs
-// one row per stage, three stages deep (two rows in flight per CTA).
-constexpr int kTabRows = 1;
-constexpr int kTabStages = 3;
+template <typename T, int G>
+cudaError_t dispatch(const QkArgs &a, int threads, int vpt, cudaStream_t stream, Geometry *geo) {
+#define SOL_CASE(NT, V) \
+  if (threads == NT && vpt == V) return launch<T, G, NT, V>(a, stream, geo);
+  SOL_QK_OTF_SPLITS(SOL_CASE)
+#undef SOL_CASE
+  return cudaErrorInvalidValue;
+}
 
 template <typename T, int G>
 cudaError_t dispatch_tab(const QkArgs &a, int threads, int vpt, cudaStream_t stream,
                          Geometry *geo) {
 #define SOL_CASE(NT, V)          \
   if (threads == NT && vpt == V) \
-    return launch_cfg<T, G, NT, V, kTabRows, kTabStages, true>(a, stream, geo);
-  SOL_QK_SPLITS(SOL_CASE)
+    return launch_cfg<T, G, NT, V, kTabRows, kTabStages, true, kTabChunk, true>(a, stream, geo);
+  SOL_QK_TAB_SPLITS(SOL_CASE)
 #undef SOL_CASE
   return cudaErrorInvalidValue;
 }
 
-template <typename T, int G>
-cudaError_t dispatch(const QkArgs &a, int threads, int vpt, cudaStream_t stream, Geometry *geo) {
-  if (a.rope_tab) return dispatch_tab<T, G>(a, threads, vpt, stream, geo);
-#define SOL_CASE(NT, V) \
-  if (threads == NT && vpt == V) return launch<T, G, NT, V>(a, stream, geo);
-  SOL_QK_SPLITS(SOL_CASE)
-#undef SOL_CASE
-  return cudaErrorInvalidValue;
+// Launch for element type T: the table-driven form (TAB, a.rope_tab set) or
+// the on-the-fly one, G = head_dim * esize / 16 lanes per head.
+template <typename T, bool TAB>
+cudaError_t launch_form(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
+  const int G = a.head_dim * static_cast<int>(sizeof(T)) / 16;
+  if (a.npairs > kMaxPairs || TAB != (a.rope_tab != nullptr)) return cudaErrorInvalidValue;
+  int threads = 0, vpt = 0;
+  if (!(TAB ? pick_split_tab : pick_split_otf)(a.nvec_q, &threads, &vpt))
+    return cudaErrorInvalidValue;
+  switch (G) {
+#define SOL_G(g)                                                                  \
+  case g:                                                                         \
+    if constexpr (TAB) return dispatch_tab<T, g>(a, threads, vpt, stream, geo); \
+    else return dispatch<T, g>(a, threads, vpt, stream, geo);
+    SOL_G(2) SOL_G(4) SOL_G(8) SOL_G(16) SOL_G(32)
+#undef SOL_G
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace qk

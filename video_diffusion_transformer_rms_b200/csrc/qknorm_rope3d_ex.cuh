@@ -329,14 +329,13 @@ cudaError_t launch_ex_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
 
 template <int G, int NT, int VPT, bool HALF, bool OUT8>
 cudaError_t launch_ex(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
-  if (a.rope_tab)
-    return launch_ex_cfg<G, NT, VPT, kTabRows, kTabStages, HALF, OUT8, true>(a, stream, geo);
   // One row per ring stage for INT8 and for half-split bf16 (half the ring,
   // more CTAs per SM; INT8 0.90 against 1.04 ms at the 5 s clip), two rows
   // per stage (one barrier per two rows) for interleaved bf16, which measured
-  // as fast or faster for it.
+  // as fast or faster for it.  Rows in round-robin chunks as the default
+  // kernel (kOtfChunk).
   constexpr int R = (OUT8 || HALF) ? 1 : (VPT <= 6 ? 2 : 1);
-  return launch_ex_cfg<G, NT, VPT, R, 2, HALF, OUT8, false>(a, stream, geo);
+  return launch_ex_cfg<G, NT, VPT, R, 2, HALF, OUT8, false, kOtfChunk, false>(a, stream, geo);
 }
 
 template <int G, bool HALF, bool OUT8>
@@ -351,6 +350,54 @@ cudaError_t dispatch_ex(const QkArgs &a, int threads, int vpt, cudaStream_t stre
   }
 #undef SOL_CASE
   return cudaErrorInvalidValue;
+}
+
+// Table-driven variants: the split, ring and row order of the table-driven
+// default kernel (pick_split_tab, kTabRows x kTabStages, chunks of
+// kTabChunk, a barrier per stage).
+template <int G, bool HALF, bool OUT8>
+cudaError_t dispatch_ex_tab(const QkArgs &a, int threads, int vpt, cudaStream_t stream,
+                            Geometry *geo) {
+#define SOL_CASE(NT, V)                                                                   \
+  if (threads == NT && vpt == V)                                                          \
+    return launch_ex_cfg<G, NT, V, kTabRows, kTabStages, HALF, OUT8, true, kTabChunk, true>( \
+        a, stream, geo);
+  SOL_QK_TAB_SPLITS(SOL_CASE)
+#undef SOL_CASE
+  return cudaErrorInvalidValue;
+}
+
+// Launch of one output type (OUT8: int8 codes, else bf16) in one form (TAB:
+// a.rope_tab set), for head_dim 64, 128 or 256 (G = 8, 16, 32 lanes per
+// head) and either rotary pair layout.
+template <bool OUT8, bool TAB>
+cudaError_t launch_ex_form(const QkArgs &a, bool half, cudaStream_t stream, Geometry *geo) {
+  const int G = a.head_dim * 2 / 16;
+  if (a.npairs > kMaxPairs || TAB != (a.rope_tab != nullptr)) return cudaErrorInvalidValue;
+  int threads = 0, vpt = 0;
+  bool split;
+  if constexpr (TAB) {
+    split = pick_split_tab(a.nvec_q, &threads, &vpt);
+  } else {
+    // the split rule of kRowSplit, which dispatch_ex instantiates
+    const bool row = half ? kRowSplit<true, OUT8> : kRowSplit<false, OUT8>;
+    split = row ? pick_split(a.nvec_q, &threads, &vpt) : pick_split_qk(a.nvec_q, &threads, &vpt);
+  }
+  if (!split) return cudaErrorInvalidValue;
+  switch (G) {
+#define SOL_G(g)                                                                     \
+  case g:                                                                            \
+    if constexpr (TAB) {                                                             \
+      return half ? dispatch_ex_tab<g, true, OUT8>(a, threads, vpt, stream, geo)     \
+                  : dispatch_ex_tab<g, false, OUT8>(a, threads, vpt, stream, geo);   \
+    } else {                                                                         \
+      return half ? dispatch_ex<g, true, OUT8>(a, threads, vpt, stream, geo)         \
+                  : dispatch_ex<g, false, OUT8>(a, threads, vpt, stream, geo);       \
+    }
+    SOL_G(8) SOL_G(16) SOL_G(32)
+#undef SOL_G
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace qk

@@ -1,0 +1,12 @@
+// QKNorm + 3D RoPE epilogue variants with bf16 output and (cos, sin) read
+// from a rotary table, for head_dim 64, 128 or 256 and either pair layout.
+#include "qknorm_rope3d_ex.cuh"
+
+namespace sol {
+
+cudaError_t launch_qknorm_rope3d_ex_tab_bf16out(const QkArgs &a, bool half_split,
+                                               cudaStream_t stream, Geometry *geo) {
+  return qk::launch_ex_form<false, true>(a, half_split, stream, geo);
+}
+
+}  // namespace sol

@@ -157,6 +157,44 @@ bool pick_split_qk(int64_t nvec, int *threads, int *vpt) {
   return false;
 }
 
+bool pick_split_otf(int64_t nvec, int *threads, int *vpt) {
+  if (nvec <= 0 || nvec > 256 * kMaxVpt) return false;
+  if (nvec <= 128) {
+    *threads = 32;
+    *vpt = static_cast<int>((nvec + 31) / 32);
+  } else if (nvec <= 1024) {
+    *threads = static_cast<int>(((nvec + 3) / 4 + 31) / 32 * 32);
+    *vpt = 4;
+  } else {
+    *threads = 256;
+    *vpt = static_cast<int>((nvec + 255) / 256);
+  }
+  return true;
+}
+
+bool pick_split_tab(int64_t nvec, int *threads, int *vpt) {
+  static const int sizes[] = {32, 64, 96, 128, 160, 192, 224, 256, 320, 384, 448, 512};
+  if (nvec <= 0 || nvec > 256 * kMaxVpt) return false;
+  if (nvec <= 32) {
+    *threads = 32;
+    *vpt = 1;
+  } else if (nvec <= 1024) {
+    const int64_t half = (nvec + 1) / 2;
+    int t = 512;
+    for (int c : sizes)
+      if (c >= half) {
+        t = c;
+        break;
+      }
+    *threads = t;
+    *vpt = 2;
+  } else {
+    *threads = 256;
+    *vpt = static_cast<int>((nvec + 255) / 256);
+  }
+  return true;
+}
+
 }  // namespace sol
 
 namespace sol {
@@ -425,8 +463,13 @@ sol_status qk_ex(const char *fn, const void *qkv, int64_t ld_qkv, void *q_out, v
   a.per_axis = layout->per_axis_freq;
   a.rope_tab = tab ? tab->data : nullptr;
   const bool half = layout->half_split != 0;
-  cudaError_t e = int8 ? launch_qknorm_rope3d_ex_int8out(a, half, stream, nullptr)
-                       : launch_qknorm_rope3d_ex_bf16out(a, half, stream, nullptr);
+  cudaError_t e;
+  if (tab)
+    e = int8 ? launch_qknorm_rope3d_ex_tab_int8out(a, half, stream, nullptr)
+             : launch_qknorm_rope3d_ex_tab_bf16out(a, half, stream, nullptr);
+  else
+    e = int8 ? launch_qknorm_rope3d_ex_int8out(a, half, stream, nullptr)
+             : launch_qknorm_rope3d_ex_bf16out(a, half, stream, nullptr);
   if (e != cudaSuccess) return cuda_fail(e, fn);
   if (quant_v) {
     QuantArgs v{};
@@ -448,6 +491,7 @@ sol_status qk_ex(const char *fn, const void *qkv, int64_t ld_qkv, void *q_out, v
 }
 
 }  // namespace
+
 }  // namespace sol
 
 using namespace sol;

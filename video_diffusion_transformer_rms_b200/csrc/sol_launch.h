@@ -44,6 +44,23 @@ bool pick_split_qk(int64_t nvec, int *threads, int *vpt);
   X(32, 1) X(32, 2) X(32, 3) X(64, 2) X(64, 3) X(128, 2) X(128, 3) X(256, 2) X(256, 3) \
   X(256, 4) X(256, 5) X(256, 6) X(256, 7) X(256, 8)
 
+// The default (on-the-fly) QKNorm + RoPE kernel: four vectors per thread
+// where the row allows, the CTA being the row's vectors / 4 rounded up to a
+// whole warp (up to 256 threads), then up to 8 vectors at 256 threads.  At
+// D = 5120 that is 160 x 4, which fills every slot.
+bool pick_split_otf(int64_t nvec, int *threads, int *vpt);
+#define SOL_QK_OTF_SPLITS(X)                                                        \
+  X(32, 1) X(32, 2) X(32, 3) X(32, 4) X(64, 4) X(96, 4) X(128, 4) X(160, 4) X(192, 4) \
+  X(224, 4) X(256, 4) X(256, 5) X(256, 6) X(256, 7) X(256, 8)
+
+// Table-driven QKNorm + RoPE kernels: two vectors per thread, the CTA being
+// the row's vectors / 2 rounded up to the next size below (up to 512
+// threads: 320 x 2 at D = 5120), then up to 8 vectors at 256 threads.
+bool pick_split_tab(int64_t nvec, int *threads, int *vpt);
+#define SOL_QK_TAB_SPLITS(X)                                                           \
+  X(32, 1) X(32, 2) X(64, 2) X(96, 2) X(128, 2) X(160, 2) X(192, 2) X(224, 2) X(256, 2) \
+  X(320, 2) X(384, 2) X(448, 2) X(512, 2) X(256, 5) X(256, 6) X(256, 7) X(256, 8)
+
 // Every (threads, vectors per thread) pick_split can return, for the
 // launchers' compile-time dispatch.
 #define SOL_SPLITS(X)                                                              \
@@ -174,15 +191,26 @@ cudaError_t launch_residual_change_noalloc(ChangeArgs a, int dtype, cudaStream_t
                                            Geometry *geo);
 cudaError_t launch_qknorm_rope3d_f32(const QkArgs &a, cudaStream_t stream, Geometry *geo);
 cudaError_t launch_qknorm_rope3d_bf16(const QkArgs &a, cudaStream_t stream, Geometry *geo);
+// the same reading (cos, sin) from the rotary table a.rope_tab
+cudaError_t launch_qknorm_rope3d_tab_f32(const QkArgs &a, cudaStream_t stream, Geometry *geo);
+cudaError_t launch_qknorm_rope3d_tab_bf16(const QkArgs &a, cudaStream_t stream, Geometry *geo);
 cudaError_t launch_qknorm_rope3d_ex_bf16out(const QkArgs &a, bool half_split, cudaStream_t stream,
                                            Geometry *geo);
 cudaError_t launch_qknorm_rope3d_ex_int8out(const QkArgs &a, bool half_split, cudaStream_t stream,
                                            Geometry *geo);
+// the same reading (cos, sin) from the rotary table a.rope_tab
+cudaError_t launch_qknorm_rope3d_ex_tab_bf16out(const QkArgs &a, bool half_split,
+                                               cudaStream_t stream, Geometry *geo);
+cudaError_t launch_qknorm_rope3d_ex_tab_int8out(const QkArgs &a, bool half_split,
+                                               cudaStream_t stream, Geometry *geo);
 // head_dim 64, 128 or 256 (8, 16 or 32 lanes per head).
 cudaError_t launch_quantize_heads_int8(const QuantArgs &a, int head_dim, cudaStream_t stream,
                                        Geometry *geo);
 inline cudaError_t launch_qknorm_rope3d(const QkArgs &a, int dtype, cudaStream_t stream,
                                         Geometry *geo) {
+  if (a.rope_tab)
+    return dtype == 0 ? launch_qknorm_rope3d_tab_f32(a, stream, geo)
+                      : launch_qknorm_rope3d_tab_bf16(a, stream, geo);
   return dtype == 0 ? launch_qknorm_rope3d_f32(a, stream, geo)
                     : launch_qknorm_rope3d_bf16(a, stream, geo);
 }

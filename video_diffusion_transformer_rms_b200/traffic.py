@@ -28,7 +28,7 @@ KERNEL_SOURCES = {
     "rms_adaln": ["rms_adaln.cu"] + _COMMON,
     "gate_residual": ["gate_residual.cu"] + _COMMON,
     "qknorm_rope3d": ["qknorm_rope3d.cuh", "qknorm_rope3d_bf16.cu"] + _COMMON,
-    "qknorm_rope3d_tab": ["qknorm_rope3d.cuh", "qknorm_rope3d_bf16.cu", "rope_table.cu"]
+    "qknorm_rope3d_tab": ["qknorm_rope3d.cuh", "qknorm_rope3d_tab_bf16.cu", "rope_table.cu"]
     + _COMMON,
 }
 
