@@ -79,9 +79,19 @@ def test_traffic_record_from_an_ncu_csv(tmp_path):
     assert len(launches) == 2
     assert launches[0][1:] == pytest.approx((668.10e6, 660.0e6))
     assert launches[1][1:] == pytest.approx((671.9e6, 664.0e6))
-    rec = traffic.make_record(launches, "qknorm_rope3d_tab", "clip5s", 32768, 4 * 32768, "cmd")
+    rec = traffic.make_record([(launches, 32768)], "qknorm_rope3d_tab", "clip5s", 4 * 32768,
+                              "cmd")
     assert rec["traffic_bytes_per_launch"] == pytest.approx(4 * (670.0e6 + 662.0e6))
-    assert rec["launches"] == 2 and rec["captured_rows"] == 32768
+    assert rec["captures"][0]["rows"] == 32768
     assert rec["source_sha256"] == traffic.source_sha("qknorm_rope3d_tab")
+    # two slices: the line through them, so a constant part (writes still in
+    # L2 when the launch ends) is not multiplied by the row ratio
+    small = [("k", 100.0, 80.0)]            # 100 rows: 100 B read, 80 B written
+    large = [("k", 200.0, 180.0)]           # 200 rows: writes = 100 per 100 rows - 20
+    rec2 = traffic.make_record([(small, 100), (large, 200)], "rms_adaln", "clip5s", 1000, "c")
+    assert rec2["read_bytes_per_launch"] == pytest.approx(1000.0)
+    assert rec2["write_bytes_per_launch"] == pytest.approx(980.0)
     with pytest.raises(ValueError):
-        traffic.make_record([], "rms_adaln", "clip5s", 1, 1, "cmd")
+        traffic.make_record([([], 1)], "rms_adaln", "clip5s", 1, "cmd")
+    with pytest.raises(ValueError):
+        traffic.make_record([(small, 100), (large, 100)], "rms_adaln", "clip5s", 1, "cmd")

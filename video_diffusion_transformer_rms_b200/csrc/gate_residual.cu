@@ -105,13 +105,13 @@ __global__ void __launch_bounds__(NT) gate_residual_kernel(const GateArgs a) {
   cp_async_wait<0>();
 }
 
-// Rows in chunks of kChunk dealt round-robin over the CTAs (the grid sweeps
+// Rows in chunks of kGateChunk dealt round-robin over the CTAs (the grid sweeps
 // one contiguous window), with a CTA barrier per iteration although nothing
 // is shared: it keeps the CTA's warps on the same rows.  0.605 against
 // 0.633 ms for a contiguous share per CTA without the barrier (5 s clip).
-constexpr int kChunk = 8;
+constexpr int kGateChunk = 8;
 
-template <typename T, int NT, int VPT, int R = (VPT <= 6 ? 2 : 1), int S = 2, int K = kChunk,
+template <typename T, int NT, int VPT, int R = (VPT <= 6 ? 2 : 1), int S = 2, int K = kGateChunk,
           bool BAR = true>
 cudaError_t launch_t(const GateArgs &a, cudaStream_t stream, Geometry *geo) {
   const void *fn =

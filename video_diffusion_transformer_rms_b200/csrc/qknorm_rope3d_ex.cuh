@@ -22,6 +22,51 @@
 namespace sol {
 namespace qk {
 
+// INT8 codes of one lane's N rotated values u[] of a head whose other values
+// sit in the G - 1 partner lanes of its aligned lane group.  1/rms is one
+// positive factor per head, so it cancels from the codes: code =
+// round(u * 127 / max|u|) on the un-normalised rotation, and only the scale
+// max|u| / rms / 127 needs it.  The sum of squares (ssq: this lane's part)
+// and the max reduce side by side.  Codes are rounded half to even (one FMA
+// with kRoundMagic) and packed four to a word, in element order.
+template <int N, int G>
+__device__ __forceinline__ void int8_codes(float (&u)[N], float ssq, float inv_hd, float eps,
+                                           uint32_t (&words)[N / 4], float &scale) {
+  float m[N / 2];
+#pragma unroll
+  for (int e = 0; e < N / 2; ++e) m[e] = fmaxf(fabsf(u[2 * e]), fabsf(u[2 * e + 1]));
+#pragma unroll
+  for (int w = N / 4; w > 0; w >>= 1)
+#pragma unroll
+    for (int e = 0; e < w; ++e) m[e] = fmaxf(m[e], m[e + w]);
+  float umax = m[0];
+#pragma unroll
+  for (int off = G / 2; off > 0; off >>= 1) {
+    ssq += __shfl_xor_sync(0xffffffffu, ssq, off);
+    umax = fmaxf(umax, __shfl_xor_sync(0xffffffffu, umax, off));
+  }
+  const float inv = rsqrtf(fmaf(ssq, inv_hd, eps));
+  // |u * is| <= 127 up to the fast division's 2 ulp, which the round to
+  // nearest keeps at 127
+  float is = umax > 0.f ? __fdividef(127.f, umax) : 0.f;
+  if (umax > 0.f && umax < 0x1p-96f) {
+    // a head of (near-)denormal inputs: 127 / umax would overflow, so scale
+    // u and umax by 2^64 (exact) first; the codes are unchanged
+#pragma unroll
+    for (int e = 0; e < N; ++e) u[e] *= 0x1p64f;
+    is = __fdividef(127.f, umax * 0x1p64f);
+  }
+  const float2 is2 = splat2(is), magic2 = splat2(kRoundMagic);
+#pragma unroll
+  for (int w = 0; w < N / 4; ++w) {
+    const float2 r0 = fma2(make_float2(u[4 * w], u[4 * w + 1]), is2, magic2);
+    const float2 r1 = fma2(make_float2(u[4 * w + 2], u[4 * w + 3]), is2, magic2);
+    words[w] = pack_low_bytes(__float_as_uint(r0.x), __float_as_uint(r0.y),
+                              __float_as_uint(r1.x), __float_as_uint(r1.y));
+  }
+  scale = umax * inv * (1.f / 127.f);
+}
+
 template <int G, int NT, int VPT, int R, int S, bool HALF, bool OUT8, bool TAB, int K = 0,
           bool BAR = false>
 __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
@@ -238,44 +283,12 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
             const int head = v / G;
             unsigned char *dst = obase + static_cast<int64_t>(head) * a.out_sh + (v % G) * VB;
             if constexpr (OUT8) {
-              // 1/rms is one positive factor per head, so it cancels from the
-              // codes: code = round(u * 127 / max|u|) on the un-normalised
-              // rotation u, and only the scale max|u| / rms / 127 needs it.
-              // The sum of squares and the max then reduce side by side.
-              float ssq = acc.x + acc.y;
-              float m4[E / 2];
-#pragma unroll
-              for (int e = 0; e < E / 2; ++e) m4[e] = fmaxf(fabsf(o[2 * e]), fabsf(o[2 * e + 1]));
-              float umax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-#pragma unroll
-              for (int off = G / 2; off > 0; off >>= 1) {
-                ssq += __shfl_xor_sync(0xffffffffu, ssq, off);
-                umax = fmaxf(umax, __shfl_xor_sync(0xffffffffu, umax, off));
-              }
-              const float inv = rsqrtf(fmaf(ssq, a.inv_hd, a.eps));
-              // |u * is| <= 127 up to the fast division's 2 ulp, which the
-              // round-to-nearest keeps at 127
-              float is = umax > 0.f ? __fdividef(127.f, umax) : 0.f;
-              if (umax > 0.f && umax < 0x1p-96f) {
-                // a head of (near-)denormal inputs: 127 / umax would overflow,
-                // so scale u and umax by 2^64 (exact) first; the codes are
-                // unchanged
-#pragma unroll
-                for (int e = 0; e < E; ++e) o[e] *= 0x1p64f;
-                is = __fdividef(127.f, umax * 0x1p64f);
-              }
-              uint32_t c[E];
-              const float2 is2 = splat2(is), magic2 = splat2(kRoundMagic);
-#pragma unroll
-              for (int m = 0; m < P; ++m) {
-                const float2 r = fma2(make_float2(o[2 * m], o[2 * m + 1]), is2, magic2);
-                c[2 * m] = __float_as_uint(r.x);
-                c[2 * m + 1] = __float_as_uint(r.y);
-              }
+              uint32_t w8[2];
+              float scale;
+              int8_codes<E, G>(o, acc.x + acc.y, a.inv_hd, a.eps, w8, scale);
               if (ok[k]) {
-                st_stream8(dst, pack_low_bytes(c[0], c[1], c[2], c[3]),
-                           pack_low_bytes(c[4], c[5], c[6], c[7]));
-                if (gl == 0) scale_row[head] = umax * inv * (1.f / 127.f);
+                st_stream8(dst, w8[0], w8[1]);
+                if (gl == 0) scale_row[head] = scale;
               }
             } else {
               const float2 inv2 = splat2(rsqrtf(fmaf(group_sum<G>(acc.x + acc.y), a.inv_hd, a.eps)));
@@ -309,6 +322,239 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
 template <bool HALF, bool OUT8>
 constexpr bool kRowSplit = HALF != OUT8;
 
+// INT8 output with interleaved pairs, 16 elements per lane.  The INT8
+// epilogue is bound by instruction issue, not DRAM, and most of its
+// per-element cost is per head and lane: the two-value shuffle reduction,
+// the reciprocals and the scale store.  Here G2 = head_dim / 16 lanes share a
+// head (8 at head_dim 128), and lane g owns the head's 16-byte chunks g and
+// g + G2, i.e. pairs 4g .. 4g+3 and 4(g+G2) .. 4(g+G2)+3.  A warp's copy of
+// the first chunks covers whole 128-byte halves of four heads, so every L2
+// sector it touches is used in full, and the second copy the other halves.
+// The reduction runs over G2 lanes for 16 elements instead of 2 * G2 lanes
+// for 8.  Codes go out as two 8-byte stores per lane.  Same ring, row order
+// and (cos, sin) sources as qknorm_rope3d_ex_kernel.
+template <int G2, int NT, int VPT, int R, int S, bool TAB, int K = 0, bool BAR = false,
+          int MINB = 1>
+__global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkArgs a) {
+  static_assert(K % R == 0, "a ring stage's rows must lie in one chunk");
+  static_assert(NT % G2 == 0 && 32 % G2 == 0, "a head's lanes must share a warp");
+  using IO = Io<__nv_bfloat16>;
+  constexpr int P = 4;  // rotary pairs per 16-byte chunk
+  constexpr int Q = 2;  // float2 lanes of (pair 2m, pair 2m+1) per chunk
+  constexpr int NTAB = 2 * R * kMaxPairs;
+  constexpr size_t HDR = TAB ? 0 : header_bytes<R>();
+  extern __shared__ __align__(16) unsigned char smem[];
+  double *freq = reinterpret_cast<double *>(smem);
+  float *cosb = reinterpret_cast<float *>(smem + kMaxPairs * 8);
+  float *sinb = cosb + NTAB;
+  uint4 *ring = reinterpret_cast<uint4 *>(smem + HDR);  // [S][R][2][VPT][2][NT]
+
+  const int tid = threadIdx.x;
+  const int g = tid % G2;
+  const int nslots = a.nvec_q / 2;  // (head, lane) slots of one part: n_heads * G2
+  const int64_t part_bytes = static_cast<int64_t>(a.nvec_q) * 16;
+  int p0[2];  // first pair of each half
+  p0[0] = P * g;
+  p0[1] = P * (g + G2);
+
+  bool ok[VPT];
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) ok[k] = k * NT + tid < nslots;
+
+  // gamma per part and half in rotary layout, as qknorm_rope3d.cuh
+  float2 gev[2][2][Q], god[2][2][Q];
+#pragma unroll
+  for (int part = 0; part < 2; ++part) {
+    const uint4 *gp = static_cast<const uint4 *>(part == 0 ? a.gamma_q : a.gamma_k);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (gp) {
+        IO::unpack_eo(ld_shared_vec(gp + g + h * G2), gev[part][h], god[part][h]);
+      } else {
+#pragma unroll
+        for (int m = 0; m < Q; ++m) gev[part][h][m] = god[part][h][m] = splat2(1.f);
+      }
+    }
+  }
+  TabPairs<P> tp[2];
+  if constexpr (TAB) {
+    tp[0].init(p0[0], a.sec_t, a.sec_th);
+    tp[1].init(p0[1], a.sec_t, a.sec_th);
+  } else {
+    for (int p = tid; p < a.npairs; p += NT) {
+      double e = -2.0 * p / a.head_dim;
+      if (a.per_axis) {
+        const int start = p < a.sec_t ? 0 : (p < a.sec_th ? a.sec_t : a.sec_th);
+        const int size = p < a.sec_t ? a.sec_t : (p < a.sec_th ? a.sec_th - a.sec_t
+                                                               : a.npairs - a.sec_th);
+        e = -static_cast<double>(p - start) / size;
+      }
+      freq[p] = pow(static_cast<double>(a.theta), e);
+    }
+  }
+
+  RowOrder<K> ro;
+  ro.init(a.rows);
+  const int count = ro.count;
+  const int iters = (count + R - 1) / R;
+  const unsigned char *qkv = static_cast<const unsigned char *>(a.qkv);
+  auto slot = [&](int s, int q, int part, int k, int h) -> uint4 * {
+    return &ring[((((s * R + q) * 2 + part) * VPT + k) * 2 + h) * NT + tid];
+  };
+  // chunk index in a part of the first chunk of slot k: head * 2 * G2 + g
+  auto chunk0 = [&](int k) -> int {
+    const int u = k * NT + tid;
+    return (u / G2) * (2 * G2) + g;
+  };
+  auto issue = [&](int it, int s) {
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      const int j = it * R + q;
+      if (j < count) {
+        const unsigned char *src = qkv + ro.row(j) * a.ld_qkv_bytes;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          const uint4 *ps = reinterpret_cast<const uint4 *>(src + part * part_bytes);
+#pragma unroll
+          for (int k = 0; k < VPT; ++k) {
+            if (ok[k]) {
+              const int c = chunk0(k);
+              cp_async16(slot(s, q, part, k, 0), ps + c);
+              cp_async16(slot(s, q, part, k, 1), ps + c + G2);
+            }
+          }
+        }
+      }
+    }
+    cp_async_commit();
+  };
+
+#pragma unroll
+  for (int s = 0; s < S - 1; ++s) issue(s, s);
+  if constexpr (!TAB) __syncthreads();
+
+  TokenCursor tok;
+  GridCursor pos;
+  int cons = 0;
+  int buf = 0;
+  for (int it = 0; it < iters; ++it) {
+    issue(it + S - 1, cons == 0 ? S - 1 : cons - 1);
+    if (ro.run_start(it * R)) {
+      tok.init(ro.row(it * R), a.L);
+      pos.init(tok.r, a.n_video, a.HW, a.W);
+    }
+    if constexpr (!TAB)
+      angle_tables<R, NT>(a, freq, tok, pos, cosb + buf * R * kMaxPairs,
+                          sinb + buf * R * kMaxPairs);
+    cp_async_wait<S - 1>();
+    if constexpr (!TAB || BAR) __syncthreads();
+
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      const int j = it * R + q;
+      if (j < count) {
+        // cos and sin of the lane's pairs, per half
+        float ct[2][P], st[2][P];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if constexpr (TAB) {
+            tp[h].read(a.rope_tab, a.npairs, p0[h], pos.t, pos.h, pos.w, ct[h], st[h]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < P; ++i) {
+              ct[h][i] = cosb[(buf * R + q) * kMaxPairs + p0[h] + i];
+              st[h][i] = sinb[(buf * R + q) * kMaxPairs + p0[h] + i];
+            }
+          }
+        }
+        const int64_t grow = ro.row(j);
+        const int64_t row_off = static_cast<int64_t>(tok.b) * a.out_sb +
+                                static_cast<int64_t>(tok.r) * a.out_sr;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          // rotation coefficients of this lane's pairs, gamma folded in
+          float2 c0[2][Q], ns1[2][Q], s0[2][Q], c1[2][Q];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int m = 0; m < Q; ++m) {
+              const float2 cs = make_float2(ct[h][2 * m], ct[h][2 * m + 1]);
+              const float2 sn = make_float2(st[h][2 * m], st[h][2 * m + 1]);
+              c0[h][m] = mul2(gev[part][h][m], cs);
+              s0[h][m] = mul2(gev[part][h][m], sn);
+              ns1[h][m] = mul2(god[part][h][m], make_float2(-sn.x, -sn.y));
+              c1[h][m] = mul2(god[part][h][m], cs);
+            }
+          }
+          unsigned char *obase = static_cast<unsigned char *>(part == 0 ? a.q_out : a.k_out) +
+                                 row_off;
+          float *scale_row = (part == 0 ? a.q_scale : a.k_scale) +
+                             grow * static_cast<int64_t>(a.n_heads);
+#pragma unroll
+          for (int k = 0; k < VPT; ++k) {
+            // every lane joins the shuffles; ok[] only guards memory accesses
+            float o[16];
+            float2 acc = splat2(0.f);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+              if (ok[k]) xv = *slot(cons, q, part, k, h);
+              float2 ev[Q], od[Q];
+              IO::unpack_eo(xv, ev, od);
+#pragma unroll
+              for (int m = 0; m < Q; ++m) {
+                acc = fma2(ev[m], ev[m], acc);
+                acc = fma2(od[m], od[m], acc);
+              }
+#pragma unroll
+              for (int m = 0; m < Q; ++m) {
+                const float2 u0 = fma2(od[m], ns1[h][m], mul2(ev[m], c0[h][m]));
+                const float2 u1 = fma2(od[m], c1[h][m], mul2(ev[m], s0[h][m]));
+                o[8 * h + 4 * m + 0] = u0.x;
+                o[8 * h + 4 * m + 1] = u1.x;
+                o[8 * h + 4 * m + 2] = u0.y;
+                o[8 * h + 4 * m + 3] = u1.y;
+              }
+            }
+            uint32_t w8[4];
+            float scale;
+            int8_codes<16, G2>(o, acc.x + acc.y, a.inv_hd, a.eps, w8, scale);
+            if (ok[k]) {
+              const int head = (k * NT + tid) / G2;
+              unsigned char *dst = obase + static_cast<int64_t>(head) * a.out_sh;
+              st_stream8(dst + g * 8, w8[0], w8[1]);
+              st_stream8(dst + (g + G2) * 8, w8[2], w8[3]);
+              if (g == 0) scale_row[head] = scale;
+            }
+          }
+        }
+        tok.next(a.L);
+        pos.next(tok.r, a.n_video, a.H, a.W);
+      }
+    }
+    buf ^= 1;
+    cons = (cons + 1 == S) ? 0 : cons + 1;
+  }
+  cp_async_wait<0>();
+}
+
+template <int G2, int NT, int VPT, int R, int S, bool TAB, int K = 0, bool BAR = false,
+          int MINB = 1>
+cudaError_t launch_int8w_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
+  const void *fn = reinterpret_cast<const void *>(
+      &qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, BAR, MINB>);
+  const size_t smem =
+      (TAB ? 0 : header_bytes<R>()) + static_cast<size_t>(S) * R * 2 * VPT * 2 * NT * 16;
+  const int per_sm = resident_blocks(fn, NT, smem);
+  if (per_sm <= 0) return cudaErrorInvalidConfiguration;
+  int64_t grid = static_cast<int64_t>(per_sm) * device_sms();
+  if (grid > a.rows) grid = a.rows;
+  if (geo) *geo = Geometry{NT, VPT, S, smem, static_cast<int>(grid)};
+  qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, BAR, MINB>
+      <<<static_cast<unsigned>(grid), NT, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
 // One launch of a fixed configuration: a wave of as many CTAs as fit.
 template <int G, int NT, int VPT, int R, int S, bool HALF, bool OUT8, bool TAB, int K = 0,
           bool BAR = false>
@@ -327,42 +573,39 @@ cudaError_t launch_ex_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
   return cudaGetLastError();
 }
 
-template <int G, int NT, int VPT, bool HALF, bool OUT8>
+// Ring and row order of the variants (standalone loops at the 5 s clip on a
+// B200; the split is kRowSplit's for both forms):
+//  - on the fly: one row per ring stage for INT8 and half-split bf16 (half
+//    the ring, more CTAs per SM; INT8 0.90 against 1.04 ms), two for
+//    interleaved bf16; rows in round-robin chunks of kOtfChunk for bf16
+//    output (0.916 against 0.925 ms in [B, H, L, hd], 0.909 against 0.929
+//    half-split), a contiguous share per CTA for INT8, which is bound by
+//    instruction issue rather than DRAM and gained nothing from chunks
+//    (0.84 against 0.80 ms);
+//  - table-driven: one row per stage, two stages, chunks of kTabChunk and
+//    a barrier per stage: 0.857 ms in [B, H, L, hd], 0.809 ms half-split
+//    (6.4 TB/s), 0.854 ms INT8.
+template <int G, int NT, int VPT, bool HALF, bool OUT8, bool TAB>
 cudaError_t launch_ex(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
-  // One row per ring stage for INT8 and for half-split bf16 (half the ring,
-  // more CTAs per SM; INT8 0.90 against 1.04 ms at the 5 s clip), two rows
-  // per stage (one barrier per two rows) for interleaved bf16, which measured
-  // as fast or faster for it.  Rows in round-robin chunks as the default
-  // kernel (kOtfChunk).
-  constexpr int R = (OUT8 || HALF) ? 1 : (VPT <= 6 ? 2 : 1);
-  return launch_ex_cfg<G, NT, VPT, R, 2, HALF, OUT8, false, kOtfChunk, false>(a, stream, geo);
+  if constexpr (TAB) {
+    return launch_ex_cfg<G, NT, VPT, 1, 2, HALF, OUT8, true, kTabChunk, true>(a, stream, geo);
+  } else {
+    constexpr int R = (OUT8 || HALF) ? 1 : (VPT <= 6 ? 2 : 1);
+    constexpr int K = OUT8 ? 0 : kOtfChunk;
+    return launch_ex_cfg<G, NT, VPT, R, 2, HALF, OUT8, false, K, false>(a, stream, geo);
+  }
 }
 
-template <int G, bool HALF, bool OUT8>
+template <int G, bool HALF, bool OUT8, bool TAB>
 cudaError_t dispatch_ex(const QkArgs &a, int threads, int vpt, cudaStream_t stream,
                         Geometry *geo) {
 #define SOL_CASE(NT, V) \
-  if (threads == NT && vpt == V) return launch_ex<G, NT, V, HALF, OUT8>(a, stream, geo);
+  if (threads == NT && vpt == V) return launch_ex<G, NT, V, HALF, OUT8, TAB>(a, stream, geo);
   if constexpr (kRowSplit<HALF, OUT8>) {
     SOL_SPLITS(SOL_CASE)
   } else {
     SOL_QK_SPLITS(SOL_CASE)
   }
-#undef SOL_CASE
-  return cudaErrorInvalidValue;
-}
-
-// Table-driven variants: the split, ring and row order of the table-driven
-// default kernel (pick_split_tab, kTabRows x kTabStages, chunks of
-// kTabChunk, a barrier per stage).
-template <int G, bool HALF, bool OUT8>
-cudaError_t dispatch_ex_tab(const QkArgs &a, int threads, int vpt, cudaStream_t stream,
-                            Geometry *geo) {
-#define SOL_CASE(NT, V)                                                                   \
-  if (threads == NT && vpt == V)                                                          \
-    return launch_ex_cfg<G, NT, V, kTabRows, kTabStages, HALF, OUT8, true, kTabChunk, true>( \
-        a, stream, geo);
-  SOL_QK_TAB_SPLITS(SOL_CASE)
 #undef SOL_CASE
   return cudaErrorInvalidValue;
 }
@@ -375,25 +618,16 @@ cudaError_t launch_ex_form(const QkArgs &a, bool half, cudaStream_t stream, Geom
   const int G = a.head_dim * 2 / 16;
   if (a.npairs > kMaxPairs || TAB != (a.rope_tab != nullptr)) return cudaErrorInvalidValue;
   int threads = 0, vpt = 0;
-  bool split;
-  if constexpr (TAB) {
-    split = pick_split_tab(a.nvec_q, &threads, &vpt);
-  } else {
-    // the split rule of kRowSplit, which dispatch_ex instantiates
-    const bool row = half ? kRowSplit<true, OUT8> : kRowSplit<false, OUT8>;
-    split = row ? pick_split(a.nvec_q, &threads, &vpt) : pick_split_qk(a.nvec_q, &threads, &vpt);
-  }
+  // the split rule of kRowSplit, which dispatch_ex instantiates
+  const bool row = half ? kRowSplit<true, OUT8> : kRowSplit<false, OUT8>;
+  const bool split =
+      row ? pick_split(a.nvec_q, &threads, &vpt) : pick_split_qk(a.nvec_q, &threads, &vpt);
   if (!split) return cudaErrorInvalidValue;
   switch (G) {
-#define SOL_G(g)                                                                     \
-  case g:                                                                            \
-    if constexpr (TAB) {                                                             \
-      return half ? dispatch_ex_tab<g, true, OUT8>(a, threads, vpt, stream, geo)     \
-                  : dispatch_ex_tab<g, false, OUT8>(a, threads, vpt, stream, geo);   \
-    } else {                                                                         \
-      return half ? dispatch_ex<g, true, OUT8>(a, threads, vpt, stream, geo)         \
-                  : dispatch_ex<g, false, OUT8>(a, threads, vpt, stream, geo);       \
-    }
+#define SOL_G(g)                                                                   \
+  case g:                                                                          \
+    return half ? dispatch_ex<g, true, OUT8, TAB>(a, threads, vpt, stream, geo)    \
+                : dispatch_ex<g, false, OUT8, TAB>(a, threads, vpt, stream, geo);
     SOL_G(8) SOL_G(16) SOL_G(32)
 #undef SOL_G
     default: return cudaErrorInvalidValue;

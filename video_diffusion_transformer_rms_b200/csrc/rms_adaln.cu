@@ -7,7 +7,7 @@
 // registers, written once as h_out and normalised without a round trip
 // through HBM.
 //
-// One persistent CTA per resident slot walks its rows (chunks of kChunk
+// One persistent CTA per resident slot walks its rows (chunks of kRmsChunk
 // consecutive rows dealt round-robin over the CTAs), R rows per iteration,
 // so the (sample, modality) of each row follows from the previous one
 // without a division inside a chunk.  Thread t owns the 16-byte
@@ -245,14 +245,14 @@ __global__ void __launch_bounds__(NT) rms_adaln_kernel(const RmsArgs a) {
 template <int VPT, bool RESID>
 constexpr int kRows = VPT <= (RESID ? 3 : 5) ? 2 : 1;
 
-// Rows go to the CTAs in chunks of kChunk dealt round-robin, so the grid
+// Rows go to the CTAs in chunks of kRmsChunk dealt round-robin, so the grid
 // works through one contiguous window of the tensors: 0.398 against
 // 0.416 ms for a contiguous share per CTA (RMS-AdaLN at the 5 s clip, output
 // bit-identical), 0.820 against 0.839 ms with the residual.
-constexpr int kChunk = 8;
+constexpr int kRmsChunk = 8;
 
 template <typename T, int NT, int VPT, bool RESID, int R = kRows<VPT, RESID>, int S = 2,
-          int K = kChunk>
+          int K = kRmsChunk>
 cudaError_t launch_t(const RmsArgs &a, cudaStream_t stream, Geometry *geo) {
   constexpr int NIN = RESID ? 2 : 1;
   const void *fn =

@@ -1,16 +1,19 @@
 """DRAM traffic records of the hot-path kernels, kept in profiles/traffic.json.
 
     python -m video_diffusion_transformer_rms_b200.traffic \
-        --csv dram.csv --kernel qknorm_rope3d_tab --workload clip5s \
-        --captured-rows 32768 --command "<the ncu command that wrote dram.csv>"
+        --csv dram8.csv --captured-rows 32658 [--csv dram16.csv --captured-rows 65316] \
+        --kernel qknorm_rope3d_tab --workload clip5s --command "<the commands>"
 
-reads an ncu CSV export (`ncu --csv --log-file ...`) of dram__bytes_read.sum
-and dram__bytes_write.sum for one kernel captured on a slice of a workload,
-averages them per launch, scales them to the workload's full row count (each
-kernel streams its rows once, so its traffic grows in proportion to the rows)
-and stores the record together with the sha256 of the sources the kernel is
-built from.  `lookup` (bench.py's `roofline.traffic`) returns the record only
-while those sources are unchanged.
+reads ncu CSV exports (`ncu --csv --log-file ...`) of dram__bytes_read.sum
+and dram__bytes_write.sum for one kernel captured on slices of a workload,
+averages them per launch and carries them to the workload's full row count.
+Each kernel streams its rows once, so its traffic is a + b * rows: with two
+slices of different sizes the line through them is evaluated at the full
+size (the constant a holds the writes still in L2 when a launch ends, which
+do not grow with the rows); with one slice the bytes are scaled by the rows.
+The record keeps the sha256 of the sources the kernel is built from, and
+`lookup` (bench.py's `roofline.traffic`) returns it only while those sources
+are unchanged.
 """
 import argparse
 import csv
@@ -64,17 +67,31 @@ def parse_ncu_csv(path):
     return [tuple(v) for _, v in sorted(launches.items(), key=lambda kv: int(kv[0]))]
 
 
-def make_record(launches, kernel, workload, captured_rows, full_rows, command, root=None):
-    if not launches:
+def make_record(captures, kernel, workload, full_rows, command, root=None):
+    """captures: [(launches from parse_ncu_csv, captured rows)], one or two."""
+    if not captures or any(not c[0] for c in captures):
         raise ValueError("the CSV holds no dram__bytes_read/write.sum rows")
-    rd = sum(x[1] for x in launches) / len(launches)
-    wr = sum(x[2] for x in launches) / len(launches)
-    scale = full_rows / captured_rows
-    return {"workload": workload, "kernel_name": launches[0][0], "launches": len(launches),
-            "captured_rows": captured_rows, "full_rows": full_rows,
-            "captured_read_bytes": rd, "captured_write_bytes": wr,
-            "traffic_bytes_per_launch": (rd + wr) * scale,
-            "scaling": f"x {scale:.4f} = full rows / captured rows (traffic grows with rows)",
+    pts = []
+    for launches, rows in captures:
+        rd = sum(x[1] for x in launches) / len(launches)
+        wr = sum(x[2] for x in launches) / len(launches)
+        pts.append((rows, rd, wr))
+    if len(pts) == 1:
+        rows, rd, wr = pts[0]
+        full_rd, full_wr = rd * full_rows / rows, wr * full_rows / rows
+        how = f"x {full_rows / rows:.4f} = full rows / captured rows"
+    else:
+        (r0, rd0, wr0), (r1, rd1, wr1) = pts[:2]
+        if r0 == r1:
+            raise ValueError("two captures need different row counts")
+        full_rd = rd0 + (rd1 - rd0) * (full_rows - r0) / (r1 - r0)
+        full_wr = wr0 + (wr1 - wr0) * (full_rows - r0) / (r1 - r0)
+        how = f"line through the {r0}- and {r1}-row captures, at {full_rows} rows"
+    return {"workload": workload, "kernel_name": captures[0][0][0][0],
+            "captures": [{"rows": r, "read_bytes": rd, "write_bytes": wr} for r, rd, wr in pts],
+            "full_rows": full_rows, "read_bytes_per_launch": full_rd,
+            "write_bytes_per_launch": full_wr,
+            "traffic_bytes_per_launch": full_rd + full_wr, "scaling": how,
             "source_sha256": source_sha(kernel, root), "command": command}
 
 
@@ -101,14 +118,17 @@ def lookup(kernel, workload, root=None):
 def main():
     from .workloads import WORKLOADS
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("--csv", required=True)
+    ap.add_argument("--csv", action="append", required=True)
+    ap.add_argument("--captured-rows", type=int, action="append", required=True)
     ap.add_argument("--kernel", required=True, choices=sorted(KERNEL_SOURCES))
     ap.add_argument("--workload", default="clip5s", choices=sorted(WORKLOADS))
-    ap.add_argument("--captured-rows", type=int, required=True)
     ap.add_argument("--command", required=True)
     args = ap.parse_args()
-    rec = make_record(parse_ncu_csv(args.csv), args.kernel, args.workload, args.captured_rows,
-                      WORKLOADS[args.workload].rows, args.command)
+    if len(args.csv) != len(args.captured_rows) or len(args.csv) > 2:
+        raise SystemExit("give one or two --csv, each with its --captured-rows")
+    caps = [(parse_ncu_csv(c), r) for c, r in zip(args.csv, args.captured_rows)]
+    rec = make_record(caps, args.kernel, args.workload, WORKLOADS[args.workload].rows,
+                      args.command)
     records = load()
     records[args.kernel] = rec
     os.makedirs(os.path.dirname(RECORDS), exist_ok=True)
