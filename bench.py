@@ -395,8 +395,8 @@ def run_ours(args):
                                s8.data_ptr() + w.rows * w.n_heads * 4, 0, 0, v8.data_ptr(),
                                vs8.data_ptr())
 
-    def k_qk_ex(lay, q_ptr, k_ptr):
-        if QK_TABLE:
+    def k_qk_ex(lay, q_ptr, k_ptr, use_table=QK_TABLE):
+        if use_table:
             return lambda: _abi.sol_qknorm_rope3d_ex_tab(
                 p["qkv"], 3 * D, q_ptr, k_ptr, lay, p["gamma_q"], p["gamma_k"], table.desc, w.B,
                 w.T, w.H, w.W, w.n_audio, w.n_heads, w.eps, dt, s)
@@ -437,6 +437,16 @@ def run_ours(args):
                                       k_qk_ex(lay_int8_v, q8.data_ptr(),
                                               q8.data_ptr() + w.rows * D)),
     }
+    # the epilogue variants with the other (cos, sin) source too
+    other = "_otf" if QK_TABLE else "_table"
+    for name, lay, qp, kp, bpr_ in (
+            ("qknorm_rope3d_ex_bhsd", lay_bhsd, qk.data_ptr(), qk.data_ptr() + half_bytes,
+             4 * row),
+            ("qknorm_rope3d_ex_half", lay_half, qk.data_ptr(), qk.data_ptr() + half_bytes,
+             4 * row),
+            ("qknorm_rope3d_ex_int8", lay_int8, q8.data_ptr(), q8.data_ptr() + w.rows * D,
+             2 * row + 2 * D + 2 * w.n_heads * 4)):
+        extra[name + other] = (bpr_, k_qk_ex(lay, qp, kp, not QK_TABLE))
     next_rows = {}
     for name, (bytes_per_row, fn) in extra.items():
         ms = dist.max_over_ranks(time_launches(fn, stream, 200))

@@ -313,12 +313,13 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
   cp_async_wait<0>();
 }
 
-// The CTA split each variant takes, measured inside a step at the 5 s clip:
-// the row-reduction rule (pick_split, <= 6 vectors per thread: 128 x 5 at
-// D = 5120, which divides the row exactly) for interleaved INT8 (0.86 against
-// 0.97 ms) and half-split bf16 (0.92 against 0.97 ms); the QK rule
-// (pick_split_qk: 256 x 3, more warps, a sixth of the vector slots empty)
-// for interleaved bf16 and half-split INT8.
+// The CTA split each variant of qknorm_rope3d_ex_kernel takes, measured
+// inside a step at the 5 s clip: the row-reduction rule (pick_split, <= 6
+// vectors per thread: 128 x 5 at D = 5120, which divides the row exactly)
+// for half-split bf16 (0.92 against 0.97 ms); the QK rule (pick_split_qk:
+// 256 x 3, more warps, a sixth of the vector slots empty) for interleaved
+// bf16 and half-split INT8.  (Interleaved INT8 runs in
+// qknorm_rope3d_int8w_kernel, split by pick_split_i8w.)
 template <bool HALF, bool OUT8>
 constexpr bool kRowSplit = HALF != OUT8;
 
@@ -610,6 +611,20 @@ cudaError_t dispatch_ex(const QkArgs &a, int threads, int vpt, cudaStream_t stre
   return cudaErrorInvalidValue;
 }
 
+// Interleaved INT8 with 16 elements per lane (qknorm_rope3d_int8w_kernel),
+// G2 = head_dim / 16 lanes per head: one row per stage, two stages and a
+// contiguous share of rows per CTA in both forms (the kernel is issue-bound;
+// chunks and barriers measured no gain), split by pick_split_i8w.
+template <int G2, bool TAB>
+cudaError_t dispatch_i8w(const QkArgs &a, int threads, int vpt, cudaStream_t stream,
+                         Geometry *geo) {
+#define SOL_CASE(NT, V) \
+  if (threads == NT && vpt == V) return launch_int8w_cfg<G2, NT, V, 1, 2, TAB>(a, stream, geo);
+  SOL_I8W_SPLITS(SOL_CASE)
+#undef SOL_CASE
+  return cudaErrorInvalidValue;
+}
+
 // Launch of one output type (OUT8: int8 codes, else bf16) in one form (TAB:
 // a.rope_tab set), for head_dim 64, 128 or 256 (G = 8, 16, 32 lanes per
 // head) and either rotary pair layout.
@@ -618,16 +633,31 @@ cudaError_t launch_ex_form(const QkArgs &a, bool half, cudaStream_t stream, Geom
   const int G = a.head_dim * 2 / 16;
   if (a.npairs > kMaxPairs || TAB != (a.rope_tab != nullptr)) return cudaErrorInvalidValue;
   int threads = 0, vpt = 0;
+  if constexpr (OUT8) {
+    if (!half) {  // interleaved INT8: 16 elements per lane, G / 2 lanes per head
+      if (!pick_split_i8w(a.nvec_q / 2, &threads, &vpt)) return cudaErrorInvalidValue;
+      switch (G) {
+        case 8: return dispatch_i8w<4, TAB>(a, threads, vpt, stream, geo);
+        case 16: return dispatch_i8w<8, TAB>(a, threads, vpt, stream, geo);
+        case 32: return dispatch_i8w<16, TAB>(a, threads, vpt, stream, geo);
+        default: return cudaErrorInvalidValue;
+      }
+    }
+  }
   // the split rule of kRowSplit, which dispatch_ex instantiates
   const bool row = half ? kRowSplit<true, OUT8> : kRowSplit<false, OUT8>;
   const bool split =
       row ? pick_split(a.nvec_q, &threads, &vpt) : pick_split_qk(a.nvec_q, &threads, &vpt);
   if (!split) return cudaErrorInvalidValue;
   switch (G) {
-#define SOL_G(g)                                                                   \
-  case g:                                                                          \
-    return half ? dispatch_ex<g, true, OUT8, TAB>(a, threads, vpt, stream, geo)    \
-                : dispatch_ex<g, false, OUT8, TAB>(a, threads, vpt, stream, geo);
+#define SOL_G(g)                                                                     \
+  case g:                                                                            \
+    if constexpr (OUT8) { /* half-split: interleaved INT8 returned above */           \
+      return dispatch_ex<g, true, OUT8, TAB>(a, threads, vpt, stream, geo);          \
+    } else {                                                                         \
+      return half ? dispatch_ex<g, true, OUT8, TAB>(a, threads, vpt, stream, geo)    \
+                  : dispatch_ex<g, false, OUT8, TAB>(a, threads, vpt, stream, geo);  \
+    }
     SOL_G(8) SOL_G(16) SOL_G(32)
 #undef SOL_G
     default: return cudaErrorInvalidValue;

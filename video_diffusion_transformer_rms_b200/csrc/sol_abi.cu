@@ -195,6 +195,18 @@ bool pick_split_tab(int64_t nvec, int *threads, int *vpt) {
   return true;
 }
 
+bool pick_split_i8w(int64_t slots, int *threads, int *vpt) {
+  for (int t = 32; t <= 256; t *= 2) {
+    const int64_t v = (slots + t - 1) / t;
+    if (slots > 0 && v <= 5) {
+      *threads = t;
+      *vpt = static_cast<int>(v);
+      return true;
+    }
+  }
+  return false;
+}
+
 }  // namespace sol
 
 namespace sol {

@@ -61,6 +61,16 @@ bool pick_split_tab(int64_t nvec, int *threads, int *vpt);
   X(32, 1) X(32, 2) X(64, 2) X(96, 2) X(128, 2) X(160, 2) X(192, 2) X(224, 2) X(256, 2) \
   X(320, 2) X(384, 2) X(448, 2) X(512, 2) X(256, 5) X(256, 6) X(256, 7) X(256, 8)
 
+// Interleaved INT8 QKNorm + RoPE (16 elements per lane): `slots` = the
+// (head, lane) pairs of one part, n_heads * head_dim / 16.  The smallest CTA
+// of {32, 64, 128, 256} threads with at most 5 slots per thread (64 x 5 at
+// D = 5120, which measured best: 0.705 ms against 0.77-0.86 ms for 128 x 3,
+// 160 x 2 and 320 x 1).
+bool pick_split_i8w(int64_t slots, int *threads, int *vpt);
+#define SOL_I8W_SPLITS(X)                                                              \
+  X(32, 1) X(32, 2) X(32, 3) X(32, 4) X(32, 5) X(64, 3) X(64, 4) X(64, 5) X(128, 3) X(128, 4) \
+  X(128, 5) X(256, 3) X(256, 4) X(256, 5)
+
 // Every (threads, vectors per thread) pick_split can return, for the
 // launchers' compile-time dispatch.
 #define SOL_SPLITS(X)                                                              \

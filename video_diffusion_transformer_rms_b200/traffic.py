@@ -33,6 +33,15 @@ KERNEL_SOURCES = {
     "qknorm_rope3d": ["qknorm_rope3d.cuh", "qknorm_rope3d_bf16.cu"] + _COMMON,
     "qknorm_rope3d_tab": ["qknorm_rope3d.cuh", "qknorm_rope3d_tab_bf16.cu", "rope_table.cu"]
     + _COMMON,
+    "gate_residual_rms_adaln": ["rms_adaln.cu"] + _COMMON,
+    "residual_change": ["residual_change.cu"] + _COMMON,
+    "qknorm_rope3d_ex_bhsd_tab": ["qknorm_rope3d.cuh", "qknorm_rope3d_ex.cuh",
+                                  "qknorm_rope3d_ex_tab_bf16.cu", "rope_table.cu"] + _COMMON,
+    "qknorm_rope3d_ex_half_tab": ["qknorm_rope3d.cuh", "qknorm_rope3d_ex.cuh",
+                                  "qknorm_rope3d_ex_tab_bf16.cu", "rope_table.cu"] + _COMMON,
+    "qknorm_rope3d_ex_int8_tab": ["qknorm_rope3d.cuh", "qknorm_rope3d_ex.cuh",
+                                  "qknorm_rope3d_ex_tab_int8.cu", "rope_table.cu"] + _COMMON,
+    "gemm_gelu": ["gemm_gelu.cu"] + _COMMON,
 }
 
 _UNITS = {"byte": 1.0, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "tbyte": 1e12}
