@@ -149,17 +149,76 @@ __device__ __forceinline__ void angle_tables(const QkArgs &a, const double *freq
   }
 }
 
-template <typename T, int G, int NT, int VPT, int R, int S, bool TAB, int K = 0, bool BAR = false>
+// Table form staged through shared memory (STAGE): the (cos, sin) of one
+// row, copied from the rotary table into dst[2][kMaxPairs] with cp.async in
+// the same group as the row's q and k, so their latency hides behind the
+// ring's prefetch like the data's.  Threads c < npairs/4 copy the cos of
+// pairs 4c .. 4c+3 (16 bytes when the four share an axis, else four 4-byte
+// copies), threads npairs/4 + c their sin.  The row's position comes from
+// its global index by division: the issuing threads run ahead of the
+// consumer's row cursor.  Readers need a CTA barrier after the wait.
+__device__ __forceinline__ void stage_table_row(const QkArgs &a, int64_t row, float *dst) {
+  const int nq = a.npairs >> 2;
+  if (static_cast<int>(threadIdx.x) >= 2 * nq) return;
+  const int b = static_cast<int>(row / a.L);
+  const int r = static_cast<int>(row - static_cast<int64_t>(b) * a.L);
+  int t, h = 0, w = 0;
+  if (r < a.n_video) {
+    t = r / a.HW;
+    const int rem = r - t * a.HW;
+    h = rem / a.W;
+    w = rem - h * a.W;
+  } else {
+    t = r - a.n_video;
+  }
+  const int64_t ld = 2 * static_cast<int64_t>(a.npairs);
+  for (int idx = threadIdx.x; idx < 2 * nq; idx += blockDim.x) {
+    const int which = idx >= nq ? 1 : 0;  // 0: cos, 1: sin
+    const int p = 4 * (idx - which * nq);
+    const float *src = a.rope_tab + which * a.npairs + p;
+    float *d = dst + which * kMaxPairs + p;
+    const int ax0 = pair_axis(p, a.sec_t, a.sec_th);
+    if (ax0 == pair_axis(p + 3, a.sec_t, a.sec_th)) {
+      const int at = ax0 == 0 ? t : (ax0 == 1 ? h : w);
+      cp_async16_ca(d, src + at * ld);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int ax = pair_axis(p + i, a.sec_t, a.sec_th);
+        const int at = ax == 0 ? t : (ax == 1 ? h : w);
+        cp_async4(d + i, src + at * ld + i);
+      }
+    }
+  }
+}
+
+// Bytes of shared memory before the ring: the fp64 frequency table and the
+// per-row angle tables of the on-the-fly form, or STAGE's table ring of
+// (S + 1) stages (one deeper than the data ring, so that a stage is only
+// overwritten once every thread has passed the barrier after its last use).
+template <int R, int S, bool TAB, bool STAGE>
+__host__ __device__ constexpr size_t head_bytes() {
+  return !TAB ? header_bytes<R>()
+              : (STAGE ? static_cast<size_t>(S + 1) * R * 2 * kMaxPairs * 4 : 0);
+}
+
+template <typename T, int G, int NT, int VPT, int R, int S, bool TAB, int K = 0, bool BAR = false,
+          bool STAGE = false>
 __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
   static_assert(K % R == 0, "a ring stage's rows must lie in one chunk");
   using IO = Io<T>;
   constexpr int E = IO::E;
   constexpr int PPV = E / 2;  // rotary pairs per 16-byte vector
   constexpr int Q = PPV / 2;  // float2 lanes of (pair 2m, pair 2m+1) per vector
+  // STAGE (table form only): each row's table entries ride in the ring
+  // (stage_table_row) instead of each thread loading its own pairs per row
+  constexpr bool DIRECT = TAB && !STAGE;
+  constexpr int TS = S + 1;  // STAGE's table ring
   constexpr int NTAB = 2 * R * kMaxPairs;
-  constexpr size_t HDR = TAB ? 0 : header_bytes<R>();
+  constexpr size_t HDR = head_bytes<R, S, TAB, STAGE>();
   extern __shared__ __align__(16) unsigned char smem[];
   double *freq = reinterpret_cast<double *>(smem);
+  float *tabr = reinterpret_cast<float *>(smem);                  // STAGE: [TS][R][2][kMaxPairs]
   float *cosb = reinterpret_cast<float *>(smem + kMaxPairs * 8);  // [2][R][kMaxPairs]
   float *sinb = cosb + NTAB;                                      // [2][R][kMaxPairs]
   uint4 *ring = reinterpret_cast<uint4 *>(smem + HDR);            // [S][R][2][VPT][NT]
@@ -190,9 +249,9 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
     }
   }
   TabPairs<PPV> tp;
-  if constexpr (TAB) {
+  if constexpr (DIRECT) {
     tp.init(p0, a.sec_t, a.sec_th);
-  } else {
+  } else if constexpr (!TAB) {
     for (int p = tid; p < a.npairs; p += NT)
       freq[p] = pow(static_cast<double>(a.theta), -2.0 * p / a.head_dim);
   }
@@ -217,6 +276,8 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
           for (int k = 0; k < VPT; ++k)
             if (ok[k]) cp_async16(slot(s, q, part, k), ps + k * NT);
         }
+        if constexpr (STAGE)
+          stage_table_row(a, ro.row(j), tabr + ((it % TS) * R + q) * 2 * kMaxPairs);
       }
     }
     cp_async_commit();
@@ -242,7 +303,7 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
                           sinb + buf * R * kMaxPairs);
 
     cp_async_wait<S - 1>();
-    if constexpr (!TAB || BAR) __syncthreads();  // angle tables of these rows visible
+    if constexpr (!DIRECT || BAR) __syncthreads();  // angle tables of these rows visible
 
 #pragma unroll
     for (int q = 0; q < R; ++q) {
@@ -250,13 +311,20 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
       if (j < count) {
         // cs[m] = (cos of pair p0+2m, cos of pair p0+2m+1); likewise sn
         float2 cs[Q], sn[Q];
-        if constexpr (TAB) {
+        if constexpr (DIRECT) {
           float c[PPV], s[PPV];
           tp.read(a.rope_tab, a.npairs, p0, pos.t, pos.h, pos.w, c, s);
 #pragma unroll
           for (int m = 0; m < Q; ++m) {
             cs[m] = make_float2(c[2 * m], c[2 * m + 1]);
             sn[m] = make_float2(s[2 * m], s[2 * m + 1]);
+          }
+        } else if constexpr (STAGE) {
+          const float *tr = tabr + ((it % TS) * R + q) * 2 * kMaxPairs + p0;
+#pragma unroll
+          for (int m = 0; m < Q; ++m) {
+            cs[m] = *reinterpret_cast<const float2 *>(tr + 2 * m);
+            sn[m] = *reinterpret_cast<const float2 *>(tr + kMaxPairs + 2 * m);
           }
         } else {
 #pragma unroll
@@ -317,18 +385,19 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
 }
 
 // One launch of a fixed configuration: a wave of as many CTAs as fit.
-template <typename T, int G, int NT, int VPT, int R, int S, bool TAB, int K = 0, bool BAR = false>
+template <typename T, int G, int NT, int VPT, int R, int S, bool TAB, int K = 0, bool BAR = false,
+          bool STAGE = false>
 cudaError_t launch_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
-  const void *fn =
-      reinterpret_cast<const void *>(&qknorm_rope3d_kernel<T, G, NT, VPT, R, S, TAB, K, BAR>);
+  const void *fn = reinterpret_cast<const void *>(
+      &qknorm_rope3d_kernel<T, G, NT, VPT, R, S, TAB, K, BAR, STAGE>);
   const size_t smem =
-      (TAB ? 0 : header_bytes<R>()) + static_cast<size_t>(S) * R * 2 * VPT * NT * 16;
+      head_bytes<R, S, TAB, STAGE>() + static_cast<size_t>(S) * R * 2 * VPT * NT * 16;
   const int per_sm = resident_blocks(fn, NT, smem);
   if (per_sm <= 0) return cudaErrorInvalidConfiguration;
   int64_t grid = static_cast<int64_t>(per_sm) * device_sms();
   if (grid > a.rows) grid = a.rows;
   if (geo) *geo = Geometry{NT, VPT, S, smem, static_cast<int>(grid)};
-  qknorm_rope3d_kernel<T, G, NT, VPT, R, S, TAB, K, BAR>
+  qknorm_rope3d_kernel<T, G, NT, VPT, R, S, TAB, K, BAR, STAGE>
       <<<static_cast<unsigned>(grid), NT, smem, stream>>>(a);
   return cudaGetLastError();
 }

@@ -68,7 +68,7 @@ __device__ __forceinline__ void int8_codes(float (&u)[N], float ssq, float inv_h
 }
 
 template <int G, int NT, int VPT, int R, int S, bool HALF, bool OUT8, bool TAB, int K = 0,
-          bool BAR = false>
+          bool BAR = false, bool STAGE = false>
 __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
   static_assert(K % R == 0, "a ring stage's rows must lie in one chunk");
   using IO = Io<__nv_bfloat16>;
@@ -77,10 +77,15 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
   constexpr int Q = P / 2;    // float2 lanes of two rotary pairs (interleaved layout)
   constexpr int VB = OUT8 ? 8 : 16;  // output bytes per vector
   constexpr int NPR = HALF ? E : P;  // rotary pairs of one thread's vector
+  // STAGE (table form only): each row's table entries ride in the ring
+  // (stage_table_row) instead of each thread loading its own pairs per row
+  constexpr bool DIRECT = TAB && !STAGE;
+  constexpr int TS = S + 1;  // STAGE's table ring
   constexpr int NTAB = 2 * R * kMaxPairs;
-  constexpr size_t HDR = TAB ? 0 : header_bytes<R>();
+  constexpr size_t HDR = head_bytes<R, S, TAB, STAGE>();
   extern __shared__ __align__(16) unsigned char smem[];
   double *freq = reinterpret_cast<double *>(smem);
+  float *tabr = reinterpret_cast<float *>(smem);  // STAGE: [TS][R][2][kMaxPairs]
   float *cosb = reinterpret_cast<float *>(smem + kMaxPairs * 8);
   float *sinb = cosb + NTAB;
   uint4 *ring = reinterpret_cast<uint4 *>(smem + HDR);
@@ -124,9 +129,9 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
   // per_axis one per section (local pair j of a section of s pairs at
   // theta^(-j/s))
   TabPairs<NPR> tp;
-  if constexpr (TAB) {
+  if constexpr (DIRECT) {
     tp.init(p0, a.sec_t, a.sec_th);
-  } else {
+  } else if constexpr (!TAB) {
     for (int p = tid; p < a.npairs; p += NT) {
       double e = -2.0 * p / a.head_dim;
       if (a.per_axis) {
@@ -160,6 +165,8 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
           for (int k = 0; k < VPT; ++k)
             if (ok[k]) cp_async16(slot(s, q, part, k), ps + k * NT);
         }
+        if constexpr (STAGE)
+          stage_table_row(a, ro.row(j), tabr + ((it % TS) * R + q) * 2 * kMaxPairs);
       }
     }
     cp_async_commit();
@@ -184,7 +191,7 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
                           sinb + buf * R * kMaxPairs);
 
     cp_async_wait<S - 1>();
-    if constexpr (!TAB || BAR) __syncthreads();
+    if constexpr (!DIRECT || BAR) __syncthreads();
 
 #pragma unroll
     for (int q = 0; q < R; ++q) {
@@ -192,8 +199,15 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
       if (j < count) {
         // cos and sin of this thread's NPR pairs p0 .. p0 + NPR - 1
         float ct[NPR], st[NPR];
-        if constexpr (TAB) {
+        if constexpr (DIRECT) {
           tp.read(a.rope_tab, a.npairs, p0, pos.t, pos.h, pos.w, ct, st);
+        } else if constexpr (STAGE) {
+          const float *tr = tabr + ((it % TS) * R + q) * 2 * kMaxPairs + p0;
+#pragma unroll
+          for (int i = 0; i < NPR; ++i) {
+            ct[i] = tr[i];
+            st[i] = tr[kMaxPairs + i];
+          }
         } else {
 #pragma unroll
           for (int i = 0; i < NPR; ++i) {
@@ -335,17 +349,22 @@ constexpr bool kRowSplit = HALF != OUT8;
 // for 8.  Codes go out as two 8-byte stores per lane.  Same ring, row order
 // and (cos, sin) sources as qknorm_rope3d_ex_kernel.
 template <int G2, int NT, int VPT, int R, int S, bool TAB, int K = 0, bool BAR = false,
-          int MINB = 1>
+          int MINB = 1, bool STAGE = false>
 __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkArgs a) {
   static_assert(K % R == 0, "a ring stage's rows must lie in one chunk");
   static_assert(NT % G2 == 0 && 32 % G2 == 0, "a head's lanes must share a warp");
   using IO = Io<__nv_bfloat16>;
   constexpr int P = 4;  // rotary pairs per 16-byte chunk
   constexpr int Q = 2;  // float2 lanes of (pair 2m, pair 2m+1) per chunk
+  // STAGE (table form only): each row's table entries ride in the ring
+  // (stage_table_row) instead of each lane loading its own pairs per row
+  constexpr bool DIRECT = TAB && !STAGE;  // lanes read the table themselves
+  constexpr int TS = S + 1;               // STAGE's table ring
   constexpr int NTAB = 2 * R * kMaxPairs;
-  constexpr size_t HDR = TAB ? 0 : header_bytes<R>();
+  constexpr size_t HDR = head_bytes<R, S, TAB, STAGE>();
   extern __shared__ __align__(16) unsigned char smem[];
   double *freq = reinterpret_cast<double *>(smem);
+  float *tabr = reinterpret_cast<float *>(smem);  // STAGE: [TS][R][2][kMaxPairs]
   float *cosb = reinterpret_cast<float *>(smem + kMaxPairs * 8);
   float *sinb = cosb + NTAB;
   uint4 *ring = reinterpret_cast<uint4 *>(smem + HDR);  // [S][R][2][VPT][2][NT]
@@ -378,10 +397,10 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
     }
   }
   TabPairs<P> tp[2];
-  if constexpr (TAB) {
+  if constexpr (DIRECT) {
     tp[0].init(p0[0], a.sec_t, a.sec_th);
     tp[1].init(p0[1], a.sec_t, a.sec_th);
-  } else {
+  } else if constexpr (!TAB) {
     for (int p = tid; p < a.npairs; p += NT) {
       double e = -2.0 * p / a.head_dim;
       if (a.per_axis) {
@@ -425,6 +444,8 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
             }
           }
         }
+        if constexpr (STAGE)
+          stage_table_row(a, ro.row(j), tabr + ((it % TS) * R + q) * 2 * kMaxPairs);
       }
     }
     cp_async_commit();
@@ -432,7 +453,7 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
 
 #pragma unroll
   for (int s = 0; s < S - 1; ++s) issue(s, s);
-  if constexpr (!TAB) __syncthreads();
+  if constexpr (!TAB) __syncthreads();  // freq[] visible
 
   TokenCursor tok;
   GridCursor pos;
@@ -448,7 +469,7 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
       angle_tables<R, NT>(a, freq, tok, pos, cosb + buf * R * kMaxPairs,
                           sinb + buf * R * kMaxPairs);
     cp_async_wait<S - 1>();
-    if constexpr (!TAB || BAR) __syncthreads();
+    if constexpr (!DIRECT || BAR) __syncthreads();
 
 #pragma unroll
     for (int q = 0; q < R; ++q) {
@@ -458,8 +479,15 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
         float ct[2][P], st[2][P];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          if constexpr (TAB) {
+          if constexpr (DIRECT) {
             tp[h].read(a.rope_tab, a.npairs, p0[h], pos.t, pos.h, pos.w, ct[h], st[h]);
+          } else if constexpr (STAGE) {
+            const float *tr = tabr + ((it % TS) * R + q) * 2 * kMaxPairs + p0[h];
+#pragma unroll
+            for (int i = 0; i < P; ++i) {
+              ct[h][i] = tr[i];
+              st[h][i] = tr[kMaxPairs + i];
+            }
           } else {
 #pragma unroll
             for (int i = 0; i < P; ++i) {
@@ -540,36 +568,36 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
 }
 
 template <int G2, int NT, int VPT, int R, int S, bool TAB, int K = 0, bool BAR = false,
-          int MINB = 1>
+          int MINB = 1, bool STAGE = false>
 cudaError_t launch_int8w_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
   const void *fn = reinterpret_cast<const void *>(
-      &qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, BAR, MINB>);
+      &qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, BAR, MINB, STAGE>);
   const size_t smem =
-      (TAB ? 0 : header_bytes<R>()) + static_cast<size_t>(S) * R * 2 * VPT * 2 * NT * 16;
+      head_bytes<R, S, TAB, STAGE>() + static_cast<size_t>(S) * R * 2 * VPT * 2 * NT * 16;
   const int per_sm = resident_blocks(fn, NT, smem);
   if (per_sm <= 0) return cudaErrorInvalidConfiguration;
   int64_t grid = static_cast<int64_t>(per_sm) * device_sms();
   if (grid > a.rows) grid = a.rows;
   if (geo) *geo = Geometry{NT, VPT, S, smem, static_cast<int>(grid)};
-  qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, BAR, MINB>
+  qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, BAR, MINB, STAGE>
       <<<static_cast<unsigned>(grid), NT, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
 // One launch of a fixed configuration: a wave of as many CTAs as fit.
 template <int G, int NT, int VPT, int R, int S, bool HALF, bool OUT8, bool TAB, int K = 0,
-          bool BAR = false>
+          bool BAR = false, bool STAGE = false>
 cudaError_t launch_ex_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
   const void *fn = reinterpret_cast<const void *>(
-      &qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8, TAB, K, BAR>);
+      &qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8, TAB, K, BAR, STAGE>);
   const size_t smem =
-      (TAB ? 0 : header_bytes<R>()) + static_cast<size_t>(S) * R * 2 * VPT * NT * 16;
+      head_bytes<R, S, TAB, STAGE>() + static_cast<size_t>(S) * R * 2 * VPT * NT * 16;
   const int per_sm = resident_blocks(fn, NT, smem);
   if (per_sm <= 0) return cudaErrorInvalidConfiguration;
   int64_t grid = static_cast<int64_t>(per_sm) * device_sms();
   if (grid > a.rows) grid = a.rows;
   if (geo) *geo = Geometry{NT, VPT, S, smem, static_cast<int>(grid)};
-  qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8, TAB, K, BAR>
+  qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8, TAB, K, BAR, STAGE>
       <<<static_cast<unsigned>(grid), NT, smem, stream>>>(a);
   return cudaGetLastError();
 }
@@ -584,8 +612,9 @@ cudaError_t launch_ex_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
 //    instruction issue rather than DRAM and gained nothing from chunks
 //    (0.84 against 0.80 ms);
 //  - table-driven: one row per stage, two stages, chunks of kTabChunk and
-//    a barrier per stage: 0.857 ms in [B, H, L, hd], 0.809 ms half-split
-//    (6.4 TB/s), 0.854 ms INT8.
+//    a barrier per stage, each thread reading its table entries: 0.809 ms
+//    half-split (6.4 TB/s).  (Interleaved bf16 from the table takes
+//    dispatch_ex_tab_interleaved, interleaved INT8 dispatch_i8w.)
 template <int G, int NT, int VPT, bool HALF, bool OUT8, bool TAB>
 cudaError_t launch_ex(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
   if constexpr (TAB) {
@@ -611,15 +640,36 @@ cudaError_t dispatch_ex(const QkArgs &a, int threads, int vpt, cudaStream_t stre
   return cudaErrorInvalidValue;
 }
 
+// Table form of interleaved bf16 output: the table's split (pick_split_tab,
+// 320 x 2 at D = 5120), one row per stage, two stages, chunks of kTabChunk,
+// table entries staged through the ring (STAGE): 0.844 ms in [B, H, L, hd]
+// at the 5 s clip, against 0.885 ms for the QK split with direct table
+// reads and 0.856 ms on the fly, in one session.
+template <int G>
+cudaError_t dispatch_ex_tab_interleaved(const QkArgs &a, int threads, int vpt,
+                                        cudaStream_t stream, Geometry *geo) {
+#define SOL_CASE(NT, V)                                                                        \
+  if (threads == NT && vpt == V)                                                               \
+    return launch_ex_cfg<G, NT, V, 1, 2, false, false, true, kTabChunk, true, true>(a, stream, \
+                                                                                    geo);
+  SOL_QK_TAB_SPLITS(SOL_CASE)
+#undef SOL_CASE
+  return cudaErrorInvalidValue;
+}
+
 // Interleaved INT8 with 16 elements per lane (qknorm_rope3d_int8w_kernel),
 // G2 = head_dim / 16 lanes per head: one row per stage, two stages and a
-// contiguous share of rows per CTA in both forms (the kernel is issue-bound;
-// chunks and barriers measured no gain), split by pick_split_i8w.
+// contiguous share of rows per CTA in both forms (chunks measured no gain),
+// split by pick_split_i8w.  The table form stages each row's table entries
+// through the ring (STAGE): with 8 warps per SM the lanes' own table loads
+// left their L2 latency exposed (0.868 against 0.749 ms staged, 0.716 ms on
+// the fly, at the 5 s clip in one session).
 template <int G2, bool TAB>
 cudaError_t dispatch_i8w(const QkArgs &a, int threads, int vpt, cudaStream_t stream,
                          Geometry *geo) {
-#define SOL_CASE(NT, V) \
-  if (threads == NT && vpt == V) return launch_int8w_cfg<G2, NT, V, 1, 2, TAB>(a, stream, geo);
+#define SOL_CASE(NT, V)          \
+  if (threads == NT && vpt == V) \
+    return launch_int8w_cfg<G2, NT, V, 1, 2, TAB, 0, false, 1, TAB>(a, stream, geo);
   SOL_I8W_SPLITS(SOL_CASE)
 #undef SOL_CASE
   return cudaErrorInvalidValue;
@@ -644,6 +694,17 @@ cudaError_t launch_ex_form(const QkArgs &a, bool half, cudaStream_t stream, Geom
       }
     }
   }
+  if constexpr (TAB && !OUT8) {
+    if (!half) {  // interleaved bf16 from the table: its own split, staged entries
+      if (!pick_split_tab(a.nvec_q, &threads, &vpt)) return cudaErrorInvalidValue;
+      switch (G) {
+        case 8: return dispatch_ex_tab_interleaved<8>(a, threads, vpt, stream, geo);
+        case 16: return dispatch_ex_tab_interleaved<16>(a, threads, vpt, stream, geo);
+        case 32: return dispatch_ex_tab_interleaved<32>(a, threads, vpt, stream, geo);
+        default: return cudaErrorInvalidValue;
+      }
+    }
+  }
   // the split rule of kRowSplit, which dispatch_ex instantiates
   const bool row = half ? kRowSplit<true, OUT8> : kRowSplit<false, OUT8>;
   const bool split =
@@ -652,7 +713,7 @@ cudaError_t launch_ex_form(const QkArgs &a, bool half, cudaStream_t stream, Geom
   switch (G) {
 #define SOL_G(g)                                                                     \
   case g:                                                                            \
-    if constexpr (OUT8) { /* half-split: interleaved INT8 returned above */           \
+    if constexpr (OUT8 || TAB) { /* interleaved: returned above */                    \
       return dispatch_ex<g, true, OUT8, TAB>(a, threads, vpt, stream, geo);          \
     } else {                                                                         \
       return half ? dispatch_ex<g, true, OUT8, TAB>(a, threads, vpt, stream, geo)    \

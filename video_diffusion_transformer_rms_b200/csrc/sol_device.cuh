@@ -30,6 +30,20 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
                : "memory");
 }
 
+// 4-byte global -> shared copy through L1 (the .cg form copies 16 bytes only).
+__device__ __forceinline__ void cp_async4(void *smem_dst, const void *gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+
+// 16-byte global -> shared copy through L1 (for small data many CTAs re-read).
+__device__ __forceinline__ void cp_async16_ca(void *smem_dst, const void *gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;\n" ::: "memory");
 }
