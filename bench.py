@@ -375,11 +375,6 @@ def run_ours(args):
     value, total_units, slowest = dist.job_throughput(w.rows * K, elapsed_s)
     per_kernel_ms = {k: dist.max_over_ranks(v) for k, v in per_kernel_ms.items()}
 
-    # ---- every config: each step kernel on its own (before the next rows:
-    # the GEMM runs at the power cap and the kernels right after it ran slow)
-    peak, peak_kind = load_peak()
-    configs = {c: time_config(WORKLOADS[c], dev, stream, peak) for c in PER_CONFIG}
-
     # ---- next-row kernels, timed on their own after the step -------------
     ws = torch.empty(_abi.sol_residual_change_workspace_bytes(w.B), dtype=torch.uint8,
                      device=dev)
@@ -460,6 +455,12 @@ def run_ours(args):
                            "bytes_per_token": bytes_per_row,
                            "GB_per_s": round(nbytes / (ms / 1e3) / 1e9, 1)}
     del ws, q8, s8, v8, vs8
+
+    # ---- every config: each step kernel on its own (before the GEMM: it runs
+    # at the power cap, and the kernels right after it ran slow) -----------
+    peak, peak_kind = load_peak()
+    configs = {c: time_config(WORKLOADS[c], dev, stream, peak) for c in PER_CONFIG}
+
     next_rows["gemm_gelu"] = time_gemm_gelu(w, D, dev, stream)
 
 

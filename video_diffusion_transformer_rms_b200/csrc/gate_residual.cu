@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(NT) gate_residual_kernel(const GateArgs a) {
 #pragma unroll
   for (int k = 0; k < VPT; ++k) ok[k] = k * NT + tid < a.nvec;
 
-  RowOrder<K> ro;
+  RowOrder<K, R> ro;
   ro.init(a.rows);
   const int count = ro.count;
   const int iters = (count + R - 1) / R;

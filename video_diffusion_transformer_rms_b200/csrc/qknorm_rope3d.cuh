@@ -256,7 +256,9 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_kernel(const QkArgs a) {
       freq[p] = pow(static_cast<double>(a.theta), -2.0 * p / a.head_dim);
   }
 
-  RowOrder<K> ro;
+  // chunks of at least 4 rows: each chunk restarts the row and position
+  // cursors with divisions, which 1- or 2-row chunks made visible
+  RowOrder<K, (K < 4 ? (K > R ? K : R) : 4)> ro;
   ro.init(a.rows);
   const int count = ro.count;
   const int iters = (count + R - 1) / R;

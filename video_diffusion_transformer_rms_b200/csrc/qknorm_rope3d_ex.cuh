@@ -144,7 +144,9 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
     }
   }
 
-  RowOrder<K> ro;
+  // chunks of at least 4 rows: each chunk restarts the row and position
+  // cursors with divisions, which 1- or 2-row chunks made visible
+  RowOrder<K, (K < 4 ? (K > R ? K : R) : 4)> ro;
   ro.init(a.rows);
   const int count = ro.count;
   const int iters = (count + R - 1) / R;
@@ -413,7 +415,9 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
     }
   }
 
-  RowOrder<K> ro;
+  // chunks of at least 4 rows: each chunk restarts the row and position
+  // cursors with divisions, which 1- or 2-row chunks made visible
+  RowOrder<K, (K < 4 ? (K > R ? K : R) : 4)> ro;
   ro.init(a.rows);
   const int count = ro.count;
   const int iters = (count + R - 1) / R;

@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(NT) rms_adaln_kernel(const RmsArgs a) {
   for (int i = tid; i < 2 * R * 32; i += NT) red[i] = 0.f;  // unused warp slots read 0
   __syncthreads();
 
-  RowOrder<K> ro;  // the CTA's rows, walked with local index j
+  RowOrder<K, R> ro;  // the CTA's rows, walked with local index j
   ro.init(a.rows);
   const int count = ro.count;
   const int iters = (count + R - 1) / R;

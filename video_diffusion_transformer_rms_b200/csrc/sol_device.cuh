@@ -176,22 +176,33 @@ __device__ __forceinline__ void cta_rows(int64_t rows, int64_t cta, int64_t ctas
 }
 
 // The rows one CTA streams, in order.  K == 0: the CTA's contiguous share
-// (cta_rows).  K > 0: chunks of K consecutive rows dealt round-robin, chunk
-// c to CTA c mod gridDim.x, so that at any moment the grid works through one
-// contiguous window of about K * gridDim.x rows instead of gridDim.x
-// far-apart streams.  Rows within a chunk (or a share) are consecutive.
-template <int K>
+// (cta_rows).  K > 0: chunks of consecutive rows dealt round-robin, chunk c
+// to CTA c mod gridDim.x, so that at any moment the grid works through one
+// contiguous window of the tensors instead of gridDim.x far-apart streams.
+// The chunk is K rows, halved (down to KMIN, at least the rows of one ring
+// stage) while the CTAs would get fewer than 16 chunks each: with few rows
+// per CTA a large chunk leaves some CTAs one chunk more than others, a tail
+// of up to K rows.  K and KMIN are powers of two.  Rows within a chunk (or a
+// share) are consecutive.
+template <int K, int KMIN = 1>
 struct RowOrder {
+  static_assert(K == 0 || (K % KMIN == 0 && (K & (K - 1)) == 0 && (KMIN & (KMIN - 1)) == 0),
+                "chunk sizes are powers of two");
   int64_t begin;  // K == 0: first row of the share
   int count;      // rows of this CTA
+  int ks;         // log2 of the chunk size
   __device__ __forceinline__ void init(int64_t rows) {
     if constexpr (K == 0) {
       cta_rows(rows, blockIdx.x, gridDim.x, begin, count);
+      ks = 0;
     } else {
-      const int64_t chunks = (rows + K - 1) / K, c = blockIdx.x, g = gridDim.x;
+      int k = K;
+      while (k > KMIN && rows < static_cast<int64_t>(gridDim.x) * k * 16) k >>= 1;
+      ks = 31 - __clz(k);
+      const int64_t chunks = (rows + k - 1) >> ks, c = blockIdx.x, g = gridDim.x;
       const int64_t mine = c < chunks ? (chunks - 1 - c) / g + 1 : 0;
-      int64_t n = mine * K;
-      if (mine > 0 && c + (mine - 1) * g == chunks - 1) n -= chunks * K - rows;  // last chunk
+      int64_t n = mine << ks;
+      if (mine > 0 && c + (mine - 1) * g == chunks - 1) n -= (chunks << ks) - rows;  // last
       begin = 0;
       count = static_cast<int>(n);
     }
@@ -201,7 +212,8 @@ struct RowOrder {
     if constexpr (K == 0) {
       return begin + j;
     } else {
-      return (static_cast<int64_t>(j / K) * gridDim.x + blockIdx.x) * K + j % K;
+      return ((static_cast<int64_t>(j >> ks) * gridDim.x + blockIdx.x) << ks) +
+             (j & ((1 << ks) - 1));
     }
   }
   // row j is the first of a run of consecutive rows (row cursors restart)
@@ -209,7 +221,7 @@ struct RowOrder {
     if constexpr (K == 0) {
       return j == 0;
     } else {
-      return j % K == 0;
+      return (j & ((1 << ks) - 1)) == 0;
     }
   }
 };
