@@ -889,3 +889,47 @@ def test_rope_table_too_small_or_overlapping_is_rejected():
     pa = api.RopeTable(5, hd, per_axis_freq=True, device=DEV)
     with pytest.raises(ValueError):
         api.qknorm_rope3d_ex(qkv, T, H, W, na, nh, hd, table=pa)
+
+
+# ----------------------------------------------------------------------------
+# Row order: the chunk of rows dealt to each CTA shrinks for small inputs
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("rows", [5000, 18945, 37887, 47361, 94721])
+def test_row_order_regimes(rows):
+    # The kernels deal rows to CTAs in chunks of up to 8 rows, halved while
+    # the CTAs would get fewer than 16 chunks; row counts on both sides of the
+    # B200's halving points (resident CTAs x chunk x 16) take different chunk
+    # sizes.  Every row must come out once and right: sampled rows (with the
+    # first, the last and the video/audio boundary) against the oracle, and
+    # the whole output against the same rows in two calls, bit for bit (each
+    # row's arithmetic does not depend on which CTA takes it).
+    D, nv = 5120, rows - 97
+    x = activation(rows, D, torch.bfloat16, DEV, 201, outliers=True)
+    h = activation(rows, D, torch.bfloat16, DEV, 202, outliers=True)
+    br = activation(rows, D, torch.bfloat16, DEV, 203, outliers=True)
+    sc = vectors((1, 2, D), 0.0, 0.5, torch.bfloat16, DEV, 204)
+    sh = vectors((1, 2, D), 0.0, 0.5, torch.bfloat16, DEV, 205)
+    gt = vectors((1, 2, D), 0.0, 0.1, torch.bfloat16, DEV, 206)
+    y = api.rms_adaln(x.view(1, rows, D), sc, sh, nv)
+    out = api.gate_residual(h.view(1, rows, D), br.view(1, rows, D), gt, nv)
+    torch.cuda.synchronize()
+    ids = sample_rows(rows, rows, nv, 1, 256, seed=207)
+    ids = np.unique(np.concatenate([ids, [0, rows - 1, nv - 1, nv]]))
+    assert_close(take_rows_gpu(y.view(rows, D), ids),
+                 oracle.rms_adaln(take_rows(x, ids), _o(sc), _o(sh), rows, nv, 1e-6,
+                                  row_ids=ids), f"rms rows={rows}")
+    assert_close(take_rows_gpu(out.view(rows, D), ids),
+                 oracle.gate_residual(take_rows(h, ids), take_rows(br, ids), _o(gt), rows, nv,
+                                      row_ids=ids), f"gate rows={rows}")
+    # the same rows in two calls (other row counts, so other chunk sizes and
+    # other CTAs per row): bit-identical to the one call
+    k = rows // 3
+    y2 = torch.cat([api.rms_adaln(x[:k].view(1, k, D), sc, sh, k),
+                    api.rms_adaln(x[k:].view(1, rows - k, D), sc, sh, nv - k)], dim=1)
+    o2 = torch.cat([api.gate_residual(h[:k].view(1, k, D), br[:k].view(1, k, D), gt, k),
+                    api.gate_residual(h[k:].view(1, rows - k, D), br[k:].view(1, rows - k, D),
+                                      gt, nv - k)], dim=1)
+    torch.cuda.synchronize()
+    assert torch.equal(y2, y)
+    assert torch.equal(o2, out)
