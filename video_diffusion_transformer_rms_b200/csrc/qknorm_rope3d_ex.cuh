@@ -351,7 +351,7 @@ constexpr bool kRowSplit = HALF != OUT8;
 // for 8.  Codes go out as two 8-byte stores per lane.  Same ring, row order
 // and (cos, sin) sources as qknorm_rope3d_ex_kernel.
 template <int G2, int NT, int VPT, int R, int S, bool TAB, int K = 0, bool BAR = false,
-          int MINB = 1, bool STAGE = false>
+          int MINB = 1, bool STAGE = false, bool PSPLIT = false>
 __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkArgs a) {
   static_assert(K % R == 0, "a ring stage's rows must lie in one chunk");
   static_assert(NT % G2 == 0 && 32 % G2 == 0, "a head's lanes must share a warp");
@@ -369,7 +369,11 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
   float *tabr = reinterpret_cast<float *>(smem);  // STAGE: [TS][R][2][kMaxPairs]
   float *cosb = reinterpret_cast<float *>(smem + kMaxPairs * 8);
   float *sinb = cosb + NTAB;
-  uint4 *ring = reinterpret_cast<uint4 *>(smem + HDR);  // [S][R][2][VPT][2][NT]
+  // PSPLIT: a CTA takes one part, q (even blockIdx) or k (odd), of the rows
+  // its pair of CTAs shares: half the ring and half the gamma registers
+  constexpr int NP = PSPLIT ? 1 : 2;
+  const int pbase = PSPLIT ? static_cast<int>(blockIdx.x & 1) : 0;
+  uint4 *ring = reinterpret_cast<uint4 *>(smem + HDR);  // [S][R][NP][VPT][2][NT]
 
   const int tid = threadIdx.x;
   const int g = tid % G2;
@@ -384,17 +388,18 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
   for (int k = 0; k < VPT; ++k) ok[k] = k * NT + tid < nslots;
 
   // gamma per part and half in rotary layout, as qknorm_rope3d.cuh
-  float2 gev[2][2][Q], god[2][2][Q];
+  float2 gev[NP][2][Q], god[NP][2][Q];
 #pragma unroll
-  for (int part = 0; part < 2; ++part) {
+  for (int pi = 0; pi < NP; ++pi) {
+    const int part = pbase + pi;
     const uint4 *gp = static_cast<const uint4 *>(part == 0 ? a.gamma_q : a.gamma_k);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       if (gp) {
-        IO::unpack_eo(ld_shared_vec(gp + g + h * G2), gev[part][h], god[part][h]);
+        IO::unpack_eo(ld_shared_vec(gp + g + h * G2), gev[pi][h], god[pi][h]);
       } else {
 #pragma unroll
-        for (int m = 0; m < Q; ++m) gev[part][h][m] = god[part][h][m] = splat2(1.f);
+        for (int m = 0; m < Q; ++m) gev[pi][h][m] = god[pi][h][m] = splat2(1.f);
       }
     }
   }
@@ -418,12 +423,16 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
   // chunks of at least 4 rows: each chunk restarts the row and position
   // cursors with divisions, which 1- or 2-row chunks made visible
   RowOrder<K, (K < 4 ? (K > R ? K : R) : 4)> ro;
-  ro.init(a.rows);
+  if constexpr (PSPLIT) {
+    ro.init(a.rows, static_cast<int>(blockIdx.x >> 1), static_cast<int>(gridDim.x >> 1));
+  } else {
+    ro.init(a.rows);
+  }
   const int count = ro.count;
   const int iters = (count + R - 1) / R;
   const unsigned char *qkv = static_cast<const unsigned char *>(a.qkv);
-  auto slot = [&](int s, int q, int part, int k, int h) -> uint4 * {
-    return &ring[((((s * R + q) * 2 + part) * VPT + k) * 2 + h) * NT + tid];
+  auto slot = [&](int s, int q, int pi, int k, int h) -> uint4 * {
+    return &ring[((((s * R + q) * NP + pi) * VPT + k) * 2 + h) * NT + tid];
   };
   // chunk index in a part of the first chunk of slot k: head * 2 * G2 + g
   auto chunk0 = [&](int k) -> int {
@@ -437,14 +446,14 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
       if (j < count) {
         const unsigned char *src = qkv + ro.row(j) * a.ld_qkv_bytes;
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const uint4 *ps = reinterpret_cast<const uint4 *>(src + part * part_bytes);
+        for (int pi = 0; pi < NP; ++pi) {
+          const uint4 *ps = reinterpret_cast<const uint4 *>(src + (pbase + pi) * part_bytes);
 #pragma unroll
           for (int k = 0; k < VPT; ++k) {
             if (ok[k]) {
               const int c = chunk0(k);
-              cp_async16(slot(s, q, part, k, 0), ps + c);
-              cp_async16(slot(s, q, part, k, 1), ps + c + G2);
+              cp_async16(slot(s, q, pi, k, 0), ps + c);
+              cp_async16(slot(s, q, pi, k, 1), ps + c + G2);
             }
           }
         }
@@ -504,7 +513,8 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
         const int64_t row_off = static_cast<int64_t>(tok.b) * a.out_sb +
                                 static_cast<int64_t>(tok.r) * a.out_sr;
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
+        for (int pi = 0; pi < NP; ++pi) {
+          const int part = pbase + pi;
           // rotation coefficients of this lane's pairs, gamma folded in
           float2 c0[2][Q], ns1[2][Q], s0[2][Q], c1[2][Q];
 #pragma unroll
@@ -513,10 +523,10 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
             for (int m = 0; m < Q; ++m) {
               const float2 cs = make_float2(ct[h][2 * m], ct[h][2 * m + 1]);
               const float2 sn = make_float2(st[h][2 * m], st[h][2 * m + 1]);
-              c0[h][m] = mul2(gev[part][h][m], cs);
-              s0[h][m] = mul2(gev[part][h][m], sn);
-              ns1[h][m] = mul2(god[part][h][m], make_float2(-sn.x, -sn.y));
-              c1[h][m] = mul2(god[part][h][m], cs);
+              c0[h][m] = mul2(gev[pi][h][m], cs);
+              s0[h][m] = mul2(gev[pi][h][m], sn);
+              ns1[h][m] = mul2(god[pi][h][m], make_float2(-sn.x, -sn.y));
+              c1[h][m] = mul2(god[pi][h][m], cs);
             }
           }
           unsigned char *obase = static_cast<unsigned char *>(part == 0 ? a.q_out : a.k_out) +
@@ -531,7 +541,7 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-              if (ok[k]) xv = *slot(cons, q, part, k, h);
+              if (ok[k]) xv = *slot(cons, q, pi, k, h);
               float2 ev[Q], od[Q];
               IO::unpack_eo(xv, ev, od);
 #pragma unroll
@@ -572,18 +582,25 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
 }
 
 template <int G2, int NT, int VPT, int R, int S, bool TAB, int K = 0, bool BAR = false,
-          int MINB = 1, bool STAGE = false>
+          int MINB = 1, bool STAGE = false, bool PSPLIT = false>
 cudaError_t launch_int8w_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
   const void *fn = reinterpret_cast<const void *>(
-      &qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, BAR, MINB, STAGE>);
+      &qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, BAR, MINB, STAGE, PSPLIT>);
+  constexpr int NP = PSPLIT ? 1 : 2;
   const size_t smem =
-      head_bytes<R, S, TAB, STAGE>() + static_cast<size_t>(S) * R * 2 * VPT * 2 * NT * 16;
+      head_bytes<R, S, TAB, STAGE>() + static_cast<size_t>(S) * R * NP * VPT * 2 * NT * 16;
   const int per_sm = resident_blocks(fn, NT, smem);
   if (per_sm <= 0) return cudaErrorInvalidConfiguration;
   int64_t grid = static_cast<int64_t>(per_sm) * device_sms();
-  if (grid > a.rows) grid = a.rows;
+  if (PSPLIT) {  // pairs of CTAs (q, k) over the same rows
+    grid &= ~static_cast<int64_t>(1);
+    if (grid > 2 * a.rows) grid = 2 * a.rows;
+    if (grid < 2) grid = 2;
+  } else if (grid > a.rows) {
+    grid = a.rows;
+  }
   if (geo) *geo = Geometry{NT, VPT, S, smem, static_cast<int>(grid)};
-  qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, BAR, MINB, STAGE>
+  qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, BAR, MINB, STAGE, PSPLIT>
       <<<static_cast<unsigned>(grid), NT, smem, stream>>>(a);
   return cudaGetLastError();
 }
@@ -668,12 +685,19 @@ cudaError_t dispatch_ex_tab_interleaved(const QkArgs &a, int threads, int vpt,
 // through the ring (STAGE): with 8 warps per SM the lanes' own table loads
 // left their L2 latency exposed (0.868 against 0.749 ms staged, 0.716 ms on
 // the fly, at the 5 s clip in one session).
+//
+// Each CTA takes one part, q or k, of the rows it shares with its pair
+// (PSPLIT): half the ring and half the gamma registers per CTA, so more CTAs
+// fit.  The table form also caps registers at 128 (512 threads' worth of
+// CTAs per SM): in one session 0.800 -> 0.739 ms with both, on the fly
+// 0.699 -> 0.688 ms with the split alone.
 template <int G2, bool TAB>
 cudaError_t dispatch_i8w(const QkArgs &a, int threads, int vpt, cudaStream_t stream,
                          Geometry *geo) {
-#define SOL_CASE(NT, V)          \
-  if (threads == NT && vpt == V) \
-    return launch_int8w_cfg<G2, NT, V, 1, 2, TAB, 0, false, 1, TAB>(a, stream, geo);
+#define SOL_CASE(NT, V)                                                                       \
+  if (threads == NT && vpt == V)                                                              \
+    return launch_int8w_cfg<G2, NT, V, 1, 2, TAB, 0, false, (TAB ? 512 / NT : 1), TAB, true>( \
+        a, stream, geo);
   SOL_I8W_SPLITS(SOL_CASE)
 #undef SOL_CASE
   return cudaErrorInvalidValue;

@@ -191,15 +191,19 @@ struct RowOrder {
   int64_t begin;  // K == 0: first row of the share
   int count;      // rows of this CTA
   int ks;         // log2 of the chunk size
-  __device__ __forceinline__ void init(int64_t rows) {
+  int cta, ctas;  // this CTA's index among the CTAs that share the rows
+  __device__ __forceinline__ void init(int64_t rows) { init(rows, blockIdx.x, gridDim.x); }
+  __device__ __forceinline__ void init(int64_t rows, int cta_, int ctas_) {
+    cta = cta_;
+    ctas = ctas_;
     if constexpr (K == 0) {
-      cta_rows(rows, blockIdx.x, gridDim.x, begin, count);
+      cta_rows(rows, cta, ctas, begin, count);
       ks = 0;
     } else {
       int k = K;
-      while (k > KMIN && rows < static_cast<int64_t>(gridDim.x) * k * 16) k >>= 1;
+      while (k > KMIN && rows < static_cast<int64_t>(ctas) * k * 16) k >>= 1;
       ks = 31 - __clz(k);
-      const int64_t chunks = (rows + k - 1) >> ks, c = blockIdx.x, g = gridDim.x;
+      const int64_t chunks = (rows + k - 1) >> ks, c = cta, g = ctas;
       const int64_t mine = c < chunks ? (chunks - 1 - c) / g + 1 : 0;
       int64_t n = mine << ks;
       if (mine > 0 && c + (mine - 1) * g == chunks - 1) n -= (chunks << ks) - rows;  // last
@@ -212,8 +216,7 @@ struct RowOrder {
     if constexpr (K == 0) {
       return begin + j;
     } else {
-      return ((static_cast<int64_t>(j >> ks) * gridDim.x + blockIdx.x) << ks) +
-             (j & ((1 << ks) - 1));
+      return ((static_cast<int64_t>(j >> ks) * ctas + cta) << ks) + (j & ((1 << ks) - 1));
     }
   }
   // row j is the first of a run of consecutive rows (row cursors restart)
