@@ -658,12 +658,21 @@ def test_qknorm_rope3d_ex_per_axis_sections(secs, tab):
     gk = vectors((hd,), 1.0, 0.1, torch.bfloat16, DEV, 83)
     table = _table(tab, T, H, W, na, hd, secs, per_axis=True)
     for half in (False, True):
-        q, k = api.qknorm_rope3d_ex(qkv, T, H, W, na, nh, hd, secs, gq, gk, half_split=half,
-                                    per_axis_freq=True, table=table)
         wq, wk = oracle.qknorm_rope3d_ex(_o(qkv.view(B * L, 3 * D)), T, H, W, na, nh, hd, secs,
                                          1e-6, 1e4, half, _o(gq), _o(gk), per_axis=True)
+        q, k = api.qknorm_rope3d_ex(qkv, T, H, W, na, nh, hd, secs, gq, gk, half_split=half,
+                                    per_axis_freq=True, table=table)
         assert_close(q.reshape(B * L, D), wq, f"per-axis sections {secs} half={half} q")
         assert_close(k.reshape(B * L, D), wk, f"per-axis sections {secs} half={half} k")
+        # INT8 too: a section edge inside a lane's 4 pairs (18, 22, 24) takes
+        # the table rows' 4-byte copies
+        q8, k8, qs, ks = api.qknorm_rope3d_ex(qkv, T, H, W, na, nh, hd, secs, gq, gk,
+                                              half_split=half, per_axis_freq=True, int8=True,
+                                              table=table)
+        torch.cuda.synchronize()
+        tag = f"per-axis sections {secs} half={half} int8"
+        _check_int8(q8.reshape(B * L, D), qs, wq, nh, hd, tag + " q")
+        _check_int8(k8.reshape(B * L, D), ks, wk, nh, hd, tag + " k")
 
 
 def test_qknorm_rope3d_packed_qk_input():
@@ -700,6 +709,32 @@ def test_qknorm_rope3d_ex_interleaved_matches_default_entry_point(tab):
         q1, k1 = api.qknorm_rope3d_ex(qkv, *args, layout=layout, table=table)
         assert torch.equal(_bshd(q1, layout).reshape(q0.shape), q0)
         assert torch.equal(_bshd(k1, layout).reshape(k0.shape), k0)
+
+
+INT8_CASES = [c for c in QK_CASES if c[6] >= 64 and c[8] == torch.bfloat16]
+
+
+@pytest.mark.parametrize("B,T,H,W,na,nh,hd,secs,dt,pad", INT8_CASES)
+@ROPE
+def test_qknorm_rope3d_ex_int8_cases(B, T, H, W, na, nh, hd, secs, dt, pad, tab):
+    # the interleaved INT8 kernel on the QK edge shapes: audio only, video
+    # only, one row, a ragged lane tail (41 heads), the widest row, padded
+    # rows, and CTA shares (q and k CTAs of a pair) that cross W, H, the
+    # video/audio split and samples
+    L = T * H * W + na
+    D = nh * hd
+    C = 3 * D + pad
+    qkv = activation(B * L, C, dt, DEV, 91, outliers=True).view(B, L, C)
+    gq = vectors((hd,), 1.0, 0.1, dt, DEV, 92)
+    gk = vectors((hd,), 1.0, 0.1, dt, DEV, 93)
+    q, k, qs, ks = api.qknorm_rope3d_ex(qkv, T, H, W, na, nh, hd, secs, gq, gk, int8=True,
+                                        table=_table(tab, T, H, W, na, hd, secs))
+    torch.cuda.synchronize()
+    wq, wk = oracle.qknorm_rope3d_ex(_o(qkv.view(B * L, C)), T, H, W, na, nh, hd, secs,
+                                     1e-6, 1e4, False, _o(gq), _o(gk))
+    tag = f"int8 B={B} T={T} H={H} W={W} na={na} nh={nh} hd={hd} table={tab}"
+    _check_int8(q.reshape(B * L, D), qs, wq, nh, hd, tag + " q")
+    _check_int8(k.reshape(B * L, D), ks, wk, nh, hd, tag + " k")
 
 
 @pytest.mark.parametrize("hd,secs", [(64, (8, 12, 12)), (256, (32, 48, 48))])

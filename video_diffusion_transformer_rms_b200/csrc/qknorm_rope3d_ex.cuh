@@ -339,44 +339,85 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
 template <bool HALF, bool OUT8>
 constexpr bool kRowSplit = HALF != OUT8;
 
+// Table form of qknorm_rope3d_int8w_kernel: the warp's lanes copy the (cos,
+// sin) of one row at rotary position (t, h, w) into the warp's own
+// dst[2][kMaxPairs], one 16-byte chunk per lane and round (chunk c <
+// npairs/4: cos of pairs 4c .. 4c+3, then the sin chunks), in the cp.async
+// group of the row's data.  Only this warp reads them, so a __syncwarp after
+// the wait orders them and the CTA needs no barrier per stage.
+__device__ __forceinline__ void stage_table_lanes(const QkArgs &a, int t, int h, int w,
+                                                  float *dst, int lane) {
+  const int nq = a.npairs >> 2;
+  const int64_t ld = 2 * static_cast<int64_t>(a.npairs);
+  for (int idx = lane; idx < 2 * nq; idx += 32) {
+    const int which = idx >= nq ? 1 : 0;  // 0: cos, 1: sin
+    const int p = 4 * (idx - which * nq);
+    const float *src = a.rope_tab + which * a.npairs + p;
+    float *d = dst + which * kMaxPairs + p;
+    const int ax0 = pair_axis(p, a.sec_t, a.sec_th);
+    if (ax0 == pair_axis(p + 3, a.sec_t, a.sec_th)) {
+      const int at = ax0 == 0 ? t : (ax0 == 1 ? h : w);
+      cp_async16_ca(d, src + at * ld);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int ax = pair_axis(p + i, a.sec_t, a.sec_th);
+        const int at = ax == 0 ? t : (ax == 1 ? h : w);
+        cp_async4(d + i, src + at * ld + i);
+      }
+    }
+  }
+}
+
+// Shared memory before qknorm_rope3d_int8w_kernel's ring: the table form's
+// per-warp table rows, (S + 1) stages deep (a stage is overwritten only after
+// every lane of the warp passed the __syncwarp that follows its last use), or
+// the on-the-fly form's fp64 frequencies and double-buffered angle tables.
+template <int R, int S, bool TAB, int NT>
+__host__ __device__ constexpr size_t i8w_head_bytes() {
+  return TAB ? static_cast<size_t>(S + 1) * (NT / 32) * R * 2 * kMaxPairs * 4 : header_bytes<R>();
+}
+
 // INT8 output with interleaved pairs, 16 elements per lane.  The INT8
-// epilogue is bound by instruction issue, not DRAM, and most of its
-// per-element cost is per head and lane: the two-value shuffle reduction,
-// the reciprocals and the scale store.  Here G2 = head_dim / 16 lanes share a
-// head (8 at head_dim 128), and lane g owns the head's 16-byte chunks g and
-// g + G2, i.e. pairs 4g .. 4g+3 and 4(g+G2) .. 4(g+G2)+3.  A warp's copy of
-// the first chunks covers whole 128-byte halves of four heads, so every L2
-// sector it touches is used in full, and the second copy the other halves.
-// The reduction runs over G2 lanes for 16 elements instead of 2 * G2 lanes
-// for 8.  Codes go out as two 8-byte stores per lane.  Same ring, row order
-// and (cos, sin) sources as qknorm_rope3d_ex_kernel.
-template <int G2, int NT, int VPT, int R, int S, bool TAB, int K = 0, bool BAR = false,
-          int MINB = 1, bool STAGE = false, bool PSPLIT = false>
+// epilogue is bound by instruction issue and latency, not DRAM, and most of
+// its per-element cost is per head and lane: the two-value shuffle
+// reduction, the reciprocals and the scale store.  Here G2 = head_dim / 16
+// lanes share a head (8 at head_dim 128), and lane g owns the head's 16-byte
+// chunks g and g + G2, i.e. pairs 4g .. 4g+3 and 4(g+G2) .. 4(g+G2)+3.  A
+// warp's copy of the first chunks covers whole 128-byte halves of four heads,
+// so every L2 sector it touches is used in full, and the second copy the
+// other halves.  The reduction runs over G2 lanes for 16 elements instead of
+// 2 * G2 lanes for 8.  Codes go out as two 8-byte stores per lane.
+//
+// PSPLIT: CTA 2i takes the q part and CTA 2i + 1 the k part of the same rows
+// (one row order for the pair), so a CTA holds half a row per ring stage and
+// one part's gamma.  The table form stages each row's (cos, sin) per warp
+// (stage_table_lanes) and has no CTA barrier in its loop; the on-the-fly form
+// builds CTA-wide angle tables behind one barrier per stage.
+template <int G2, int NT, int VPT, int R, int S, bool TAB, int K = 0, int MINB = 1,
+          bool PSPLIT = true>
 __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkArgs a) {
   static_assert(K % R == 0, "a ring stage's rows must lie in one chunk");
-  static_assert(NT % G2 == 0 && 32 % G2 == 0, "a head's lanes must share a warp");
+  static_assert(NT % 32 == 0 && 32 % G2 == 0, "a head's lanes must share a warp");
   using IO = Io<__nv_bfloat16>;
-  constexpr int P = 4;  // rotary pairs per 16-byte chunk
-  constexpr int Q = 2;  // float2 lanes of (pair 2m, pair 2m+1) per chunk
-  // STAGE (table form only): each row's table entries ride in the ring
-  // (stage_table_row) instead of each lane loading its own pairs per row
-  constexpr bool DIRECT = TAB && !STAGE;  // lanes read the table themselves
-  constexpr int TS = S + 1;               // STAGE's table ring
+  constexpr int P = 4;       // rotary pairs per 16-byte chunk
+  constexpr int Q = 2;       // float2 lanes of (pair 2m, pair 2m+1) per chunk
+  constexpr int TS = S + 1;  // the table form's ring of per-warp table rows
+  constexpr int NW = NT / 32;
   constexpr int NTAB = 2 * R * kMaxPairs;
-  constexpr size_t HDR = head_bytes<R, S, TAB, STAGE>();
+  constexpr size_t HDR = i8w_head_bytes<R, S, TAB, NT>();
   extern __shared__ __align__(16) unsigned char smem[];
-  double *freq = reinterpret_cast<double *>(smem);
-  float *tabr = reinterpret_cast<float *>(smem);  // STAGE: [TS][R][2][kMaxPairs]
-  float *cosb = reinterpret_cast<float *>(smem + kMaxPairs * 8);
+  double *freq = reinterpret_cast<double *>(smem);                // on the fly
+  float *cosb = reinterpret_cast<float *>(smem + kMaxPairs * 8);  // on the fly: [2][R][kMaxPairs]
   float *sinb = cosb + NTAB;
-  // PSPLIT: a CTA takes one part, q (even blockIdx) or k (odd), of the rows
-  // its pair of CTAs shares: half the ring and half the gamma registers
+  float *tabw = reinterpret_cast<float *>(smem);  // table: [TS][NW][R][2][kMaxPairs]
   constexpr int NP = PSPLIT ? 1 : 2;
   const int pbase = PSPLIT ? static_cast<int>(blockIdx.x & 1) : 0;
   uint4 *ring = reinterpret_cast<uint4 *>(smem + HDR);  // [S][R][NP][VPT][2][NT]
 
   const int tid = threadIdx.x;
   const int g = tid % G2;
+  const int warp = tid >> 5, lane = tid & 31;
   const int nslots = a.nvec_q / 2;  // (head, lane) slots of one part: n_heads * G2
   const int64_t part_bytes = static_cast<int64_t>(a.nvec_q) * 16;
   int p0[2];  // first pair of each half
@@ -403,11 +444,7 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
       }
     }
   }
-  TabPairs<P> tp[2];
-  if constexpr (DIRECT) {
-    tp[0].init(p0[0], a.sec_t, a.sec_th);
-    tp[1].init(p0[1], a.sec_t, a.sec_th);
-  } else if constexpr (!TAB) {
+  if constexpr (!TAB) {
     for (int p = tid; p < a.npairs; p += NT) {
       double e = -2.0 * p / a.head_dim;
       if (a.per_axis) {
@@ -439,6 +476,12 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
     const int u = k * NT + tid;
     return (u / G2) * (2 * G2) + g;
   };
+  // the table form's table row of issue iteration it, row q, for this warp
+  auto wtab = [&](int it, int q) -> float * {
+    return tabw + (((it % TS) * NW + warp) * R + q) * 2 * kMaxPairs;
+  };
+  TokenCursor itok;  // table form: the row being issued, S - 1 rows ahead
+  GridCursor ipos;
   auto issue = [&](int it, int s) {
 #pragma unroll
     for (int q = 0; q < R; ++q) {
@@ -457,8 +500,15 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
             }
           }
         }
-        if constexpr (STAGE)
-          stage_table_row(a, ro.row(j), tabr + ((it % TS) * R + q) * 2 * kMaxPairs);
+        if constexpr (TAB) {
+          if (ro.run_start(j)) {
+            itok.init(ro.row(j), a.L);
+            ipos.init(itok.r, a.n_video, a.HW, a.W);
+          }
+          stage_table_lanes(a, ipos.t, ipos.h, ipos.w, wtab(it, q), lane);
+          itok.next(a.L);
+          ipos.next(itok.r, a.n_video, a.H, a.W);
+        }
       }
     }
     cp_async_commit();
@@ -476,38 +526,33 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
     issue(it + S - 1, cons == 0 ? S - 1 : cons - 1);
     if (ro.run_start(it * R)) {
       tok.init(ro.row(it * R), a.L);
-      pos.init(tok.r, a.n_video, a.HW, a.W);
+      if constexpr (!TAB) pos.init(tok.r, a.n_video, a.HW, a.W);
     }
     if constexpr (!TAB)
       angle_tables<R, NT>(a, freq, tok, pos, cosb + buf * R * kMaxPairs,
                           sinb + buf * R * kMaxPairs);
     cp_async_wait<S - 1>();
-    if constexpr (!DIRECT || BAR) __syncthreads();
+    if constexpr (TAB) {
+      __syncwarp();  // the warp's table row visible to all its lanes
+    } else {
+      __syncthreads();  // angle tables of these rows visible
+    }
 
 #pragma unroll
     for (int q = 0; q < R; ++q) {
       const int j = it * R + q;
       if (j < count) {
-        // cos and sin of the lane's pairs, per half
+        // cos and sin of the lane's pairs, per half (16-byte aligned: p0 is
+        // a multiple of 4 pairs and table rows are kMaxPairs long)
         float ct[2][P], st[2][P];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          if constexpr (DIRECT) {
-            tp[h].read(a.rope_tab, a.npairs, p0[h], pos.t, pos.h, pos.w, ct[h], st[h]);
-          } else if constexpr (STAGE) {
-            const float *tr = tabr + ((it % TS) * R + q) * 2 * kMaxPairs + p0[h];
-#pragma unroll
-            for (int i = 0; i < P; ++i) {
-              ct[h][i] = tr[i];
-              st[h][i] = tr[kMaxPairs + i];
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < P; ++i) {
-              ct[h][i] = cosb[(buf * R + q) * kMaxPairs + p0[h] + i];
-              st[h][i] = sinb[(buf * R + q) * kMaxPairs + p0[h] + i];
-            }
-          }
+          const float *cr = TAB ? wtab(it, q) + p0[h] : cosb + (buf * R + q) * kMaxPairs + p0[h];
+          const float *sr = TAB ? cr + kMaxPairs : sinb + (buf * R + q) * kMaxPairs + p0[h];
+          const float4 c4 = *reinterpret_cast<const float4 *>(cr);
+          const float4 s4 = *reinterpret_cast<const float4 *>(sr);
+          ct[h][0] = c4.x, ct[h][1] = c4.y, ct[h][2] = c4.z, ct[h][3] = c4.w;
+          st[h][0] = s4.x, st[h][1] = s4.y, st[h][2] = s4.z, st[h][3] = s4.w;
         }
         const int64_t grow = ro.row(j);
         const int64_t row_off = static_cast<int64_t>(tok.b) * a.out_sb +
@@ -572,7 +617,7 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
           }
         }
         tok.next(a.L);
-        pos.next(tok.r, a.n_video, a.H, a.W);
+        if constexpr (!TAB) pos.next(tok.r, a.n_video, a.H, a.W);
       }
     }
     buf ^= 1;
@@ -581,14 +626,14 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
   cp_async_wait<0>();
 }
 
-template <int G2, int NT, int VPT, int R, int S, bool TAB, int K = 0, bool BAR = false,
-          int MINB = 1, bool STAGE = false, bool PSPLIT = false>
+template <int G2, int NT, int VPT, int R, int S, bool TAB, int K = 0, int MINB = 1,
+          bool PSPLIT = true>
 cudaError_t launch_int8w_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
   const void *fn = reinterpret_cast<const void *>(
-      &qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, BAR, MINB, STAGE, PSPLIT>);
+      &qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, MINB, PSPLIT>);
   constexpr int NP = PSPLIT ? 1 : 2;
   const size_t smem =
-      head_bytes<R, S, TAB, STAGE>() + static_cast<size_t>(S) * R * NP * VPT * 2 * NT * 16;
+      i8w_head_bytes<R, S, TAB, NT>() + static_cast<size_t>(S) * R * NP * VPT * 2 * NT * 16;
   const int per_sm = resident_blocks(fn, NT, smem);
   if (per_sm <= 0) return cudaErrorInvalidConfiguration;
   int64_t grid = static_cast<int64_t>(per_sm) * device_sms();
@@ -600,7 +645,7 @@ cudaError_t launch_int8w_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo
     grid = a.rows;
   }
   if (geo) *geo = Geometry{NT, VPT, S, smem, static_cast<int>(grid)};
-  qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, BAR, MINB, STAGE, PSPLIT>
+  qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, MINB, PSPLIT>
       <<<static_cast<unsigned>(grid), NT, smem, stream>>>(a);
   return cudaGetLastError();
 }
@@ -681,23 +726,20 @@ cudaError_t dispatch_ex_tab_interleaved(const QkArgs &a, int threads, int vpt,
 // Interleaved INT8 with 16 elements per lane (qknorm_rope3d_int8w_kernel),
 // G2 = head_dim / 16 lanes per head: one row per stage, two stages and a
 // contiguous share of rows per CTA in both forms (chunks measured no gain),
-// split by pick_split_i8w.  The table form stages each row's table entries
-// through the ring (STAGE): with 8 warps per SM the lanes' own table loads
-// left their L2 latency exposed (0.868 against 0.749 ms staged, 0.716 ms on
-// the fly, at the 5 s clip in one session).
-//
-// Each CTA takes one part, q or k, of the rows it shares with its pair
-// (PSPLIT): half the ring and half the gamma registers per CTA, so more CTAs
-// fit.  The table form also caps registers at 128 (512 threads' worth of
-// CTAs per SM): in one session 0.800 -> 0.739 ms with both, on the fly
-// 0.699 -> 0.688 ms with the split alone.
+// split by pick_split_i8w, q and k on paired CTAs (half the ring and gamma
+// registers per CTA: table form 0.800 -> 0.739 ms, on the fly 0.699 ->
+// 0.688 ms in one session).  The table form caps registers at 128 (512
+// threads' worth of CTAs per SM) and stages each row's table entries per
+// warp, which drops the CTA barrier from its loop: 0.781 -> 0.706 ms in one
+// interleaved session at the 5 s clip (the on-the-fly form 0.713 ms there;
+// staging per CTA behind a barrier, or lanes reading the table themselves,
+// were the slower alternatives).
 template <int G2, bool TAB>
 cudaError_t dispatch_i8w(const QkArgs &a, int threads, int vpt, cudaStream_t stream,
                          Geometry *geo) {
-#define SOL_CASE(NT, V)                                                                       \
-  if (threads == NT && vpt == V)                                                              \
-    return launch_int8w_cfg<G2, NT, V, 1, 2, TAB, 0, false, (TAB ? 512 / NT : 1), TAB, true>( \
-        a, stream, geo);
+#define SOL_CASE(NT, V)                                                                           \
+  if (threads == NT && vpt == V)                                                                  \
+    return launch_int8w_cfg<G2, NT, V, 1, 2, TAB, 0, (TAB ? 512 / NT : 1), true>(a, stream, geo);
   SOL_I8W_SPLITS(SOL_CASE)
 #undef SOL_CASE
   return cudaErrorInvalidValue;
