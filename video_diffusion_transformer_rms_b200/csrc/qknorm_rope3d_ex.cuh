@@ -22,23 +22,31 @@
 namespace sol {
 namespace qk {
 
-// INT8 codes of one lane's N rotated values u[] of a head whose other values
-// sit in the G - 1 partner lanes of its aligned lane group.  1/rms is one
-// positive factor per head, so it cancels from the codes: code =
-// round(u * 127 / max|u|) on the un-normalised rotation, and only the scale
-// max|u| / rms / 127 needs it.  The sum of squares (ssq: this lane's part)
-// and the max reduce side by side.  Codes are rounded half to even (one FMA
-// with kRoundMagic) and packed four to a word, in element order.
-template <int N, int G>
-__device__ __forceinline__ void int8_codes(float (&u)[N], float ssq, float inv_hd, float eps,
-                                           uint32_t (&words)[N / 4], float &scale) {
-  float m[N / 2];
+// INT8 codes of one lane's 2 * NV rotated values of a head, held as NV
+// float2 in the registers the rotation leaves them in, whose other values
+// sit in the G - 1 partner lanes of its aligned lane group.  ROT: v[2w] and
+// v[2w + 1] are the first and the second components of two rotary pairs
+// (elements 4w, 4w+2 and 4w+1, 4w+3), as the interleaved rotation produces
+// them; else v[i] holds elements 2i, 2i+1.  Taking them as they are keeps the
+// packed rounding FMAs free of register moves.  1/rms is one positive factor
+// per head, so it cancels from the codes: code = round(u * 127 / max|u|) on
+// the un-normalised rotation, and only the scale max|u| / rms / 127 needs it.
+// The sum of squares (ssq: this lane's part) and the max reduce side by side.
+// Codes are rounded half to even (one FMA with kRoundMagic) and packed four
+// to a word, in element order.
+template <int NV, int G, bool ROT>
+__device__ __forceinline__ void int8_codes(float2 (&v)[NV], float ssq, float inv_hd, float eps,
+                                           uint32_t (&words)[NV / 2], float &scale) {
+  constexpr int W = NV / 2;  // words, 4 elements each
+  float m[W];
 #pragma unroll
-  for (int e = 0; e < N / 2; ++e) m[e] = fmaxf(fabsf(u[2 * e]), fabsf(u[2 * e + 1]));
+  for (int w = 0; w < W; ++w)
+    m[w] = fmaxf(fmaxf(fabsf(v[2 * w].x), fabsf(v[2 * w].y)),
+                 fmaxf(fabsf(v[2 * w + 1].x), fabsf(v[2 * w + 1].y)));
 #pragma unroll
-  for (int w = N / 4; w > 0; w >>= 1)
+  for (int k = W / 2; k > 0; k >>= 1)
 #pragma unroll
-    for (int e = 0; e < w; ++e) m[e] = fmaxf(m[e], m[e + w]);
+    for (int e = 0; e < k; ++e) m[e] = fmaxf(m[e], m[e + k]);
   float umax = m[0];
 #pragma unroll
   for (int off = G / 2; off > 0; off >>= 1) {
@@ -52,17 +60,20 @@ __device__ __forceinline__ void int8_codes(float (&u)[N], float ssq, float inv_h
   if (umax > 0.f && umax < 0x1p-96f) {
     // a head of (near-)denormal inputs: 127 / umax would overflow, so scale
     // u and umax by 2^64 (exact) first; the codes are unchanged
+    const float2 big = splat2(0x1p64f);
 #pragma unroll
-    for (int e = 0; e < N; ++e) u[e] *= 0x1p64f;
+    for (int e = 0; e < NV; ++e) v[e] = mul2(v[e], big);
     is = __fdividef(127.f, umax * 0x1p64f);
   }
   const float2 is2 = splat2(is), magic2 = splat2(kRoundMagic);
 #pragma unroll
-  for (int w = 0; w < N / 4; ++w) {
-    const float2 r0 = fma2(make_float2(u[4 * w], u[4 * w + 1]), is2, magic2);
-    const float2 r1 = fma2(make_float2(u[4 * w + 2], u[4 * w + 3]), is2, magic2);
-    words[w] = pack_low_bytes(__float_as_uint(r0.x), __float_as_uint(r0.y),
-                              __float_as_uint(r1.x), __float_as_uint(r1.y));
+  for (int w = 0; w < W; ++w) {
+    const float2 r0 = fma2(v[2 * w], is2, magic2);
+    const float2 r1 = fma2(v[2 * w + 1], is2, magic2);
+    words[w] = ROT ? pack_low_bytes(__float_as_uint(r0.x), __float_as_uint(r1.x),
+                                    __float_as_uint(r0.y), __float_as_uint(r1.y))
+                   : pack_low_bytes(__float_as_uint(r0.x), __float_as_uint(r0.y),
+                                    __float_as_uint(r1.x), __float_as_uint(r1.y));
   }
   scale = umax * inv * (1.f / 127.f);
 }
@@ -257,6 +268,7 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
             // rotated outputs in element order, not yet multiplied by the
             // head's 1/rms; acc: this thread's part of the sum of squares
             float o[E];
+            float2 uv[P];  // the same values as pairs, for int8_codes
             float2 acc;
             if constexpr (HALF) {
               uint4 pv;
@@ -275,6 +287,7 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
                 const float2 u = fma2(own[m], ca[m], mul2(par[m], sb[m]));
                 o[2 * m] = u.x;
                 o[2 * m + 1] = u.y;
+                uv[m] = u;
               }
             } else {
               float2 ev[Q], od[Q];
@@ -294,6 +307,8 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
                 o[4 * m + 1] = u1.x;
                 o[4 * m + 2] = u0.y;
                 o[4 * m + 3] = u1.y;
+                uv[2 * m] = u0;
+                uv[2 * m + 1] = u1;
               }
             }
             const int head = v / G;
@@ -301,7 +316,7 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
             if constexpr (OUT8) {
               uint32_t w8[2];
               float scale;
-              int8_codes<E, G>(o, acc.x + acc.y, a.inv_hd, a.eps, w8, scale);
+              int8_codes<P, G, !HALF>(uv, acc.x + acc.y, a.inv_hd, a.eps, w8, scale);
               if (ok[k]) {
                 st_stream8(dst, w8[0], w8[1]);
                 if (gl == 0) scale_row[head] = scale;
@@ -427,6 +442,8 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
   bool ok[VPT];
 #pragma unroll
   for (int k = 0; k < VPT; ++k) ok[k] = k * NT + tid < nslots;
+  // output address of slot k: the slot-0 head of this lane plus k * hstep
+  const int64_t hstep = static_cast<int64_t>(NT / G2) * a.out_sh;
 
   // gamma per part and half in rotary layout, as qknorm_rope3d.cuh
   float2 gev[NP][2][Q], god[NP][2][Q];
@@ -575,13 +592,13 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
             }
           }
           unsigned char *obase = static_cast<unsigned char *>(part == 0 ? a.q_out : a.k_out) +
-                                 row_off;
+                                 row_off + static_cast<int64_t>(tid / G2) * a.out_sh;
           float *scale_row = (part == 0 ? a.q_scale : a.k_scale) +
                              grow * static_cast<int64_t>(a.n_heads);
 #pragma unroll
           for (int k = 0; k < VPT; ++k) {
             // every lane joins the shuffles; ok[] only guards memory accesses
-            float o[16];
+            float2 uv[8];  // rotation pairs as produced: (u0, u1) of chunk h, pairs 2m, 2m+1
             float2 acc = splat2(0.f);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -598,18 +615,16 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
               for (int m = 0; m < Q; ++m) {
                 const float2 u0 = fma2(od[m], ns1[h][m], mul2(ev[m], c0[h][m]));
                 const float2 u1 = fma2(od[m], c1[h][m], mul2(ev[m], s0[h][m]));
-                o[8 * h + 4 * m + 0] = u0.x;
-                o[8 * h + 4 * m + 1] = u1.x;
-                o[8 * h + 4 * m + 2] = u0.y;
-                o[8 * h + 4 * m + 3] = u1.y;
+                uv[4 * h + 2 * m] = u0;
+                uv[4 * h + 2 * m + 1] = u1;
               }
             }
             uint32_t w8[4];
             float scale;
-            int8_codes<16, G2>(o, acc.x + acc.y, a.inv_hd, a.eps, w8, scale);
+            int8_codes<8, G2, true>(uv, acc.x + acc.y, a.inv_hd, a.eps, w8, scale);
             if (ok[k]) {
               const int head = (k * NT + tid) / G2;
-              unsigned char *dst = obase + static_cast<int64_t>(head) * a.out_sh;
+              unsigned char *dst = obase + k * hstep;
               st_stream8(dst + g * 8, w8[0], w8[1]);
               st_stream8(dst + (g + G2) * 8, w8[2], w8[3]);
               if (g == 0) scale_row[head] = scale;
