@@ -265,10 +265,12 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
             const int v = k * NT + tid;
             uint4 xv = make_uint4(0u, 0u, 0u, 0u);
             if (ok[k]) xv = *slot(cons, q, part, k);
-            // rotated outputs in element order, not yet multiplied by the
-            // head's 1/rms; acc: this thread's part of the sum of squares
-            float o[E];
-            float2 uv[P];  // the same values as pairs, for int8_codes
+            // rotated outputs, not yet multiplied by the head's 1/rms, as the
+            // rotation leaves them in registers: half-split, uv[m] = elements
+            // (2m, 2m+1); interleaved, uv[2m] / uv[2m+1] = first / second
+            // components of pairs 2m and 2m+1.  acc: this thread's part of
+            // the sum of squares
+            float2 uv[P];
             float2 acc;
             if constexpr (HALF) {
               uint4 pv;
@@ -284,10 +286,7 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
               for (int m = 1; m < P; ++m) acc = fma2(own[m], own[m], acc);
 #pragma unroll
               for (int m = 0; m < P; ++m) {
-                const float2 u = fma2(own[m], ca[m], mul2(par[m], sb[m]));
-                o[2 * m] = u.x;
-                o[2 * m + 1] = u.y;
-                uv[m] = u;
+                uv[m] = fma2(own[m], ca[m], mul2(par[m], sb[m]));
               }
             } else {
               float2 ev[Q], od[Q];
@@ -301,14 +300,8 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
               }
 #pragma unroll
               for (int m = 0; m < Q; ++m) {
-                const float2 u0 = fma2(od[m], ns1[m], mul2(ev[m], c0[m]));
-                const float2 u1 = fma2(od[m], c1[m], mul2(ev[m], s0[m]));
-                o[4 * m + 0] = u0.x;
-                o[4 * m + 1] = u1.x;
-                o[4 * m + 2] = u0.y;
-                o[4 * m + 3] = u1.y;
-                uv[2 * m] = u0;
-                uv[2 * m + 1] = u1;
+                uv[2 * m] = fma2(od[m], ns1[m], mul2(ev[m], c0[m]));
+                uv[2 * m + 1] = fma2(od[m], c1[m], mul2(ev[m], s0[m]));
               }
             }
             const int head = v / G;
@@ -325,12 +318,19 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
               const float2 inv2 = splat2(rsqrtf(fmaf(group_sum<G>(acc.x + acc.y), a.inv_hd, a.eps)));
               float2 pr[P];
 #pragma unroll
-              for (int m = 0; m < P; ++m) pr[m] = mul2(make_float2(o[2 * m], o[2 * m + 1]), inv2);
+              for (int m = 0; m < P; ++m) pr[m] = mul2(uv[m], inv2);
               // a plain (evict-normal) store: in head-strided layouts such as
               // [B, H, L, hd] consecutive rows of a head are adjacent, and L2
               // can merge a CTA's successive rows before writing back (4%
               // faster there than evict-first; the same in [B, L, H, hd])
-              if (ok[k]) *reinterpret_cast<uint4 *>(dst) = IO::pack(pr);
+              if (ok[k]) {
+                if constexpr (HALF) {
+                  *reinterpret_cast<uint4 *>(dst) = IO::pack(pr);
+                } else {
+                  const float2 f0[Q] = {pr[0], pr[2]}, f1[Q] = {pr[1], pr[3]};
+                  *reinterpret_cast<uint4 *>(dst) = IO::pack_eo(f0, f1);
+                }
+              }
             }
           }
         }
