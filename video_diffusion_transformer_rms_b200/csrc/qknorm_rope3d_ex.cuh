@@ -743,18 +743,18 @@ cudaError_t dispatch_ex_tab_interleaved(const QkArgs &a, int threads, int vpt,
 // contiguous share of rows per CTA in both forms (chunks measured no gain),
 // split by pick_split_i8w, q and k on paired CTAs (half the ring and gamma
 // registers per CTA: table form 0.800 -> 0.739 ms, on the fly 0.699 ->
-// 0.688 ms in one session).  The table form caps registers at 128 (512
-// threads' worth of CTAs per SM) and stages each row's table entries per
-// warp, which drops the CTA barrier from its loop: 0.781 -> 0.706 ms in one
-// interleaved session at the 5 s clip (the on-the-fly form 0.713 ms there;
-// staging per CTA behind a barrier, or lanes reading the table themselves,
+// 0.688 ms in one session).  Both forms cap registers at 128 (512 threads'
+// worth of CTAs per SM: on the fly 0.707 -> 0.690 ms).  The table form
+// stages each row's table entries per warp, which drops the CTA barrier from
+// its loop: 0.781 -> 0.706 ms in one interleaved session at the 5 s clip
+// (staging per CTA behind a barrier, or lanes reading the table themselves,
 // were the slower alternatives).
 template <int G2, bool TAB>
 cudaError_t dispatch_i8w(const QkArgs &a, int threads, int vpt, cudaStream_t stream,
                          Geometry *geo) {
 #define SOL_CASE(NT, V)                                                                           \
   if (threads == NT && vpt == V)                                                                  \
-    return launch_int8w_cfg<G2, NT, V, 1, 2, TAB, 0, (TAB ? 512 / NT : 1), true>(a, stream, geo);
+    return launch_int8w_cfg<G2, NT, V, 1, 2, TAB, 0, 512 / NT, true>(a, stream, geo);
   SOL_I8W_SPLITS(SOL_CASE)
 #undef SOL_CASE
   return cudaErrorInvalidValue;
