@@ -410,7 +410,7 @@ __host__ __device__ constexpr size_t i8w_head_bytes() {
 // (stage_table_lanes) and has no CTA barrier in its loop; the on-the-fly form
 // builds CTA-wide angle tables behind one barrier per stage.
 template <int G2, int NT, int VPT, int R, int S, bool TAB, int K = 0, int MINB = 1,
-          bool PSPLIT = true>
+          bool PSPLIT = true, bool FULL = false>
 __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkArgs a) {
   static_assert(K % R == 0, "a ring stage's rows must lie in one chunk");
   static_assert(NT % 32 == 0 && 32 % G2 == 0, "a head's lanes must share a warp");
@@ -439,9 +439,11 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
   p0[0] = P * g;
   p0[1] = P * (g + G2);
 
+  // FULL: the split covers a part's slots exactly (NT * VPT == nslots), so
+  // every slot is real and no access needs a guard
   bool ok[VPT];
 #pragma unroll
-  for (int k = 0; k < VPT; ++k) ok[k] = k * NT + tid < nslots;
+  for (int k = 0; k < VPT; ++k) ok[k] = FULL || k * NT + tid < nslots;
   // output address of slot k: the slot-0 head of this lane plus k * hstep
   const int64_t hstep = static_cast<int64_t>(NT / G2) * a.out_sh;
 
@@ -642,10 +644,11 @@ __global__ void __launch_bounds__(NT, MINB) qknorm_rope3d_int8w_kernel(const QkA
 }
 
 template <int G2, int NT, int VPT, int R, int S, bool TAB, int K = 0, int MINB = 1,
-          bool PSPLIT = true>
+          bool PSPLIT = true, bool FULL = false>
 cudaError_t launch_int8w_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
+  if (FULL && a.nvec_q / 2 != NT * VPT) return cudaErrorInvalidValue;
   const void *fn = reinterpret_cast<const void *>(
-      &qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, MINB, PSPLIT>);
+      &qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, MINB, PSPLIT, FULL>);
   constexpr int NP = PSPLIT ? 1 : 2;
   const size_t smem =
       i8w_head_bytes<R, S, TAB, NT>() + static_cast<size_t>(S) * R * NP * VPT * 2 * NT * 16;
@@ -660,7 +663,7 @@ cudaError_t launch_int8w_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo
     grid = a.rows;
   }
   if (geo) *geo = Geometry{NT, VPT, S, smem, static_cast<int>(grid)};
-  qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, MINB, PSPLIT>
+  qknorm_rope3d_int8w_kernel<G2, NT, VPT, R, S, TAB, K, MINB, PSPLIT, FULL>
       <<<static_cast<unsigned>(grid), NT, smem, stream>>>(a);
   return cudaGetLastError();
 }
@@ -687,22 +690,25 @@ cudaError_t launch_ex_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
 // B200; the split is kRowSplit's for both forms):
 //  - on the fly: one row per ring stage for INT8 and half-split bf16 (half
 //    the ring, more CTAs per SM; INT8 0.90 against 1.04 ms), two for
-//    interleaved bf16; rows in round-robin chunks of kOtfChunk for bf16
-//    output (0.916 against 0.925 ms in [B, H, L, hd], 0.909 against 0.929
-//    half-split), a contiguous share per CTA for INT8, which is bound by
-//    instruction issue rather than DRAM and gained nothing from chunks
-//    (0.84 against 0.80 ms);
+//    interleaved bf16; rows in round-robin chunks of kExOtfChunk for bf16
+//    output (32 rows: each CTA writes longer runs of a head's rows in
+//    [B, H, L, hd], 0.922 -> 0.872 ms against chunks of 8, which had beaten
+//    contiguous shares; half-split the same for 8 to 32), a contiguous share
+//    per CTA for INT8, which is bound by instruction issue rather than DRAM
+//    and gained nothing from chunks (0.84 against 0.80 ms);
 //  - table-driven: one row per stage, two stages, chunks of kTabChunk and
 //    a barrier per stage, each thread reading its table entries: 0.809 ms
 //    half-split (6.4 TB/s).  (Interleaved bf16 from the table takes
 //    dispatch_ex_tab_interleaved, interleaved INT8 dispatch_i8w.)
+constexpr int kExOtfChunk = 32;
+
 template <int G, int NT, int VPT, bool HALF, bool OUT8, bool TAB>
 cudaError_t launch_ex(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
   if constexpr (TAB) {
     return launch_ex_cfg<G, NT, VPT, 1, 2, HALF, OUT8, true, kTabChunk, true>(a, stream, geo);
   } else {
     constexpr int R = (OUT8 || HALF) ? 1 : (VPT <= 6 ? 2 : 1);
-    constexpr int K = OUT8 ? 0 : kOtfChunk;
+    constexpr int K = OUT8 ? 0 : kExOtfChunk;
     return launch_ex_cfg<G, NT, VPT, R, 2, HALF, OUT8, false, K, false>(a, stream, geo);
   }
 }
@@ -748,13 +754,18 @@ cudaError_t dispatch_ex_tab_interleaved(const QkArgs &a, int threads, int vpt,
 // stages each row's table entries per warp, which drops the CTA barrier from
 // its loop: 0.781 -> 0.706 ms in one interleaved session at the 5 s clip
 // (staging per CTA behind a barrier, or lanes reading the table themselves,
-// were the slower alternatives).
+// were the slower alternatives).  A split that covers a part's slots
+// exactly (64 x 5 at D = 5120) takes the unguarded instantiation (FULL):
+// 0.708 -> 0.661 ms with the table, 0.704 -> 0.648 ms on the fly, in one
+// session.
 template <int G2, bool TAB>
 cudaError_t dispatch_i8w(const QkArgs &a, int threads, int vpt, cudaStream_t stream,
                          Geometry *geo) {
-#define SOL_CASE(NT, V)                                                                           \
-  if (threads == NT && vpt == V)                                                                  \
-    return launch_int8w_cfg<G2, NT, V, 1, 2, TAB, 0, 512 / NT, true>(a, stream, geo);
+#define SOL_CASE(NT, V)                                                                     \
+  if (threads == NT && vpt == V)                                                            \
+    return a.nvec_q / 2 == NT * V                                                           \
+               ? launch_int8w_cfg<G2, NT, V, 1, 2, TAB, 0, 512 / NT, true, true>(a, stream, geo) \
+               : launch_int8w_cfg<G2, NT, V, 1, 2, TAB, 0, 512 / NT, true, false>(a, stream, geo);
   SOL_I8W_SPLITS(SOL_CASE)
 #undef SOL_CASE
   return cudaErrorInvalidValue;
