@@ -79,7 +79,7 @@ __device__ __forceinline__ void int8_codes(float2 (&v)[NV], float ssq, float inv
 }
 
 template <int G, int NT, int VPT, int R, int S, bool HALF, bool OUT8, bool TAB, int K = 0,
-          bool BAR = false, bool STAGE = false>
+          bool BAR = false, bool STAGE = false, bool FULL = false>
 __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
   static_assert(K % R == 0, "a ring stage's rows must lie in one chunk");
   using IO = Io<__nv_bfloat16>;
@@ -108,9 +108,11 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
   const int p0 = HALF ? (gl % (G / 2)) * E : gl * (E / 2);
   const int64_t part_bytes = static_cast<int64_t>(a.nvec_q) * 16;
 
+  // FULL: the split covers a part's vectors exactly (NT * VPT == nvec_q),
+  // so no access needs a guard
   bool ok[VPT];
 #pragma unroll
-  for (int k = 0; k < VPT; ++k) ok[k] = k * NT + tid < a.nvec_q;
+  for (int k = 0; k < VPT; ++k) ok[k] = FULL || k * NT + tid < a.nvec_q;
 
   // gamma: interleaved as in qknorm_rope3d.cuh; half-split as own / partner
   // elements in natural pairs
@@ -670,10 +672,11 @@ cudaError_t launch_int8w_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo
 
 // One launch of a fixed configuration: a wave of as many CTAs as fit.
 template <int G, int NT, int VPT, int R, int S, bool HALF, bool OUT8, bool TAB, int K = 0,
-          bool BAR = false, bool STAGE = false>
+          bool BAR = false, bool STAGE = false, bool FULL = false>
 cudaError_t launch_ex_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
+  if (FULL && a.nvec_q != NT * VPT) return cudaErrorInvalidValue;
   const void *fn = reinterpret_cast<const void *>(
-      &qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8, TAB, K, BAR, STAGE>);
+      &qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8, TAB, K, BAR, STAGE, FULL>);
   const size_t smem =
       head_bytes<R, S, TAB, STAGE>() + static_cast<size_t>(S) * R * 2 * VPT * NT * 16;
   const int per_sm = resident_blocks(fn, NT, smem);
@@ -681,7 +684,7 @@ cudaError_t launch_ex_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
   int64_t grid = static_cast<int64_t>(per_sm) * device_sms();
   if (grid > a.rows) grid = a.rows;
   if (geo) *geo = Geometry{NT, VPT, S, smem, static_cast<int>(grid)};
-  qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8, TAB, K, BAR, STAGE>
+  qknorm_rope3d_ex_kernel<G, NT, VPT, R, S, HALF, OUT8, TAB, K, BAR, STAGE, FULL>
       <<<static_cast<unsigned>(grid), NT, smem, stream>>>(a);
   return cudaGetLastError();
 }
@@ -700,12 +703,21 @@ cudaError_t launch_ex_cfg(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
 //    a barrier per stage, each thread reading its table entries: 0.809 ms
 //    half-split (6.4 TB/s).  (Interleaved bf16 from the table takes
 //    dispatch_ex_tab_interleaved, interleaved INT8 dispatch_i8w.)
+//  - a table-form split that covers a part's vectors exactly (FULL, 128 x 5
+//    and 320 x 2 at D = 5120) drops the guards: half-split 0.863 -> 0.812
+//    ms, [B, H, L, hd] 0.862 -> 0.836 ms in one session; the on-the-fly
+//    half-split measured 2% slower unguarded and keeps its guards.
 constexpr int kExOtfChunk = 32;
 
 template <int G, int NT, int VPT, bool HALF, bool OUT8, bool TAB>
 cudaError_t launch_ex(const QkArgs &a, cudaStream_t stream, Geometry *geo) {
   if constexpr (TAB) {
-    return launch_ex_cfg<G, NT, VPT, 1, 2, HALF, OUT8, true, kTabChunk, true>(a, stream, geo);
+    // a split with no slot past the row's end takes the unguarded kernel
+    return a.nvec_q == NT * VPT
+               ? launch_ex_cfg<G, NT, VPT, 1, 2, HALF, OUT8, true, kTabChunk, true, false, true>(
+                     a, stream, geo)
+               : launch_ex_cfg<G, NT, VPT, 1, 2, HALF, OUT8, true, kTabChunk, true, false, false>(
+                     a, stream, geo);
   } else {
     constexpr int R = (OUT8 || HALF) ? 1 : (VPT <= 6 ? 2 : 1);
     constexpr int K = OUT8 ? 0 : kExOtfChunk;
@@ -735,10 +747,13 @@ cudaError_t dispatch_ex(const QkArgs &a, int threads, int vpt, cudaStream_t stre
 template <int G>
 cudaError_t dispatch_ex_tab_interleaved(const QkArgs &a, int threads, int vpt,
                                         cudaStream_t stream, Geometry *geo) {
-#define SOL_CASE(NT, V)                                                                        \
-  if (threads == NT && vpt == V)                                                               \
-    return launch_ex_cfg<G, NT, V, 1, 2, false, false, true, kTabChunk, true, true>(a, stream, \
-                                                                                    geo);
+#define SOL_CASE(NT, V)                                                                       \
+  if (threads == NT && vpt == V)                                                              \
+    return a.nvec_q == NT * V                                                                 \
+               ? launch_ex_cfg<G, NT, V, 1, 2, false, false, true, kTabChunk, true, true, true>( \
+                     a, stream, geo)                                                          \
+               : launch_ex_cfg<G, NT, V, 1, 2, false, false, true, kTabChunk, true, true,       \
+                               false>(a, stream, geo);
   SOL_QK_TAB_SPLITS(SOL_CASE)
 #undef SOL_CASE
   return cudaErrorInvalidValue;

@@ -66,7 +66,7 @@ __device__ __forceinline__ void load_modulation(const RmsArgs &a, int key, int t
   }
 }
 
-template <typename T, int NT, int VPT, int R, int S, bool RESID, int K = 0>
+template <typename T, int NT, int VPT, int R, int S, bool RESID, int K = 0, bool FULL = false>
 __global__ void __launch_bounds__(NT) rms_adaln_kernel(const RmsArgs a) {
   static_assert(K % R == 0, "an iteration's rows must lie in one chunk");
   using IO = Io<T>;
@@ -82,9 +82,11 @@ __global__ void __launch_bounds__(NT) rms_adaln_kernel(const RmsArgs a) {
   const int warp = tid >> 5;
   const int64_t row_bytes = static_cast<int64_t>(a.nvec) * 16;
 
-  bool ok[VPT];  // slot k holds vector k*NT + tid of the row
+  // slot k holds vector k*NT + tid of the row; FULL: the split covers the
+  // row exactly, no access needs a guard
+  bool ok[VPT];
 #pragma unroll
-  for (int k = 0; k < VPT; ++k) ok[k] = k * NT + tid < a.nvec;
+  for (int k = 0; k < VPT; ++k) ok[k] = FULL || k * NT + tid < a.nvec;
 
   for (int i = tid; i < 2 * R * 32; i += NT) red[i] = 0.f;  // unused warp slots read 0
   __syncthreads();
@@ -251,28 +253,35 @@ constexpr int kRows = VPT <= (RESID ? 3 : 5) ? 2 : 1;
 // bit-identical), 0.820 against 0.839 ms with the residual.
 constexpr int kRmsChunk = 8;
 
-template <typename T, int NT, int VPT, bool RESID, int R = kRows<VPT, RESID>, int S = 2,
-          int K = kRmsChunk>
+template <typename T, int NT, int VPT, bool RESID, bool FULL, int R = kRows<VPT, RESID>,
+          int S = 2, int K = kRmsChunk>
 cudaError_t launch_t(const RmsArgs &a, cudaStream_t stream, Geometry *geo) {
   constexpr int NIN = RESID ? 2 : 1;
+  if (FULL && a.nvec != NT * VPT) return cudaErrorInvalidValue;
   const void *fn =
-      reinterpret_cast<const void *>(&rms_adaln_kernel<T, NT, VPT, R, S, RESID, K>);
+      reinterpret_cast<const void *>(&rms_adaln_kernel<T, NT, VPT, R, S, RESID, K, FULL>);
   const size_t smem = 2 * R * 32 * 4 + static_cast<size_t>(S) * R * NIN * VPT * NT * 16;
   const int per_sm = resident_blocks(fn, NT, smem);
   if (per_sm <= 0) return cudaErrorInvalidConfiguration;
   int64_t grid = static_cast<int64_t>(per_sm) * device_sms();
   if (grid > a.rows) grid = a.rows;
   if (geo) *geo = Geometry{NT, VPT, S, smem, static_cast<int>(grid)};
-  rms_adaln_kernel<T, NT, VPT, R, S, RESID, K>
+  rms_adaln_kernel<T, NT, VPT, R, S, RESID, K, FULL>
       <<<static_cast<unsigned>(grid), NT, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
+// A split that covers the row exactly (128 x 5 at D = 5120) takes the
+// unguarded instantiation (FULL): RMS-AdaLN 0.417 -> 0.407 ms at the 5 s
+// clip in one interleaved session, bit-identical; the residual form is the
+// same either way.
 template <typename T, bool RESID>
 cudaError_t dispatch(const RmsArgs &a, int threads, int vpt, cudaStream_t stream,
                      Geometry *geo) {
-#define SOL_CASE(NT, V) \
-  if (threads == NT && vpt == V) return launch_t<T, NT, V, RESID>(a, stream, geo);
+#define SOL_CASE(NT, V)                                                         \
+  if (threads == NT && vpt == V)                                                \
+    return a.nvec == NT * V ? launch_t<T, NT, V, RESID, true>(a, stream, geo)   \
+                            : launch_t<T, NT, V, RESID, false>(a, stream, geo);
   SOL_SPLITS(SOL_CASE)
 #undef SOL_CASE
   return cudaErrorInvalidValue;
