@@ -271,17 +271,21 @@ cudaError_t launch_t(const RmsArgs &a, cudaStream_t stream, Geometry *geo) {
   return cudaGetLastError();
 }
 
-// A split that covers the row exactly (128 x 5 at D = 5120) takes the
-// unguarded instantiation (FULL): RMS-AdaLN 0.417 -> 0.407 ms at the 5 s
-// clip in one interleaved session, bit-identical; the residual form is the
-// same either way.
+// A short launch whose split covers the row exactly (128 x 5 at D = 5120)
+// takes the unguarded instantiation (FULL): at 8,264 rows it streams 5.5
+// instead of 4.35 TB/s.  Longer launches keep the guards, which measured
+// 3-4% faster there (126,552 and 371,592 rows, two boxes, four bench runs
+// each way); the results are bit-identical either way.
+constexpr int64_t kFullMaxRows = 16384;
+
 template <typename T, bool RESID>
 cudaError_t dispatch(const RmsArgs &a, int threads, int vpt, cudaStream_t stream,
                      Geometry *geo) {
-#define SOL_CASE(NT, V)                                                         \
-  if (threads == NT && vpt == V)                                                \
-    return a.nvec == NT * V ? launch_t<T, NT, V, RESID, true>(a, stream, geo)   \
-                            : launch_t<T, NT, V, RESID, false>(a, stream, geo);
+#define SOL_CASE(NT, V)                                                       \
+  if (threads == NT && vpt == V)                                              \
+    return a.nvec == NT * V && a.rows <= kFullMaxRows                         \
+               ? launch_t<T, NT, V, RESID, true>(a, stream, geo)              \
+               : launch_t<T, NT, V, RESID, false>(a, stream, geo);
   SOL_SPLITS(SOL_CASE)
 #undef SOL_CASE
   return cudaErrorInvalidValue;
