@@ -968,3 +968,25 @@ def test_row_order_regimes(rows):
     torch.cuda.synchronize()
     assert torch.equal(y2, y)
     assert torch.equal(o2, out)
+
+
+def test_rms_adaln_guarded_and_unguarded_agree():
+    # At D = 5120 the 128 x 5 split covers a row exactly; launches of up to
+    # 16,384 rows take the kernel without per-slot bounds checks, longer ones
+    # the guarded kernel.  16,385 rows (guarded) and their first 16,384 rows
+    # alone (unguarded) must give the same bits on those rows, and both
+    # must match the oracle on sampled rows.
+    D, rows = 5120, 16385
+    nv = rows - 201
+    x = activation(rows, D, torch.bfloat16, DEV, 211, outliers=True)
+    sc = vectors((1, 2, D), 0.0, 0.5, torch.bfloat16, DEV, 212)
+    sh = vectors((1, 2, D), 0.0, 0.5, torch.bfloat16, DEV, 213)
+    y_long = api.rms_adaln(x.view(1, rows, D), sc, sh, nv)
+    y_short = api.rms_adaln(x[:rows - 1].view(1, rows - 1, D), sc, sh, nv)
+    torch.cuda.synchronize()
+    assert torch.equal(y_short.view(rows - 1, D), y_long.view(rows, D)[:rows - 1])
+    ids = sample_rows(rows, rows, nv, 1, 256, seed=214)
+    ids = np.unique(np.concatenate([ids, [0, rows - 1, nv - 1, nv]]))
+    assert_close(take_rows_gpu(y_long.view(rows, D), ids),
+                 oracle.rms_adaln(take_rows(x, ids), _o(sc), _o(sh), rows, nv, 1e-6,
+                                  row_ids=ids), "rms guarded")
