@@ -349,7 +349,8 @@ __global__ void __launch_bounds__(NT) qknorm_rope3d_ex_kernel(const QkArgs a) {
 // The CTA split each variant of qknorm_rope3d_ex_kernel takes, measured
 // inside a step at the 5 s clip: the row-reduction rule (pick_split, <= 6
 // vectors per thread: 128 x 5 at D = 5120, which divides the row exactly)
-// for half-split bf16 (0.92 against 0.97 ms); the QK rule (pick_split_qk:
+// for half-split bf16 from the table (0.92 against 0.97 ms; on the fly it
+// takes dispatch_ex_half_otf); the QK rule (pick_split_qk:
 // 256 x 3, more warps, a sixth of the vector slots empty) for interleaved
 // bf16 and half-split INT8.  (Interleaved INT8 runs in
 // qknorm_rope3d_int8w_kernel, split by pick_split_i8w.)
@@ -759,6 +760,20 @@ cudaError_t dispatch_ex_tab_interleaved(const QkArgs &a, int threads, int vpt,
   return cudaErrorInvalidValue;
 }
 
+// Half-split bf16 on the fly: the on-the-fly QK split (pick_split_otf, 160 x
+// 4 at D = 5120, one row per stage): 0.906 -> 0.876 ms at the 5 s clip in
+// one interleaved session against the row-reduction split (128 x 5); for
+// [B, H, L, hd] interleaved output 160 x 4 was 8% slower than 256 x 3.
+template <int G>
+cudaError_t dispatch_ex_half_otf(const QkArgs &a, int threads, int vpt, cudaStream_t stream,
+                                 Geometry *geo) {
+#define SOL_CASE(NT, V) \
+  if (threads == NT && vpt == V) return launch_ex<G, NT, V, true, false, false>(a, stream, geo);
+  SOL_QK_OTF_SPLITS(SOL_CASE)
+#undef SOL_CASE
+  return cudaErrorInvalidValue;
+}
+
 // Interleaved INT8 with 16 elements per lane (qknorm_rope3d_int8w_kernel),
 // G2 = head_dim / 16 lanes per head: one row per stage, two stages and a
 // contiguous share of rows per CTA in both forms (chunks measured no gain),
@@ -812,6 +827,17 @@ cudaError_t launch_ex_form(const QkArgs &a, bool half, cudaStream_t stream, Geom
         case 8: return dispatch_ex_tab_interleaved<8>(a, threads, vpt, stream, geo);
         case 16: return dispatch_ex_tab_interleaved<16>(a, threads, vpt, stream, geo);
         case 32: return dispatch_ex_tab_interleaved<32>(a, threads, vpt, stream, geo);
+        default: return cudaErrorInvalidValue;
+      }
+    }
+  }
+  if constexpr (!TAB && !OUT8) {
+    if (half) {  // half-split bf16 on the fly: the on-the-fly QK split
+      if (!pick_split_otf(a.nvec_q, &threads, &vpt)) return cudaErrorInvalidValue;
+      switch (G) {
+        case 8: return dispatch_ex_half_otf<8>(a, threads, vpt, stream, geo);
+        case 16: return dispatch_ex_half_otf<16>(a, threads, vpt, stream, geo);
+        case 32: return dispatch_ex_half_otf<32>(a, threads, vpt, stream, geo);
         default: return cudaErrorInvalidValue;
       }
     }
