@@ -50,6 +50,7 @@ TRAFFIC_NAME = {"rms_adaln": "rms_adaln", "gate_residual": "gate_residual",
 # every config of the task, each step kernel timed on its own (clip5s is the
 # headline step above)
 PER_CONFIG = ("clip5s", "clip15s", "cfg5s", "cfg5s_d3072", "medium")
+COOL_DOWN_S = 2.0  # idle seconds before the per-config block (outside every timed region)
 L2_FLUSH_BYTES = 256 << 20   # written between reps where the inputs fit in L2
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
@@ -457,8 +458,12 @@ def run_ours(args):
     del ws, q8, s8, v8, vs8
 
     # ---- every config: each step kernel on its own (before the GEMM: it runs
-    # at the power cap, and the kernels right after it ran slow) -----------
+    # at the power cap, and the kernels right after it ran slow).  An idle
+    # pause first: the next rows' 200-launch loops leave the GPU at its power
+    # cap, and the first config timed right after them dipped in some runs.
     peak, peak_kind = load_peak()
+    torch.cuda.synchronize()
+    time.sleep(COOL_DOWN_S)
     configs = {c: time_config(WORKLOADS[c], dev, stream, peak) for c in PER_CONFIG}
 
     next_rows["gemm_gelu"] = time_gemm_gelu(w, D, dev, stream)
